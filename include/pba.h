@@ -1,0 +1,132 @@
+/*
+ * libpba: pair-biased gated attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the attention of AlphaFold3-style models as described on the
+ * "AlphaFold3 open-source implementation" page (Ligo Biosciences README), section
+ * "Model Efficiency": a pair bias, projected from the pair representation, is added
+ * after the key-query dot product; the bias is broadcast over a batch-like axis (the
+ * rows of a triangle attention, the sequences of an MSA, or the 48 noise-level copies
+ * of the diffusion module, which that section folds into the batch dimension), so its
+ * gradient is the gradient of the scaled logits summed over that axis.  With the
+ * sigmoid gate, for every broadcast row b, head h and query i:
+ *
+ *   s[b,h,i,j] = scale * <q[b,i,h,:], k[b,j,h,:]> + bias[h,i,j]   (masked keys: -inf)
+ *   out[b,i,h,:] = sigmoid(gate[b,i,h,:]) * sum_j softmax_j(s[b,h,i,:]) v[b,j,h,:]
+ *   lse[b,h,i]   = ln sum_j exp(s[b,h,i,j])
+ *
+ * and the backward pass returns dq, dk, dv, dgate and dbias[h,i,j] = sum_b dS[b,h,i,j].
+ * A query row whose keys are all masked gets out = 0, lse = -inf and no gradient.
+ *
+ * Conventions for every entry point:
+ *  - Element types: q, k, v, gate, out, dout, dq, dk, dv, dgate and bias are bf16 (passed
+ *    as uint16_t bit patterns); lse and dbias are fp32; key_mask is uint8 (nonzero = the
+ *    key is attended, 0 = masked).  Arithmetic is bf16 x bf16 -> fp32 on the tensor
+ *    cores, fp32 elsewhere.
+ *  - All pointers are DEVICE pointers, owned by the caller; the library keeps none of
+ *    them after a call returns and allocates nothing per call.  Outputs are written in
+ *    full (never accumulated into).
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are detected on the host and returned before
+ *    anything is launched.
+ *  - Every wait inside the kernels is bounded (about one second).  A wait that runs out
+ *    makes the kernel stop early and record a device error word; pba_device_status()
+ *    reports it as PBA_ERR_TIMEOUT.
+ */
+#ifndef PBA_H
+#define PBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PBA_VERSION 1
+
+typedef uint16_t pba_bf16; /* bf16 bit pattern */
+
+typedef enum {
+    PBA_OK = 0,
+    PBA_ERR_INVALID_ARG = 1,  /* null required pointer, negative size, bad stride/alignment */
+    PBA_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement (e.g. C>64) */
+    PBA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (see pba_last_error) */
+    PBA_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait ran out (device watchdog) */
+    PBA_ERR_WORKSPACE = 5     /* workspace too small */
+} pba_status;
+
+/*
+ * Problem sizes and layouts.
+ *  q, gate, out, dout, dq, dgate : [B, Nq, H, C]      k, v, dk, dv : [B, Nk, H, C]
+ *  The channel (C) stride is 1; s?[0], s?[1], s?[2] are the element strides of the
+ *  B, N and H dimensions (so = out and dout, sq = q and dq, sk = k and dk, sv = v and
+ *  dv, sg = gate and dgate).  Every such stride must be a multiple of 8 elements and
+ *  every base pointer 16-byte aligned (the tiles are moved by the Tensor Memory
+ *  Accelerator), C a multiple of 8 in [8, 64].
+ *  bias : [H, Nq, Nk], key stride 1; sbias[0], sbias[1] = element strides of H and Nq
+ *         (multiples of 8).
+ *  key_mask : [B, Nk] uint8, key stride 1, row stride smask_b (0 = one row for all b).
+ *  lse : [B, H, Nq] fp32, contiguous.      dbias : [H, Nq, Nk] fp32, contiguous.
+ *  scale : multiplier of <q,k>; 0 selects 1/sqrt(C) (the true C, not a padded one).
+ */
+typedef struct {
+    int32_t B, H, Nq, Nk, C;
+    float scale;
+    int64_t sq[3], sk[3], sv[3], sg[3], so[3];
+    int64_t sbias[2];
+    int64_t smask_b;
+} pba_dims;
+
+/* Fill `d` with dense strides for the layouts above (mask shared by all b). */
+void pba_dims_dense(pba_dims *d, int32_t B, int32_t H, int32_t Nq, int32_t Nk, int32_t C,
+                    float scale);
+
+/*
+ * Forward pass (the operator stated in the header comment).
+ *  bias may be NULL (no pair bias), key_mask may be NULL (every key attended), gate
+ *  may be NULL (no gate: out = softmax(s) v).  out and lse are required.
+ * Returns PBA_OK once the kernel is queued on `stream`.
+ */
+pba_status pba_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                   const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                   pba_bf16 *out, float *lse, const pba_dims *dims, void *stream);
+
+/* Bytes of device workspace pba_bwd needs for these dims (0 for an empty problem). */
+size_t pba_bwd_workspace_size(const pba_dims *dims);
+
+/*
+ * Backward pass: given the forward inputs, the forward outputs (out, lse) and dout,
+ * writes dq, dk, dv (required), dgate (required iff gate is not NULL, else ignored)
+ * and dbias (may be NULL to skip it; computed even when bias is NULL, as the gradient
+ * with respect to a zero bias).  dbias is the sum over the B broadcast rows of the
+ * logits' gradient, reduced in a fixed order, so it is bit-identical from run to run.
+ * workspace: caller-owned device memory of at least pba_bwd_workspace_size(dims) bytes,
+ * 256-byte aligned; its contents on entry do not matter and on return are undefined.
+ */
+pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                   const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                   const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                   pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                   void *workspace, size_t workspace_bytes, const pba_dims *dims,
+                   void *stream);
+
+/*
+ * Synchronizes `stream`, then reports and clears the device watchdog word of the
+ * current device: PBA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
+ * since the last call, PBA_ERR_CUDA if the synchronization itself failed, else PBA_OK.
+ */
+pba_status pba_device_status(void *stream);
+
+/* Static description of a status code. */
+const char *pba_status_string(pba_status s);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char *pba_last_error(void);
+
+int pba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PBA_H */

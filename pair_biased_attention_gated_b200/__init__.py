@@ -1,0 +1,178 @@
+"""Python binding of libpba (pair-biased gated attention for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+`libpba.so`, reached through its C ABI (`include/pba.h`).  PyTorch provides device memory
+and streams.  There is no fallback: if the library is missing this import fails.
+
+Tensor layouts (bf16 unless noted): q, gate, out, dout [B, Nq, H, C]; k, v [B, Nk, H, C];
+bias [H, Nq, Nk]; key_mask uint8/bool [Nk] (shared by all B) or [B, Nk] (1 = attended);
+lse fp32 [B, H, Nq]; dbias fp32 [H, Nq, Nk].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpba.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libpba.so is not built; run `python pair_biased_attention_gated_b200/build.py` "
+        "(there is no non-CUDA implementation of this package)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+PBA_OK = 0
+STATUS = {0: "PBA_OK", 1: "PBA_ERR_INVALID_ARG", 2: "PBA_ERR_UNSUPPORTED", 3: "PBA_ERR_CUDA",
+          4: "PBA_ERR_TIMEOUT", 5: "PBA_ERR_WORKSPACE"}
+
+
+class PbaDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Nq", ctypes.c_int32),
+                ("Nk", ctypes.c_int32), ("C", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("sq", ctypes.c_int64 * 3), ("sk", ctypes.c_int64 * 3),
+                ("sv", ctypes.c_int64 * 3), ("sg", ctypes.c_int64 * 3),
+                ("so", ctypes.c_int64 * 3), ("sbias", ctypes.c_int64 * 2),
+                ("smask_b", ctypes.c_int64)]
+
+
+_vp = ctypes.c_void_p
+lib.pba_dims_dense.argtypes = [ctypes.POINTER(PbaDims)] + [ctypes.c_int32] * 5 + [ctypes.c_float]
+lib.pba_dims_dense.restype = None
+lib.pba_fwd.argtypes = [_vp] * 8 + [ctypes.POINTER(PbaDims), _vp]
+lib.pba_fwd.restype = ctypes.c_int
+lib.pba_bwd_workspace_size.argtypes = [ctypes.POINTER(PbaDims)]
+lib.pba_bwd_workspace_size.restype = ctypes.c_size_t
+lib.pba_bwd.argtypes = [_vp] * 14 + [_vp, ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
+lib.pba_bwd.restype = ctypes.c_int
+lib.pba_device_status.argtypes = [_vp]
+lib.pba_device_status.restype = ctypes.c_int
+lib.pba_status_string.argtypes = [ctypes.c_int]
+lib.pba_status_string.restype = ctypes.c_char_p
+lib.pba_last_error.argtypes = []
+lib.pba_last_error.restype = ctypes.c_char_p
+lib.pba_version.argtypes = []
+lib.pba_version.restype = ctypes.c_int
+
+
+class PbaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__("%s: %s" % (STATUS.get(status, status), detail))
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status != PBA_OK:
+        raise PbaError(status, lib.pba_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _s3(t):
+    st = t.stride()
+    if st[3] != 1:
+        raise ValueError("the channel (last) dimension must have stride 1")
+    return (ctypes.c_int64 * 3)(st[0], st[1], st[2])
+
+
+def make_dims(q, k, v, gate=None, out=None, bias=None, key_mask=None, scale: float = 0.0,
+              dout=None) -> PbaDims:
+    """pba_dims from tensors: q/gate/out [B,Nq,H,C], k/v [B,Nk,H,C], bias [H,Nq,Nk]."""
+    B, Nq, H, C = q.shape
+    Nk = k.shape[1]
+    d = PbaDims()
+    d.B, d.H, d.Nq, d.Nk, d.C = B, H, Nq, Nk, C
+    d.scale = float(scale or 0.0)
+    d.sq, d.sk, d.sv = _s3(q), _s3(k), _s3(v)
+    d.sg = _s3(gate) if gate is not None else _s3(q)
+    ref_o = out if out is not None else dout
+    d.so = _s3(ref_o) if ref_o is not None else _s3(q)
+    if bias is not None:
+        if bias.stride(2) != 1:
+            raise ValueError("bias key stride must be 1")
+        d.sbias = (ctypes.c_int64 * 2)(bias.stride(0), bias.stride(1))
+    if key_mask is not None:
+        if key_mask.stride(-1) != 1:
+            raise ValueError("key_mask key stride must be 1")
+        d.smask_b = 0 if key_mask.dim() == 1 else key_mask.stride(0)
+    return d
+
+
+def dims_dense(B, H, Nq, Nk, C, scale=0.0) -> PbaDims:
+    d = PbaDims()
+    lib.pba_dims_dense(ctypes.byref(d), B, H, Nq, Nk, C, float(scale))
+    return d
+
+
+def pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale: float = 0.0, stream=None) -> None:
+    """Forward pass into preallocated `out` (bf16, like q) and `lse` (fp32 [B,H,Nq])."""
+    d = make_dims(q, k, v, gate, out, bias, key_mask, scale)
+    _check(lib.pba_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
+                       _ptr(out), _ptr(lse), ctypes.byref(d), _stream(stream)))
+
+
+def pba_bwd_workspace_size(dims: PbaDims) -> int:
+    return int(lib.pba_bwd_workspace_size(ctypes.byref(dims)))
+
+
+def pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
+            workspace, scale: float = 0.0, stream=None) -> None:
+    """Backward pass into preallocated dq, dk, dv (like q/k/v), dbias (fp32 [H,Nq,Nk] or
+    None), dgate (like gate, or None).  `workspace`: a uint8 CUDA tensor of at least
+    pba_bwd_workspace_size(dims) bytes."""
+    d = make_dims(q, k, v, gate, out, bias, key_mask, scale, dout=dout)
+    for name, a, b in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v), ("dgate", dgate, gate),
+                       ("dout", dout, out)):
+        if a is not None and b is not None and a.stride() != b.stride():
+            raise ValueError("%s must have the same strides as its forward tensor" % name)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pba_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
+                       _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                       _ptr(dbias), _ptr(dgate), _ptr(workspace), ws_bytes, ctypes.byref(d),
+                       _stream(stream)))
+
+
+def pba_device_status(stream=None) -> None:
+    """Synchronize the stream and raise if a kernel's bounded wait ran out."""
+    _check(lib.pba_device_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------------------------------
+# allocating conveniences (torch allocates; the library computes)
+# ---------------------------------------------------------------------------------------
+
+def attention_fwd(q, k, v, bias=None, key_mask=None, gate=None, scale: float = 0.0,
+                  stream=None):
+    import torch
+    B, Nq, H, C = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale, stream)
+    return out, lse
+
+
+def attention_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, scale: float = 0.0,
+                  want_dbias: bool = True, stream=None):
+    import torch
+    B, Nq, H, C = q.shape
+    Nk = k.shape[1]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dgate = torch.empty_like(gate) if gate is not None else None
+    dbias = (torch.empty((H, Nq, Nk), dtype=torch.float32, device=q.device)
+             if want_dbias else None)
+    d = make_dims(q, k, v, gate, out, bias, key_mask, scale, dout=dout)
+    ws = torch.empty(max(pba_bwd_workspace_size(d), 1), dtype=torch.uint8, device=q.device)
+    pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, ws,
+            scale, stream)
+    return dq, dk, dv, dgate, dbias

@@ -1,0 +1,289 @@
+// libpba host side: argument validation, TMA tensor maps, launches, the C ABI of pba.h.
+//
+// The library allocates nothing per call.  The CUDA driver's tensor-map encoder is
+// fetched through the runtime's entry-point query on first use, so the shared library
+// itself loads (and its symbols can be inspected) on a machine without a GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/pba.h"
+#include "pba_bwd.cuh"
+#include "pba_fwd.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pba_status fail(pba_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+pba_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(PBA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+pba_status get_encoder() {
+    std::call_once(g_encode_once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        g_encode_err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                        cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return fail(PBA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)",
+                               cudaGetErrorString(g_encode_err));
+    return PBA_OK;
+}
+
+CUtensorMapSwizzle swizzle_for_row_bytes(int rowb) {
+    return rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                       : (rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// A [B, N, H, C] bf16 tensor (C stride 1) as a 4-D map (C, H, N, B), box (CP, 1, 128, 1).
+pba_status map_bnhc(CUtensorMap *m, const void *base, int B, int N, int H, int C,
+                    const int64_t s[3], int CP, const char *name) {
+    cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)(N > 0 ? N : 1),
+                          (cuuint64_t)(B > 0 ? B : 1)};
+    // a dimension of extent 1 is never stepped along: give it a harmless legal stride
+    cuuint64_t strides[3] = {(cuuint64_t)(H > 1 ? s[2] * 2 : 16),
+                             (cuuint64_t)(N > 1 ? s[1] * 2 : 16),
+                             (cuuint64_t)(B > 1 ? s[0] * 2 : 16)};
+    cuuint32_t box[4] = {(cuuint32_t)CP, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle_for_row_bytes(CP * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "tensor map for %s failed (CUresult %d)", name, (int)r);
+    return PBA_OK;
+}
+
+// The [H, Nq, Nk] bias as a 3-D map (Nk, Nq, H), box (64, 128, 1), 128-byte swizzle.
+pba_status map_bias(CUtensorMap *m, const void *base, int H, int Nq, int Nk, const int64_t s[2]) {
+    cuuint64_t dims[3] = {(cuuint64_t)(Nk > 0 ? Nk : 1), (cuuint64_t)(Nq > 0 ? Nq : 1), (cuuint64_t)H};
+    cuuint64_t strides[2] = {(cuuint64_t)(Nq > 1 ? s[1] * 2 : 16), (cuuint64_t)(H > 1 ? s[0] * 2 : 16)};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "tensor map for bias failed (CUresult %d)", (int)r);
+    return PBA_OK;
+}
+
+// ---------------------------------------------------------------------------- validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pba_status check_strides(const int64_t s[3], int B, int N, int H, const char *name) {
+    const int ext[3] = {B, N, H};
+    for (int d = 0; d < 3; ++d) {
+        if (ext[d] <= 1) continue;
+        if (s[d] <= 0 || (s[d] % 8) != 0)
+            return fail(PBA_ERR_INVALID_ARG,
+                        "%s: stride of dim %d is %lld elements; must be a positive multiple of 8",
+                        name, d, (long long)s[d]);
+        if (s[d] * 2 >= (int64_t(1) << 40))
+            return fail(PBA_ERR_UNSUPPORTED, "%s: stride of dim %d too large", name, d);
+    }
+    return PBA_OK;
+}
+
+pba_status check_dims(const pba_dims *d) {
+    if (!d) return fail(PBA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->B < 0 || d->H < 0 || d->Nq < 0 || d->Nk < 0 || d->C < 0)
+        return fail(PBA_ERR_INVALID_ARG, "negative size");
+    if (d->C < 8 || d->C > 64 || (d->C % 8) != 0)
+        return fail(PBA_ERR_UNSUPPORTED, "C=%d: head dim must be a multiple of 8 in [8, 64]", d->C);
+    if (d->H < 1) return fail(PBA_ERR_INVALID_ARG, "H must be >= 1");
+    if (d->Nq > (1 << 24) || d->Nk > (1 << 24) || d->B > (1 << 24) || d->H > 4096)
+        return fail(PBA_ERR_UNSUPPORTED, "sizes too large");
+    if (!(d->scale >= 0.f) || !std::isfinite(d->scale))
+        return fail(PBA_ERR_INVALID_ARG, "scale must be finite and >= 0 (0 = 1/sqrt(C))");
+    return PBA_OK;
+}
+
+pba_status check_layouts(const pba_dims *d) {
+    pba_status st;
+    if ((st = check_strides(d->sq, d->B, d->Nq, d->H, "q")) != PBA_OK) return st;
+    if ((st = check_strides(d->sk, d->B, d->Nk, d->H, "k")) != PBA_OK) return st;
+    if ((st = check_strides(d->sv, d->B, d->Nk, d->H, "v")) != PBA_OK) return st;
+    if ((st = check_strides(d->so, d->B, d->Nq, d->H, "out")) != PBA_OK) return st;
+    return PBA_OK;
+}
+
+pba_status check_bias(const pba_dims *d) {
+    if (d->H > 1 && (d->sbias[0] <= 0 || d->sbias[0] % 8))
+        return fail(PBA_ERR_INVALID_ARG, "bias: H stride must be a positive multiple of 8");
+    if (d->Nq > 1 && (d->sbias[1] <= 0 || d->sbias[1] % 8))
+        return fail(PBA_ERR_INVALID_ARG, "bias: Nq stride must be a positive multiple of 8");
+    return PBA_OK;
+}
+
+int padded_c(int C) { return C <= 16 ? 16 : (C <= 32 ? 32 : 64); }
+
+float eff_scale(const pba_dims *d) {
+    return d->scale > 0.f ? d->scale : 1.0f / std::sqrt((float)d->C);
+}
+
+template <typename K>
+pba_status set_smem(K kernel, int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    return PBA_OK;
+}
+
+template <int CP>
+pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                      const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
+                      pba_bf16 *out, float *lse, const pba_dims *d, cudaStream_t stream) {
+    using T = pba::FwdTraits<CP>;
+    CUtensorMap tq, tk, tv, tb;
+    pba_status st;
+    if ((st = map_bnhc(&tq, q, d->B, d->Nq, d->H, d->C, d->sq, CP, "q")) != PBA_OK) return st;
+    if ((st = map_bnhc(&tk, k, d->B, d->Nk, d->H, d->C, d->sk, CP, "k")) != PBA_OK) return st;
+    if ((st = map_bnhc(&tv, v, d->B, d->Nk, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
+    if (bias) {
+        if ((st = map_bias(&tb, bias, d->H, d->Nq, d->Nk, d->sbias)) != PBA_OK) return st;
+    } else {
+        std::memset(&tb, 0, sizeof(tb));
+    }
+    pba::FwdArgs a;
+    a.B = d->B; a.H = d->H; a.Nq = d->Nq; a.Nk = d->Nk; a.C = d->C;
+    a.nI = (d->Nq + 127) / 128;
+    a.nJ = (d->Nk + 127) / 128;
+    // rows per CTA: as many as TMEM holds, fewer when that would leave SMs idle
+    const long long tiles = (long long)a.nI * d->H;
+    int bc = T::BCMAX;
+    while (bc > 2 && tiles * ((d->B + bc - 1) / bc) < 2LL * 148) bc /= 2;
+    a.bc = bc;
+    a.nChunks = (d->B + bc - 1) / bc;
+    a.scale = eff_scale(d);
+    a.has_bias = bias != nullptr;
+    a.mask = mask;
+    a.smask_b = d->smask_b;
+    a.gate = reinterpret_cast<const __nv_bfloat16 *>(gate);
+    a.sg0 = d->sg[0]; a.sg1 = d->sg[1]; a.sg2 = d->sg[2];
+    a.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
+    a.lse = lse;
+    if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
+    const long long grid = tiles * a.nChunks;
+    pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pba_fwd_kernel launch");
+    return PBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void pba_dims_dense(pba_dims *d, int32_t B, int32_t H, int32_t Nq, int32_t Nk, int32_t C,
+                    float scale) {
+    std::memset(d, 0, sizeof(*d));
+    d->B = B; d->H = H; d->Nq = Nq; d->Nk = Nk; d->C = C;
+    d->scale = scale;
+    const int64_t q3[3] = {(int64_t)Nq * H * C, (int64_t)H * C, C};
+    const int64_t k3[3] = {(int64_t)Nk * H * C, (int64_t)H * C, C};
+    for (int i = 0; i < 3; ++i) {
+        d->sq[i] = q3[i]; d->sg[i] = q3[i]; d->so[i] = q3[i];
+        d->sk[i] = k3[i]; d->sv[i] = k3[i];
+    }
+    d->sbias[0] = (int64_t)Nq * Nk;
+    d->sbias[1] = Nk;
+    d->smask_b = 0;
+}
+
+pba_status pba_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                   const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                   pba_bf16 *out, float *lse, const pba_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->B == 0 || d->Nq == 0) return PBA_OK;  // nothing to compute
+    if ((st = check_layouts(d)) != PBA_OK) return st;
+    if (!q || !k || !v || !out || !lse) return fail(PBA_ERR_INVALID_ARG, "q, k, v, out and lse are required");
+    if (d->Nk > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v)))
+        return fail(PBA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
+    if (!aligned16(out)) return fail(PBA_ERR_INVALID_ARG, "out must be 16-byte aligned");
+    if (gate) {
+        if (!aligned16(gate)) return fail(PBA_ERR_INVALID_ARG, "gate must be 16-byte aligned");
+        if ((st = check_strides(d->sg, d->B, d->Nq, d->H, "gate")) != PBA_OK) return st;
+    }
+    if (bias) {
+        if (!aligned16(bias)) return fail(PBA_ERR_INVALID_ARG, "bias must be 16-byte aligned");
+        if ((st = check_bias(d)) != PBA_OK) return st;
+    }
+    if (key_mask && d->smask_b < 0) return fail(PBA_ERR_INVALID_ARG, "smask_b must be >= 0");
+    if ((st = get_encoder()) != PBA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (padded_c(d->C)) {
+        case 16: return launch_fwd<16>(q, k, v, bias, key_mask, gate, out, lse, d, s);
+        case 32: return launch_fwd<32>(q, k, v, bias, key_mask, gate, out, lse, d, s);
+        default: return launch_fwd<64>(q, k, v, bias, key_mask, gate, out, lse, d, s);
+    }
+}
+
+size_t pba_bwd_workspace_size(const pba_dims *d) { (void)d; return 0; }
+
+pba_status pba_bwd(const pba_bf16 *, const pba_bf16 *, const pba_bf16 *, const pba_bf16 *,
+                   const uint8_t *, const pba_bf16 *, const pba_bf16 *, const float *,
+                   const pba_bf16 *, pba_bf16 *, pba_bf16 *, pba_bf16 *, float *, pba_bf16 *,
+                   void *, size_t, const pba_dims *, void *) {
+    return fail(PBA_ERR_UNSUPPORTED, "backward not built yet");
+}
+
+pba_status pba_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int w = 0, site = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&w, pba::g_pba_watchdog, sizeof(w));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the watchdog word");
+    if (w) {
+        cudaMemcpyFromSymbol(&site, pba::g_pba_watchdog_site, sizeof(site));
+        cudaMemcpyToSymbol(pba::g_pba_watchdog, &zero, sizeof(zero));
+        cudaMemcpyToSymbol(pba::g_pba_watchdog_site, &zero, sizeof(zero));
+        return fail(PBA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (site 0x%x)", site);
+    }
+    return PBA_OK;
+}
+
+const char *pba_status_string(pba_status s) {
+    switch (s) {
+        case PBA_OK: return "PBA_OK";
+        case PBA_ERR_INVALID_ARG: return "PBA_ERR_INVALID_ARG";
+        case PBA_ERR_UNSUPPORTED: return "PBA_ERR_UNSUPPORTED";
+        case PBA_ERR_CUDA: return "PBA_ERR_CUDA";
+        case PBA_ERR_TIMEOUT: return "PBA_ERR_TIMEOUT";
+        case PBA_ERR_WORKSPACE: return "PBA_ERR_WORKSPACE";
+    }
+    return "PBA_ERR_UNKNOWN";
+}
+
+const char *pba_last_error(void) { return g_last_error.c_str(); }
+
+int pba_version(void) { return PBA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function that
+include/pba.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pba():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "pba_build", os.path.join(ROOT, "pair_biased_attention_gated_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
+    import pair_biased_attention_gated_b200 as p
+    return p
+
+
+def _declared_functions():
+    names = []
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if not hdr.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(pba_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("pba_fwd", "pba_bwd", "pba_bwd_workspace_size", "pba_status_string",
+                     "pba_device_status", "pba_dims_dense", "pba_last_error", "pba_version"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(pba):
+    lib = ctypes.CDLL(pba.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(pba):
+    assert pba.lib.pba_version() == 1
+    for code, name in pba.STATUS.items():
+        assert pba.lib.pba_status_string(code).decode() == name
+
+
+def test_dims_dense(pba):
+    d = pba.dims_dense(3, 4, 5, 6, 32)
+    assert (d.B, d.H, d.Nq, d.Nk, d.C) == (3, 4, 5, 6, 32)
+    assert list(d.sq) == [5 * 4 * 32, 4 * 32, 32]
+    assert list(d.sk) == [6 * 4 * 32, 4 * 32, 32]
+    assert list(d.sbias) == [5 * 6, 6]
+    assert d.smask_b == 0
+
+
+def _fwd_status(pba, d, q=16, k=16, v=16, out=16, lse=16, bias=None, gate=None):
+    st = pba.lib.pba_fwd(q, k, v, bias, None, gate, out, lse, ctypes.byref(d), None)
+    return st, pba.lib.pba_last_error().decode()
+
+
+def test_host_side_argument_errors(pba):
+    d = pba.dims_dense(2, 2, 64, 64, 32)
+    assert _fwd_status(pba, d, q=None)[0] == 1
+    assert _fwd_status(pba, d, out=None)[0] == 1
+    assert _fwd_status(pba, d, q=24)[0] == 1          # misaligned pointer
+    d2 = pba.dims_dense(2, 2, 64, 64, 12)            # C not a multiple of 8
+    assert _fwd_status(pba, d2)[0] == 2
+    d3 = pba.dims_dense(2, 2, 64, 64, 128)           # C > 64
+    assert _fwd_status(pba, d3)[0] == 2
+    d4 = pba.dims_dense(2, 2, 64, 64, 32)
+    d4.sq[1] = 100                                    # stride not a multiple of 8
+    st, msg = _fwd_status(pba, d4)
+    assert st == 1 and "stride" in msg
+    d5 = pba.dims_dense(2, 2, 64, 64, 32)
+    d5.scale = float("nan")
+    assert _fwd_status(pba, d5)[0] == 1
+    d6 = pba.dims_dense(-1, 2, 64, 64, 32)
+    assert _fwd_status(pba, d6)[0] == 1
+    d7 = pba.dims_dense(2, 2, 64, 60, 32)            # bias row stride 60: not TMA-able
+    assert _fwd_status(pba, d7, bias=16)[0] == 1
+
+
+def test_empty_problem_is_a_no_op(pba):
+    d = pba.dims_dense(0, 2, 64, 64, 32)
+    assert _fwd_status(pba, d, q=None, k=None, v=None, out=None, lse=None)[0] == 0
+    d = pba.dims_dense(2, 2, 0, 64, 32)
+    assert _fwd_status(pba, d, q=None, k=None, v=None, out=None, lse=None)[0] == 0
