@@ -196,6 +196,155 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     return PBA_OK;
 }
 
+// ---------------------------------------------------------------------------- backward
+struct BwdPlan {
+    int nI, nJ, NqPad, NkPad, splits, rows_per_split;
+    size_t off_rs, off_doa, off_dq, off_part, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+BwdPlan plan_bwd(const pba_dims *d) {
+    BwdPlan p;
+    p.nI = (d->Nq + 127) / 128;
+    p.nJ = (d->Nk + 127) / 128;
+    p.NqPad = p.nI * 128;
+    p.NkPad = p.nJ * 128;
+    // splits of the broadcast rows for the dbias kernel: a fixed function of the sizes,
+    // so the reduction order (and every bit of dbias) depends on nothing else
+    const long long tiles = (long long)d->H * p.nI * p.nJ;
+    long long splits = tiles > 0 ? (2LL * 148 + tiles - 1) / tiles : 1;
+    if (splits < 1) splits = 1;
+    if (splits > d->B) splits = d->B > 0 ? d->B : 1;
+    if (splits > 64) splits = 64;
+    p.rows_per_split = d->B > 0 ? (int)((d->B + splits - 1) / splits) : 1;
+    p.splits = d->B > 0 ? (d->B + p.rows_per_split - 1) / p.rows_per_split : 1;
+    const size_t rows = (size_t)d->B * d->H * p.NqPad;
+    const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
+    p.off_rs = 0;
+    p.off_doa = align256(p.off_rs + rows * sizeof(float2));
+    p.off_dq = align256(p.off_doa + elems * 2);
+    p.off_part = align256(p.off_dq + elems * 4);
+    p.total = align256(p.off_part + (size_t)p.splits * d->H * p.NqPad * p.NkPad * 4);
+    return p;
+}
+
+__global__ void zero_rows_kernel(__nv_bfloat16 *dk, __nv_bfloat16 *dv, pba::BwdArgs a) {
+    const int c8n = a.C / 8;
+    const long long n = (long long)a.B * a.Nk * a.H * c8n;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int c8 = (int)(e % c8n);
+        const long long r = e / c8n;
+        const int h = (int)(r % a.H);
+        const long long bj = r / a.H;
+        const int j = (int)(bj % a.Nk);
+        const int b = (int)(bj / a.Nk);
+        *reinterpret_cast<uint4 *>(dk + b * a.sk0 + (long long)j * a.sk1 + h * a.sk2 + c8 * 8) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(dv + b * a.sv0 + (long long)j * a.sv1 + h * a.sv2 + c8 * 8) = make_uint4(0, 0, 0, 0);
+    }
+}
+
+unsigned grid_for(long long n, int threads) {
+    long long g = (n + threads - 1) / threads;
+    if (g > 148LL * 32) g = 148LL * 32;
+    return (unsigned)(g > 0 ? g : 1);
+}
+
+pba_status launch_zero_rows(pba_bf16 *dk, pba_bf16 *dv, const pba_dims *d, cudaStream_t s) {
+    if (!aligned16(dk) || !aligned16(dv)) return fail(PBA_ERR_INVALID_ARG, "dk, dv must be 16-byte aligned");
+    pba::BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = d->B; a.H = d->H; a.Nk = d->Nk; a.C = d->C;
+    a.sk0 = d->sk[0]; a.sk1 = d->sk[1]; a.sk2 = d->sk[2];
+    a.sv0 = d->sv[0]; a.sv1 = d->sv[1]; a.sv2 = d->sv[2];
+    const long long n = (long long)d->B * d->Nk * d->H * (d->C / 8);
+    zero_rows_kernel<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<__nv_bfloat16 *>(dk),
+                                                       reinterpret_cast<__nv_bfloat16 *>(dv), a);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PBA_OK : cuda_fail(e, "zero_rows_kernel launch");
+}
+
+template <int CP>
+pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                      const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
+                      const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                      pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                      void *ws, const BwdPlan &pl, const pba_dims *d, cudaStream_t s) {
+    using MT = pba::BwdTraits<CP>;
+    using DT = pba::DbTraits<CP>;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    pba::BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = d->B; a.H = d->H; a.Nq = d->Nq; a.Nk = d->Nk; a.C = d->C;
+    a.nI = pl.nI; a.nJ = pl.nJ; a.NqPad = pl.NqPad; a.NkPad = pl.NkPad;
+    a.splits = pl.splits; a.rows_per_split = pl.rows_per_split;
+    a.scale = eff_scale(d);
+    a.has_bias = bias != nullptr;
+    a.has_gate = gate != nullptr;
+    a.mask = mask;
+    a.smask_b = d->smask_b;
+    a.gate = reinterpret_cast<const __nv_bfloat16 *>(gate);
+    a.out = reinterpret_cast<const __nv_bfloat16 *>(out);
+    a.dout = reinterpret_cast<const __nv_bfloat16 *>(dout);
+    a.sg0 = d->sg[0]; a.sg1 = d->sg[1]; a.sg2 = d->sg[2];
+    a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
+    a.lse = lse;
+    a.dq = reinterpret_cast<__nv_bfloat16 *>(dq);
+    a.dk = reinterpret_cast<__nv_bfloat16 *>(dk);
+    a.dv = reinterpret_cast<__nv_bfloat16 *>(dv);
+    a.dgate = reinterpret_cast<__nv_bfloat16 *>(dgate);
+    a.sq0 = d->sq[0]; a.sq1 = d->sq[1]; a.sq2 = d->sq[2];
+    a.sk0 = d->sk[0]; a.sk1 = d->sk[1]; a.sk2 = d->sk[2];
+    a.sv0 = d->sv[0]; a.sv1 = d->sv[1]; a.sv2 = d->sv[2];
+    a.dbias = dbias;
+    a.rowstats = reinterpret_cast<float2 *>(w + pl.off_rs);
+    a.doa = reinterpret_cast<__nv_bfloat16 *>(w + pl.off_doa);
+    a.dqacc = reinterpret_cast<float *>(w + pl.off_dq);
+    a.dbias_part = reinterpret_cast<float *>(w + pl.off_part);
+
+    pba_status st;
+    CUtensorMap tq, tk, tv, tdo, tb;
+    if ((st = map_bnhc(&tq, q, d->B, d->Nq, d->H, d->C, d->sq, CP, "q")) != PBA_OK) return st;
+    if ((st = map_bnhc(&tk, k, d->B, d->Nk, d->H, d->C, d->sk, CP, "k")) != PBA_OK) return st;
+    if ((st = map_bnhc(&tv, v, d->B, d->Nk, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
+    if (gate) {
+        const int64_t sd[3] = {(int64_t)d->Nq * d->H * d->C, (int64_t)d->H * d->C, d->C};
+        if ((st = map_bnhc(&tdo, a.doa, d->B, d->Nq, d->H, d->C, sd, CP, "dOa")) != PBA_OK) return st;
+    } else {
+        if ((st = map_bnhc(&tdo, dout, d->B, d->Nq, d->H, d->C, d->so, CP, "dout")) != PBA_OK) return st;
+    }
+    if (bias) {
+        if ((st = map_bias(&tb, bias, d->H, d->Nq, d->Nk, d->sbias)) != PBA_OK) return st;
+    } else {
+        std::memset(&tb, 0, sizeof(tb));
+    }
+    cudaError_t e;
+    const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
+    if ((e = cudaMemsetAsync(a.dqacc, 0, elems * 4, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    const long long pre_rows = (long long)d->B * pl.NqPad * d->H;
+    pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows, 256), 256, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_pre_kernel launch");
+    if (pl.nJ > 0) {
+        if ((st = set_smem(pba::pba_bwd_main_kernel<CP>, MT::SMEM_BYTES)) != PBA_OK) return st;
+        const long long grid = (long long)d->B * d->H * pl.nJ;
+        pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 320, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
+        if (dbias) {
+            if ((st = set_smem(pba::pba_dbias_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
+            const long long g2 = (long long)pl.splits * d->H * pl.nI * pl.nJ;
+            pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
+            const long long n = (long long)d->H * d->Nq * d->Nk;
+            pba::pba_dbias_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(a);
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_reduce_kernel launch");
+        }
+    }
+    pba::pba_dq_convert_kernel<<<grid_for((long long)elems / 8, 256), 256, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dq_convert_kernel launch");
+    return PBA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -246,13 +395,59 @@ pba_status pba_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     }
 }
 
-size_t pba_bwd_workspace_size(const pba_dims *d) { (void)d; return 0; }
+size_t pba_bwd_workspace_size(const pba_dims *d) {
+    if (!d || check_dims(d) != PBA_OK) return 0;
+    return plan_bwd(d).total;
+}
 
-pba_status pba_bwd(const pba_bf16 *, const pba_bf16 *, const pba_bf16 *, const pba_bf16 *,
-                   const uint8_t *, const pba_bf16 *, const pba_bf16 *, const float *,
-                   const pba_bf16 *, pba_bf16 *, pba_bf16 *, pba_bf16 *, float *, pba_bf16 *,
-                   void *, size_t, const pba_dims *, void *) {
-    return fail(PBA_ERR_UNSUPPORTED, "backward not built yet");
+pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                   const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                   const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                   pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                   void *workspace, size_t workspace_bytes, const pba_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->B == 0) return PBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d->Nq == 0) {
+        // no query: every key gradient is zero, there is no dq, dgate or dbias element
+        if (d->Nk == 0) return PBA_OK;
+        if (!dk || !dv) return fail(PBA_ERR_INVALID_ARG, "dk and dv are required");
+        if ((st = check_strides(d->sk, d->B, d->Nk, d->H, "k")) != PBA_OK) return st;
+        if ((st = check_strides(d->sv, d->B, d->Nk, d->H, "v")) != PBA_OK) return st;
+        if ((st = get_encoder()) != PBA_OK) return st;  // (keeps error handling uniform)
+        return launch_zero_rows(dk, dv, d, s);
+    }
+    if ((st = check_layouts(d)) != PBA_OK) return st;
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
+        return fail(PBA_ERR_INVALID_ARG, "q, k, v, out, lse, dout, dq, dk and dv are required");
+    if (gate && !dgate) return fail(PBA_ERR_INVALID_ARG, "dgate is required when gate is given");
+    const void *aligned_ptrs[] = {q, k, v, out, dout, dq, dk, dv};
+    for (const void *p : aligned_ptrs)
+        if (!aligned16(p)) return fail(PBA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    if (gate) {
+        if (!aligned16(gate) || !aligned16(dgate))
+            return fail(PBA_ERR_INVALID_ARG, "gate and dgate must be 16-byte aligned");
+        if ((st = check_strides(d->sg, d->B, d->Nq, d->H, "gate")) != PBA_OK) return st;
+    }
+    if (bias) {
+        if (!aligned16(bias)) return fail(PBA_ERR_INVALID_ARG, "bias must be 16-byte aligned");
+        if ((st = check_bias(d)) != PBA_OK) return st;
+    }
+    if (key_mask && d->smask_b < 0) return fail(PBA_ERR_INVALID_ARG, "smask_b must be >= 0");
+    const BwdPlan pl = plan_bwd(d);
+    if (!workspace || workspace_bytes < pl.total)
+        return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+                    pl.total);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(PBA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if ((st = get_encoder()) != PBA_OK) return st;
+    switch (padded_c(d->C)) {
+        case 16: return launch_bwd<16>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
+        case 32: return launch_bwd<32>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
+        default: return launch_bwd<64>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
+    }
 }
 
 pba_status pba_device_status(void *stream) {
