@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of pair-biased gated attention on B200: fwd+bwd TFLOP/s and % of roofline.
+
+A step is one pass of the whole hot path: the forward kernel (out, lse) and the backward
+kernels (dq, dk, dv, dgate, dbias) over one batch of synthetic, seeded bf16 input shaped
+like the MSA row attention workload (128 MSA rows share one [8, 256, 256] pair bias;
+`--config` selects another workload).  Inputs are resident in HBM when the timed region
+starts; L2 is flushed before every timed step, outside the timed events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU, each an independent replica of the
+workload (the path has no exchange step); rank 0 prints one JSON line.  `--impl
+reference` times the fp64 CPU oracle (the only other implementation of the operation)
+on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import pba_inputs as pi  # noqa: E402
+
+METRIC = "pair-bias attention fwd / fwd+bwd TFLOP/s and %roofline on 1 B200"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic work (unmasked keys only; c is the true head dim)
+# ---------------------------------------------------------------------------------------
+
+def work(cfg: pi.Config, B=None):
+    B = cfg.B if B is None else B
+    H, N, c, nv = cfg.H, cfg.N, cfg.c, cfg.n_valid_keys
+    unit = B * H * N * nv * c
+    e = B * N * H * c                       # elements of one [B, N, H, c] tensor
+    bias_b = H * N * N * 2
+    lse_b = B * H * N * 4
+    mask_b = N
+    f = {
+        "fwd_flops": 4 * unit,
+        "bwd_flops": 10 * unit,
+        # q, k, v, g in; out out; lse out; bias; mask
+        "fwd_bytes": 5 * e * 2 + lse_b + bias_b + mask_b,
+        # q, k, v, g, out, dout in; dq, dk, dv, dg out; lse; bias; mask; dbias out
+        "bwd_bytes": 10 * e * 2 + lse_b + bias_b + mask_b + H * N * N * 4,
+    }
+    # per-kernel algorithmic figures (what each kernel must move / multiply at minimum)
+    f["kernels"] = {
+        "pba_fwd_kernel": (4 * unit, 5 * e * 2 + lse_b + bias_b + mask_b),
+        # q, k, v, dOa, (lse, D) in; dq, dk, dv out; bias; mask
+        "pba_bwd_main_kernel": (10 * unit, 7 * e * 2 + B * H * N * 8 + bias_b + mask_b),
+        # q, k, v, dOa, (lse, D) in; bias; dbias out
+        "pba_dbias_kernel": (0, 4 * e * 2 + B * H * N * 8 + bias_b + H * N * N * 4),
+        # out, dout, g, lse in; dOa, dg, (lse, D) out
+        "pba_bwd_pre_kernel": (0, 5 * e * 2 + lse_b + B * H * N * 8),
+        "pba_dbias_reduce_kernel": (0, 2 * H * N * N * 4),
+        "pba_dq_convert_kernel": (0, e * 4 + e * 2),
+    }
+    return f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        with open(os.path.join(cdir, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    ent = d.get("kernels", {}).get(kernel, {}).get(workload)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region (NVML polling thread; reads only)
+# ---------------------------------------------------------------------------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # no NVML: clocks are reported as unavailable
+            self._nv = None
+        self.period = period_s
+        self._t = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local_rank])
+        except (ValueError, IndexError):
+            return local_rank
+    return local_rank
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the `--impl reference` arm)
+# ---------------------------------------------------------------------------------------
+
+def time_oracle(cfg: pi.Config, target_s: float, seed: int = 0, max_rows=None):
+    """fp64 oracle fwd+bwd on the first B_s broadcast rows of the workload, B_s sized for
+    about `target_s` seconds (the whole workload, repeated, when that is faster)."""
+    import oracle
+    import numpy as np
+
+    def run(Bs):
+        d = pi.make_inputs(cfg, seed=seed, B=Bs)
+        f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+        t0 = time.perf_counter()
+        oracle.fwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"))
+        oracle.bwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"), f["dout"])
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    per_row = max(t1, 1e-4)
+    Bs = int(max(1, min(cfg.B, target_s / per_row)))
+    if max_rows:
+        Bs = min(Bs, max_rows)
+    reps, elapsed = 0, 0.0
+    while True:
+        elapsed += run(Bs)
+        reps += 1
+        if elapsed >= target_s * 0.5 or Bs < cfg.B:
+            break
+    w = work(cfg, B=Bs)
+    flops = (w["fwd_flops"] + w["bwd_flops"]) * reps
+    threads = oracle.threads()
+    return {
+        "value": flops / elapsed / 1e12, "unit": "TFLOP/s",
+        "cores": min(threads, Bs * cfg.H), "kind": "oracle",
+        "sample": "%s fwd+bwd on %d of %d broadcast rows, x%d, %.1f s; fp64 C loops, OpenMP: "
+                  "fwd over (b,h) pairs, bwd over the %d heads (%d threads available)"
+                  % (cfg.name, Bs, cfg.B, reps, elapsed, cfg.H, threads),
+        "seconds": elapsed, "rows": Bs, "reps": reps,
+    }
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def run_ours(args, cfg):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    lib_path = os.path.join(ROOT, "pair_biased_attention_gated_b200", "libpba.so")
+    if not os.path.exists(lib_path):
+        if rank == 0:
+            import importlib.util
+            spec = importlib.util.spec_from_file_location(
+                "pba_build", os.path.join(ROOT, "pair_biased_attention_gated_b200", "build.py"))
+            mod = importlib.util.module_from_spec(spec)
+            spec.loader.exec_module(mod)
+            mod.build()
+        if pg:
+            pg.barrier()
+    import numpy as np
+    import pair_biased_attention_gated_b200 as pba
+
+    d = pi.make_inputs(cfg, seed=args.seed)
+    host = {}
+    for k, a in d.items():
+        t = torch.from_numpy(np.ascontiguousarray(a)) if k == "keep" else \
+            torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        host[k] = t.pin_memory()
+    dev = {k: v.cuda() for k, v in host.items()}
+    q, kk, v, g, bias, keep, dout = (dev["q"], dev["k"], dev["v"], dev.get("g"), dev["bias"],
+                                     dev["keep"], dev["dout"])
+    B, N, H, C = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(kk), torch.empty_like(v)
+    dg = torch.empty_like(g) if g is not None else None
+    db = torch.empty(H, N, N, dtype=torch.float32, device="cuda")
+    dims = pba.make_dims(q, kk, v, g, out, bias, keep)
+    ws = torch.empty(pba.pba_bwd_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pba.pba_fwd(q, kk, v, bias, keep, g, out, lse)
+        pba.pba_bwd(q, kk, v, bias, keep, g, out, lse, dout, dq, dk, dv, db, dg, ws)
+
+    def l2_flush(i):
+        flush.fill_(i & 0xFF)
+
+    for i in range(args.warmup):
+        l2_flush(i)
+        step()
+    pba.pba_device_status()
+
+    # ---- device-timed region: inputs resident in HBM
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    pba.profile_read()                   # drop anything recorded before
+    pba.profile_enable(True)
+    sampler.start()
+    for i in range(K):
+        l2_flush(i)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop()
+    pba.profile_enable(False)
+    kstats = pba.profile_read()
+    pba.pba_device_status()
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in ev)
+
+    # ---- end-to-end region: host buffers, copies inside the timed events
+    houts = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+             "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
+             "dq": torch.empty(dq.shape, dtype=dq.dtype).pin_memory(),
+             "dk": torch.empty(dk.shape, dtype=dk.dtype).pin_memory(),
+             "dv": torch.empty(dv.shape, dtype=dv.dtype).pin_memory(),
+             "db": torch.empty(db.shape, dtype=db.dtype).pin_memory()}
+    if dg is not None:
+        houts["dg"] = torch.empty(dg.shape, dtype=dg.dtype).pin_memory()
+    douts = {"out": out, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "db": db, "dg": dg}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in houts.values())
+    K2 = max(1, min(K, 20))
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K2)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    for i in range(K2):
+        l2_flush(i)
+        ev2[i][0].record(stream)
+        for k2, t in host.items():
+            dev[k2].copy_(t, non_blocking=True)
+        step()
+        for k2, t in houts.items():
+            t.copy_(douts[k2], non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    pba.pba_device_status()
+
+    if pg:
+        t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+
+    w = work(cfg)
+    step_flops = w["fwd_flops"] + w["bwd_flops"]
+    value = world * step_flops * K / (elapsed_ms / 1e3) / 1e12
+    e2e_value = world * step_flops * K2 / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tens = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    # dominant kernel and its roofline
+    total_k = sum(ms for _, ms in kstats.values()) or 1.0
+    dom = max(kstats.items(), key=lambda kv: kv[1][1])[0] if kstats else None
+    roof = None
+    if dom:
+        launches, ms = kstats[dom]
+        avg_s = ms / launches / 1e3
+        kf, kb = w["kernels"].get(dom, (0, 0))
+        t_tensor, t_hbm = kf / (tens * 1e12), kb / (hbm * 1e9)
+        if t_tensor > t_hbm:
+            achieved, peak, unit, bound = kf / avg_s / 1e12, tens, "TFLOP/s", "tensor"
+        else:
+            achieved, peak, unit, bound = kb / avg_s / 1e9, hbm, "GB/s", "hbm"
+        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
+                "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
+                "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
+                "algorithmic_per_launch": {"flops": kf, "bytes": kb},
+                "avg_launch_us": round(avg_s * 1e6, 2),
+                "traffic": ncu_traffic(dom, cfg.name)}
+    # the whole step against its own roofline
+    t_step_roof = max(step_flops / (tens * 1e12),
+                      (w["fwd_bytes"] + w["bwd_bytes"]) / (hbm * 1e9))
+    ms_per_step = elapsed_ms / K
+    fwd_ms = kstats.get("pba_fwd_kernel", (K, 0.0))[1] / K
+    kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
+               for n, (l, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1])}
+    launches_total = sum(l for l, _ in kstats.values())
+
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 q/k/v/gate/dout, N(0,%g^2) bias, shapes of "
+                "the named workload" % cfg.bias_std,
+        "config": {"workload": "%s: %s" % (cfg.name, cfg.desc), "B": cfg.B, "H": cfg.H,
+                   "N": cfg.N, "c": cfg.c, "masked_keys": cfg.N - cfg.n_valid_keys,
+                   "gate": cfg.gate, "passes": "fwd+bwd (dq, dk, dv, dgate, dbias)",
+                   "l2": "flushed before every timed step (256 MiB write outside the events)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "step_roofline": {"time_us": round(t_step_roof * 1e6, 2),
+                          "frac": round(t_step_roof * 1e3 / ms_per_step, 4)},
+        "fwd_tflops": round(w["fwd_flops"] / (fwd_ms / 1e3) / 1e12, 3) if fwd_ms > 0 else None,
+        "fwd_roofline_frac": round(max(w["fwd_flops"] / (tens * 1e12),
+                                       w["fwd_bytes"] / (hbm * 1e9)) * 1e3 / fwd_ms, 4)
+        if fwd_ms > 0 else None,
+        "kernels": kernels,
+        "gpu_launches": launches_total,
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": K2},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = time_oracle(cfg, target_s=args.cpu_seconds, seed=args.seed)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return res if rank == 0 else None
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    W, K = args.warmup, args.steps
+    # size one step so the whole run stays within a few minutes
+    per_step_s = max(0.2, min(4.0, 150.0 / max(1, K + W)))
+    cal = time_oracle(cfg, target_s=per_step_s, seed=args.seed)
+    Bs = cal["rows"]
+    import oracle
+    import numpy as np  # noqa: F401
+    d = pi.make_inputs(cfg, seed=args.seed, B=Bs)
+    f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+
+    def step():
+        oracle.fwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"))
+        oracle.bwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"), f["dout"])
+
+    for _ in range(W):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        step()
+    el = time.perf_counter() - t0
+    w = work(cfg, B=Bs)
+    value = (w["fwd_flops"] + w["bwd_flops"]) * K / el / 1e12
+    threads = oracle.threads()
+    sample = ("%s fwd+bwd on %d of %d broadcast rows per step; fp64 C loops, OpenMP (fwd over "
+              "(b,h), bwd over the %d heads; %d threads available)"
+              % (cfg.name, Bs, cfg.B, cfg.H, threads))
+    return {
+        "metric": METRIC, "impl": "reference", "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(el / K * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded bf16 inputs of the named workload, widened to fp64",
+        "config": {"workload": "%s: %s" % (cfg.name, cfg.desc), "B": cfg.B, "H": cfg.H,
+                   "N": cfg.N, "c": cfg.c, "sample_rows": Bs,
+                   "passes": "fwd+bwd (dq, dk, dv, dgate, dbias)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": min(threads, Bs * cfg.H), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="C2", choices=sorted(pi.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = pi.CONFIGS[args.config]
+    res = run_reference(args, cfg) if args.impl == "reference" else run_ours(args, cfg)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

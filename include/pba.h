@@ -117,6 +117,23 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
  */
 pba_status pba_device_status(void *stream);
 
+/*
+ * Kernel timing for benchmarks.  While enabled, every kernel this library launches is
+ * bracketed by two CUDA events recorded on the kernel's own stream, and counted.
+ * pba_profile_read() waits for the recorded events, writes one entry per kernel name
+ * (launch count and summed device time) into `out` (at most `max` entries), clears the
+ * records and returns the number of entries (or -1 on a CUDA error).  The events are
+ * CUDA event objects owned by the library and reused; no device memory is allocated.
+ */
+typedef struct {
+    char name[48];
+    int64_t launches;
+    double total_ms;
+} pba_kernel_stat;
+
+pba_status pba_profile_enable(int on);
+int pba_profile_read(pba_kernel_stat *out, int max);
+
 /* Static description of a status code. */
 const char *pba_status_string(pba_status s);
 

@@ -51,8 +51,15 @@ def _load():
                                        d, d]
         lib.pba_oracle_dbias_row.argtypes = [i, i, i, i, i, f, i, i, d, d, d, d, u8, ll, d, d,
                                              d]
+        lib.pba_oracle_threads.argtypes = []
+        lib.pba_oracle_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def threads() -> int:
+    """OpenMP threads available to the oracle's parallel loops."""
+    return int(_load().pba_oracle_threads())
 
 
 def _d(a: Optional[np.ndarray]):

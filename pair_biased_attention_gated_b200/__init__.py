@@ -57,6 +57,17 @@ lib.pba_version.argtypes = []
 lib.pba_version.restype = ctypes.c_int
 
 
+class PbaKernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
+
+
+lib.pba_profile_enable.argtypes = [ctypes.c_int]
+lib.pba_profile_enable.restype = ctypes.c_int
+lib.pba_profile_read.argtypes = [ctypes.POINTER(PbaKernelStat), ctypes.c_int]
+lib.pba_profile_read.restype = ctypes.c_int
+
+
 class PbaError(RuntimeError):
     def __init__(self, status: int, detail: str):
         super().__init__("%s: %s" % (STATUS.get(status, status), detail))
@@ -176,3 +187,20 @@ def attention_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, scale: float = 
     pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, ws,
             scale, stream)
     return dq, dk, dv, dgate, dbias
+
+
+# ---------------------------------------------------------------------------------------
+# kernel timing (CUDA events around every launch of the library)
+# ---------------------------------------------------------------------------------------
+
+def profile_enable(on: bool = True) -> None:
+    _check(lib.pba_profile_enable(1 if on else 0))
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total device ms)} since the last read."""
+    arr = (PbaKernelStat * 16)()
+    n = lib.pba_profile_read(arr, 16)
+    if n < 0:
+        raise PbaError(3, "reading kernel timing events failed")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}

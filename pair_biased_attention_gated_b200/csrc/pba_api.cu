@@ -13,6 +13,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/pba.h"
 #include "pba_bwd.cuh"
@@ -35,6 +36,52 @@ pba_status fail(pba_status s, const char *fmt, ...) {
 pba_status cuda_fail(cudaError_t e, const char *what) {
     return fail(PBA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+// ---------------------------------------------------------------------------- profiling
+enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DBIAS_REDUCE, K_DQ_CONVERT, K_ZERO_ROWS, K_COUNT };
+const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
+                                           "pba_dbias_kernel", "pba_dbias_reduce_kernel",
+                                           "pba_dq_convert_kernel", "zero_rows_kernel"};
+struct ProfRec {
+    int kid;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets one kernel launch with events when profiling is on.
+struct ProfScope {
+    int kid;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr;
+    ProfScope(int k, cudaStream_t st) : kid(k), s(st) {
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        if (!g_prof_on) return;
+        a = prof_event();
+        if (a) cudaEventRecord(a, s);
+    }
+    ~ProfScope() {
+        if (!a) return;
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        cudaEvent_t b = prof_event();
+        if (!b) return;
+        cudaEventRecord(b, s);
+        g_prof_recs.push_back({kid, a, b});
+    }
+};
 
 // ---------------------------------------------------------------------------- tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -190,7 +237,10 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.lse = lse;
     if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
     const long long grid = tiles * a.nChunks;
-    pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);
+    {
+        ProfScope ps(K_FWD, stream);
+        pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pba_fwd_kernel launch");
     return PBA_OK;
@@ -259,8 +309,11 @@ pba_status launch_zero_rows(pba_bf16 *dk, pba_bf16 *dv, const pba_dims *d, cudaS
     a.sk0 = d->sk[0]; a.sk1 = d->sk[1]; a.sk2 = d->sk[2];
     a.sv0 = d->sv[0]; a.sv1 = d->sv[1]; a.sv2 = d->sv[2];
     const long long n = (long long)d->B * d->Nk * d->H * (d->C / 8);
-    zero_rows_kernel<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<__nv_bfloat16 *>(dk),
-                                                       reinterpret_cast<__nv_bfloat16 *>(dv), a);
+    {
+        ProfScope ps(K_ZERO_ROWS, s);
+        zero_rows_kernel<<<grid_for(n, 256), 256, 0, s>>>(reinterpret_cast<__nv_bfloat16 *>(dk),
+                                                           reinterpret_cast<__nv_bfloat16 *>(dv), a);
+    }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PBA_OK : cuda_fail(e, "zero_rows_kernel launch");
 }
@@ -323,24 +376,39 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
     if ((e = cudaMemsetAsync(a.dqacc, 0, elems * 4, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     const long long pre_rows = (long long)d->B * pl.NqPad * d->H;
-    pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows, 256), 256, 0, s>>>(a);
+    {
+        ProfScope ps(K_BWD_PRE, s);
+        pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows, 256), 256, 0, s>>>(a);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_pre_kernel launch");
     if (pl.nJ > 0) {
         if ((st = set_smem(pba::pba_bwd_main_kernel<CP>, MT::SMEM_BYTES)) != PBA_OK) return st;
         const long long grid = (long long)d->B * d->H * pl.nJ;
-        pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 320, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+        {
+            ProfScope ps(K_BWD_MAIN, s);
+            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 320, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {
             if ((st = set_smem(pba::pba_dbias_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
             const long long g2 = (long long)pl.splits * d->H * pl.nI * pl.nJ;
-            pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+            {
+                ProfScope ps(K_DBIAS, s);
+                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+            }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
             const long long n = (long long)d->H * d->Nq * d->Nk;
-            pba::pba_dbias_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(a);
+            {
+                ProfScope ps(K_DBIAS_REDUCE, s);
+                pba::pba_dbias_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(a);
+            }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_reduce_kernel launch");
         }
     }
-    pba::pba_dq_convert_kernel<<<grid_for((long long)elems / 8, 256), 256, 0, s>>>(a);
+    {
+        ProfScope ps(K_DQ_CONVERT, s);
+        pba::pba_dq_convert_kernel<<<grid_for((long long)elems / 8, 256), 256, 0, s>>>(a);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dq_convert_kernel launch");
     return PBA_OK;
 }
@@ -463,6 +531,50 @@ pba_status pba_device_status(void *stream) {
         return fail(PBA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (site 0x%x)", site);
     }
     return PBA_OK;
+}
+
+pba_status pba_profile_enable(int on) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_on = on != 0;
+    return PBA_OK;
+}
+
+int pba_profile_read(pba_kernel_stat *out, int max) {
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        recs.swap(g_prof_recs);
+    }
+    int64_t launches[K_COUNT] = {0};
+    double ms[K_COUNT] = {0};
+    bool err = false;
+    for (const ProfRec &r : recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            err = true;
+        launches[r.kid] += 1;
+        ms[r.kid] += t;
+    }
+    {
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        for (const ProfRec &r : recs) {
+            g_prof_pool.push_back(r.a);
+            g_prof_pool.push_back(r.b);
+        }
+    }
+    if (err) return -1;
+    int n = 0;
+    for (int k = 0; k < K_COUNT; ++k) {
+        if (!launches[k]) continue;
+        if (out && n < max) {
+            std::memset(&out[n], 0, sizeof(out[n]));
+            std::snprintf(out[n].name, sizeof(out[n].name), "%s", kKernelNames[k]);
+            out[n].launches = launches[k];
+            out[n].total_ms = ms[k];
+        }
+        ++n;
+    }
+    return n < max ? n : max;
 }
 
 const char *pba_status_string(pba_status s) {
