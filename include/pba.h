@@ -111,6 +111,31 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                    void *stream);
 
 /*
+ * Backward pass for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this entry point exists for users of the library, not for the method.
+ * Some callers have no way to obtain scratch memory: a plugin running inside another
+ * framework's executor that owns all device memory and forbids cudaMalloc while it
+ * runs, or a binding from a language with no device allocator.  This variant takes the
+ * same arguments as pba_bwd except the workspace, and uses instead a scratch array built
+ * into the library (64 MiB in device global memory, held by every GPU that loads the
+ * library until the process exits).  It allocates nothing: no cudaMalloc, no cudaFree.
+ *  - Sizes whose workspace (pba_bwd_workspace_size) exceeds 64 MiB are rejected with
+ *    PBA_ERR_UNSUPPORTED before anything is launched; use pba_bwd for those.
+ *  - The first call on a device looks up the scratch array's device address with that
+ *    device current (one cudaGetSymbolAddress per device); make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array and leaves the last call's contents in
+ *    it (the parts that must start at zero are cleared by each call).  Calls whose
+ *    execution overlaps on the GPU (different streams, no ordering between them) race on
+ *    the array and give wrong results: order them.
+ */
+pba_status pba_bwd_noalloc(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                           const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                           const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                           pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias,
+                           pba_bf16 *dgate, const pba_dims *dims, void *stream);
+
+/*
  * Synchronizes `stream`, then reports and clears the device watchdog word of the
  * current device: PBA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, PBA_ERR_CUDA if the synchronization itself failed, else PBA_OK.

@@ -47,6 +47,8 @@ lib.pba_bwd_workspace_size.argtypes = [ctypes.POINTER(PbaDims)]
 lib.pba_bwd_workspace_size.restype = ctypes.c_size_t
 lib.pba_bwd.argtypes = [_vp] * 14 + [_vp, ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
 lib.pba_bwd.restype = ctypes.c_int
+lib.pba_bwd_noalloc.argtypes = [_vp] * 14 + [ctypes.POINTER(PbaDims), _vp]
+lib.pba_bwd_noalloc.restype = ctypes.c_int
 lib.pba_device_status.argtypes = [_vp]
 lib.pba_device_status.restype = ctypes.c_int
 lib.pba_status_string.argtypes = [ctypes.c_int]
@@ -152,6 +154,17 @@ def pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dg
                        _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                        _ptr(dbias), _ptr(dgate), _ptr(workspace), ws_bytes, ctypes.byref(d),
                        _stream(stream)))
+
+
+def pba_bwd_noalloc(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
+                    scale: float = 0.0, stream=None) -> None:
+    """pba_bwd without a workspace argument, for callers that cannot allocate device
+    memory: the library's built-in 64 MiB scratch array is used instead (see pba.h)."""
+    d = make_dims(q, k, v, gate, out, bias, key_mask, scale, dout=dout)
+    _check(lib.pba_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask),
+                               _ptr(gate), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(dbias), _ptr(dgate),
+                               ctypes.byref(d), _stream(stream)))
 
 
 def pba_device_status(stream=None) -> None:

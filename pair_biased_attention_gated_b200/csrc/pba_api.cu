@@ -413,6 +413,32 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     return PBA_OK;
 }
 
+// ---------------------------------------------------------------------------- no-alloc
+// Scratch of pba_bwd_noalloc: a file-scope device array, so callers that cannot allocate
+// can still run the backward pass.  In host code its name is only a stand-in; the
+// device address comes from cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+__device__ __align__(256) unsigned char g_pba_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::vector<void *> g_noalloc_addr;  // per device ordinal; nullptr until looked up
+
+pba_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if ((int)g_noalloc_addr.size() <= dev) g_noalloc_addr.resize(dev + 1, nullptr);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_pba_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return PBA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -516,6 +542,26 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         case 32: return launch_bwd<32>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
         default: return launch_bwd<64>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
     }
+}
+
+pba_status pba_bwd_noalloc(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                           const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                           const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                           pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias,
+                           pba_bf16 *dgate, const pba_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_dims(d);
+    if (st != PBA_OK) return st;
+    const size_t need = plan_bwd(d).total;
+    if (need > kNoAllocScratchBytes)
+        return fail(PBA_ERR_UNSUPPORTED,
+                    "pba_bwd_noalloc: these sizes need %zu bytes of scratch, more than the %zu "
+                    "built into the library; call pba_bwd with a workspace instead",
+                    need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != PBA_OK) return st;
+    return pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
+                   scratch, kNoAllocScratchBytes, d, stream);
 }
 
 pba_status pba_device_status(void *stream) {
