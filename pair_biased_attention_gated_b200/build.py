@@ -5,6 +5,7 @@ build entry point.  nvcc cross-compiles without a GPU.
 """
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -40,12 +41,45 @@ def nvcc() -> str:
     return "nvcc"
 
 
+# Kernels that split their registers between warpgroups with setmaxnreg.  The split adds
+# up to at most the registers the CTA is launched with (threads x the count ptxas assigns);
+# if ptxas assigned a different count the split could wait forever, so the build refuses.
+SETMAXNREG_KERNELS = {"pba_fwd_kernel": 168}
+
+
+def check_registers(ptxas_log: str) -> None:
+    current = None
+    seen = {}
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current:
+            seen[current] = int(m.group(1))
+            current = None
+    for name, want in SETMAXNREG_KERNELS.items():
+        hits = {k: v for k, v in seen.items() if name in k}
+        if not hits:
+            raise RuntimeError("ptxas output has no register count for %s" % name)
+        bad = {k: v for k, v in hits.items() if v != want}
+        if bad:
+            raise RuntimeError("register count of %s is %s, expected %d: the setmaxnreg split "
+                               "would not match the launch" % (name, bad, want))
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not needs_build():
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp, SRC]
-    subprocess.check_call(cmd)
+    cmd = [nvcc()] + NVCC_FLAGS + ["-Xptxas", "-v", "-o", tmp, SRC]
+    proc = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+    if verbose or proc.returncode != 0:
+        print(proc.stdout)
+    if proc.returncode != 0:
+        raise subprocess.CalledProcessError(proc.returncode, cmd, proc.stdout)
+    check_registers(proc.stdout)
     os.replace(tmp, LIB)
     return LIB
 

@@ -230,6 +230,7 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.has_bias = bias != nullptr;
     a.mask = mask;
     a.smask_b = d->smask_b;
+    a.mask_shared = (mask == nullptr || d->smask_b == 0 || d->B == 1) ? 1 : 0;
     a.gate = reinterpret_cast<const __nv_bfloat16 *>(gate);
     a.sg0 = d->sg[0]; a.sg1 = d->sg[1]; a.sg2 = d->sg[2];
     a.out = reinterpret_cast<__nv_bfloat16 *>(out);
