@@ -159,6 +159,16 @@ typedef struct {
 pba_status pba_profile_enable(int on);
 int pba_profile_read(pba_kernel_stat *out, int max);
 
+/*
+ * Test hook for the device watchdog (no production use).  With step >= 0, the next
+ * pba_fwd calls make their TMA producer skip the Q/K load of that step of every CTA, so
+ * the barrier it would have completed never does: the MMA issuer's bounded wait runs
+ * out (about one second), every role of the CTA drains what it issued and returns, and
+ * pba_device_status() then reports PBA_ERR_TIMEOUT.  No GPU fault is raised and the
+ * context stays usable.  step < 0 switches the hook off (the default).
+ */
+void pba_debug_skip_load(int step);
+
 /* Static description of a status code. */
 const char *pba_status_string(pba_status s);
 

@@ -55,6 +55,8 @@ lib.pba_status_string.argtypes = [ctypes.c_int]
 lib.pba_status_string.restype = ctypes.c_char_p
 lib.pba_last_error.argtypes = []
 lib.pba_last_error.restype = ctypes.c_char_p
+lib.pba_debug_skip_load.argtypes = [ctypes.c_int]
+lib.pba_debug_skip_load.restype = None
 lib.pba_version.argtypes = []
 lib.pba_version.restype = ctypes.c_int
 

@@ -22,6 +22,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+int g_debug_skip_step = -1;   // test hook, see pba_debug_skip_load
 
 pba_status fail(pba_status s, const char *fmt, ...) {
     char buf[512];
@@ -236,6 +237,7 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.out = reinterpret_cast<__nv_bfloat16 *>(out);
     a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
     a.lse = lse;
+    a.skip_step = g_debug_skip_step;
     if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
     const long long grid = tiles * a.nChunks;
     {
@@ -639,5 +641,7 @@ const char *pba_status_string(pba_status s) {
 const char *pba_last_error(void) { return g_last_error.c_str(); }
 
 int pba_version(void) { return PBA_VERSION; }
+
+void pba_debug_skip_load(int step) { g_debug_skip_step = step < 0 ? -1 : step; }
 
 }  // extern "C"

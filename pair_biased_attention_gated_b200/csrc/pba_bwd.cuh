@@ -272,6 +272,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tc_fence_after();
     const uint32_t tbase = s_tmem_base;
     volatile int *abort_flag = &s_abort;
+    // query tiles whose Q/dOa/row-stat (bias) loads were issued: [0, q_done) ([0, bias_done))
+    int q_done = 0, bias_done = 0;
 
     if (warp == 8) {
         // ------------------------------------------------------------------ producer
@@ -302,6 +304,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tma_load_4d(qdst + T::TILE_BYTES, &tmDO, b_q_full(st), 0, h, i0, b);
                 bulk_load(sbase + T::OFF_RS + st * 1024,
                           a.rowstats + ((long long)b * a.H + h) * a.NqPad + i0, 1024, b_q_full(st));
+                q_done = t + 1;
                 if (t >= BS) ok = mbar_wait(b_bias_empty(bs), ((t / BS) - 1) & 1, abort_flag, SITE_BWD_PROD);
                 if (!ok) break;
                 if (a.has_bias) {
@@ -312,11 +315,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 } else {
                     mbar_arrive(b_bias_full(bs));
                 }
-            }
-            if (!ok) {
-                mbar_wait_drain(b_kv, 0);
-                for (int tt = max(0, t - QS); tt <= t && tt < nI; ++tt)
-                    mbar_wait_drain(b_q_full(tt % QS), (tt / QS) & 1);
+                bias_done = t + 1;
             }
         }
     } else if (warp == 9) {
@@ -386,12 +385,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 umma_commit(b_q_empty(st));
                 umma_commit(b_dq_full(t & 1));
             }
-            if (ok) {
-                umma_commit(b_done);
-            } else {
-                umma_commit(b_drain);
-                mbar_wait_drain(b_drain, 0);
-            }
+            if (ok) umma_commit(b_done);
         }
     } else {
         // ------------------------------------------------------------------ elementwise
@@ -514,6 +508,22 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a wait ran out: let the copies and MMAs already issued finish before shared memory
+        // and TMEM are released (bounded waits)
+        if (warp == 8 && lane == 0) {
+            mbar_wait_drain(b_kv, 0);
+            for (int tt = max(0, q_done - QS); tt < q_done; ++tt) mbar_wait_drain(b_q_full(tt % QS), (tt / QS) & 1);
+            for (int tt = max(0, bias_done - BS); tt < bias_done; ++tt)
+                mbar_wait_drain(b_bias_full(tt % BS), (tt / BS) & 1);
+        }
+        if (warp == 9 && lane == 0) {
+            umma_commit(b_drain);
+            mbar_wait_drain(b_drain, 0);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 9) {
         __syncwarp();
         tc_fence_after();
@@ -595,6 +605,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc_fence_after();
     const uint32_t tbase = s_tmem_base;
     volatile int *abort_flag = &s_abort;
+    int n_done = 0;   // rows b whose stage loads were issued: [0, n_done)
 
     if (warp == 8) {
         // ------------------------------------------------------------------ producer
@@ -635,10 +646,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 bulk_load(s0 + 4 * T::TILE_BYTES, a.rowstats + ((long long)b * a.H + h) * a.NqPad + i0,
                           1024, b_full(st));
             }
-        }
-        if (!ok && lane == 0) {
-            mbar_wait_drain(b_bias, 0);
-            for (int nn = max(0, n - NS); nn < n; ++nn) mbar_wait_drain(b_full(nn % NS), (nn / NS) & 1);
+            n_done = n + 1;
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer
@@ -664,10 +672,6 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
                 umma_commit(b_sd_full(x));
                 umma_commit(b_empty(st));
-            }
-            if (!ok) {
-                umma_commit(b_drain);
-                mbar_wait_drain(b_drain, 0);
             }
         }
     } else {
@@ -714,6 +718,18 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        if (warp == 8 && lane == 0) {
+            mbar_wait_drain(b_bias, 0);
+            for (int nn = max(0, n_done - NS); nn < n_done; ++nn) mbar_wait_drain(b_full(nn % NS), (nn / NS) & 1);
+        }
+        if (warp == 9 && lane == 0) {
+            umma_commit(b_drain);
+            mbar_wait_drain(b_drain, 0);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 9) {
         __syncwarp();
         tc_fence_after();

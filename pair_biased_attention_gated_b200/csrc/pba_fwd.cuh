@@ -45,6 +45,7 @@ struct FwdArgs {
     __nv_bfloat16 *out;
     long long so0, so1, so2;
     float *lse;
+    int skip_step;   // test hook: the producer skips this step's Q/K load (-1: never)
 };
 
 template <int CP>
@@ -171,6 +172,10 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tbase = s_tmem_base;
     volatile int *abort_flag = &s_abort;
 
+    // steps whose Q/K (V) loads the producer issued are [0, qk_done) ([0, v_done)); bias
+    // tiles [0, n_bias): what has to land before the CTA may exit after an abort
+    int qk_done = 0, v_done = 0, n_bias = 0;
+
     if (warp >= 8) reg_dealloc<T::REGS_OTHER>();   // the whole third warpgroup, same point
     if (warp == 8) {
         // ------------------------------------------------------------------ producer
@@ -199,7 +204,6 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         };
         bool ok = true;
         int k = 0;
-        int n_qk = 0, n_v = 0, n_bias = 0;   // loads issued (for the drain after an abort)
         for (int j = 0; j < nJ && ok; ++j) {
             const int bs = j % BS;
             if (j >= BS) ok = mbar_wait(b_bias_empty(bs), ((j / BS) - 1) & 1, abort_flag, SITE_FWD_PROD | 0x20 | (j << 12));
@@ -226,13 +230,13 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 const int b = b0 + s;
-                if (lane == 0) {
+                if (lane == 0 && k != a.skip_step) {
                     const uint32_t dst = sbase + T::OFF_QK + sq * 2 * T::TILE_BYTES;
                     mbar_arrive_tx(b_qk_full(sq), 2 * T::TILE_BYTES);
                     tma_load_4d(dst, &tmQ, b_qk_full(sq), 0, h, i0, b);
                     tma_load_4d(dst + T::TILE_BYTES, &tmK, b_qk_full(sq), 0, h, j * 128, b);
                 }
-                ++n_qk;
+                qk_done = k + 1;
                 if (uv >= 1) ok = mbar_wait(b_v_empty(sv), (uv - 1) & 1, abort_flag, SITE_FWD_PROD | 0x10 | (k << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -246,14 +250,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     mbar_arrive_tx(b_v_full(sv), T::TILE_BYTES);
                     tma_load_4d(sbase + T::OFF_V + sv * T::TILE_BYTES, &tmV, b_v_full(sv), 0, h, j * 128, b);
                 }
-                ++n_v;
+                v_done = k + 1;
             }
-        }
-        if (!ok && lane == 0) {
-            // let every copy already issued land before the CTA's shared memory goes away
-            for (int kk = max(0, n_qk - QKS); kk < n_qk; ++kk) mbar_wait_drain(b_qk_full(kk % QKS), (kk / QKS) & 1);
-            for (int kk = max(0, n_v - VS); kk < n_v; ++kk) mbar_wait_drain(b_v_full(kk % VS), (kk / VS) & 1);
-            for (int jj = max(0, n_bias - BS); jj < n_bias; ++jj) mbar_wait_drain(b_bias_full(jj % BS), (jj / BS) & 1);
         }
     } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------------ MMA issuers
@@ -323,12 +321,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 k = kn;
                 ++n;
             }
-            if (ok) {
-                umma_commit(b_ofinal);   // each issuer arrives once (count = nW)
-            } else {
-                umma_commit(b_drain(w));
-                mbar_wait_drain(b_drain(w), 0);
-            }
+            if (ok) umma_commit(b_ofinal);   // each issuer arrives once (count = nW)
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------------ softmax
@@ -527,6 +520,22 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---------------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // Some wait ran out.  Every role has stopped; before shared memory and TMEM are
+        // released, let the copies and MMAs already issued finish (bounded waits).
+        if (warp == 8 && lane == 0) {
+            for (int kk = max(0, qk_done - QKS); kk < qk_done; ++kk)
+                if (kk != a.skip_step) mbar_wait_drain(b_qk_full(kk % QKS), (kk / QKS) & 1);
+            for (int kk = max(0, v_done - VS); kk < v_done; ++kk) mbar_wait_drain(b_v_full(kk % VS), (kk / VS) & 1);
+            for (int jj = max(0, n_bias - BS); jj < n_bias; ++jj) mbar_wait_drain(b_bias_full(jj % BS), (jj / BS) & 1);
+        }
+        if ((warp == 9 || warp == 10) && lane == 0 && warp - 9 < nW) {
+            umma_commit(b_drain(warp - 9));
+            mbar_wait_drain(b_drain(warp - 9), 0);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 9) {
         __syncwarp();
         tc_fence_after();
