@@ -17,14 +17,13 @@ namespace pba {
 __device__ unsigned int g_pba_watchdog;       // nonzero once any bounded wait ran out
 __device__ unsigned int g_pba_watchdog_site;  // the first site that gave up
 
-// A wait that is still unsatisfied after this long is treated as a hang.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+// A wait that is still unsatisfied after this many SM cycles is treated as a hang: about
+// 2 s at the clocks these parts run at, and at least 1 s at any clock up to 4 GHz.  The SM's
+// own cycle counter is used (monotonic on the SM the thread runs on), not the global
+// nanosecond timer, which the driver keeps in step with host time.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
+__device__ __forceinline__ long long sm_cycles() { return clock64(); }
 
 __device__ __forceinline__ void watchdog_fire(unsigned site) {
     atomicCAS(&g_pba_watchdog_site, 0u, site);
@@ -65,17 +64,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.  Returns false (and
 // raises the CTA's abort flag and the device watchdog) if it does not complete within
-// kWaitLimitNs, or if another role of the CTA has already aborted.
+// kWaitLimitCycles, or if another role of the CTA has already aborted.
 // `site` identifies the wait (kernel role and, in its upper bits, the step) in the device
 // watchdog word, so a report says where a kernel gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort_flag, unsigned site) {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
+    const long long t0 = sm_cycles();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (sm_cycles() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
             watchdog_fire(site);
             return false;
@@ -98,9 +97,9 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
-    const unsigned long long t0 = globaltimer();
+    const long long t0 = sm_cycles();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > kWaitLimitNs) return;
+        if (sm_cycles() - t0 > kWaitLimitCycles) return;
     }
 }
 

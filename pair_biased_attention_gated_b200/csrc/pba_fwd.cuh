@@ -7,25 +7,20 @@
 //
 // One CTA owns one (head h, 128-query tile, chunk of `bc` broadcast rows).  Its loop runs
 // over key tiles j (outer) and the chunk's rows b (inner), so each 128x128 bias tile is
-// moved into shared memory once and reused by all rows of the chunk.  Each step (j, b)
-// streams the Q and K tiles of row b through one ring of stages, released as soon as
-// Q K^T is done, and the V tile through a deeper ring, released after P V.
+// moved into shared memory once and reused by all rows of the chunk.  The Q tiles of the
+// chunk stay resident; K/V tiles stream through a ring.
 //
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup 0: the chunk's even rows (slot s = 0, 2, ...)
 //   warps 4-7  softmax warpgroup 1: the odd rows
 //   warp 8     TMA producer (Q, K, V, bias tiles) and key-mask bits
-//   warp 9     TMEM allocator; lane 0 issues the tcgen05 MMAs of softmax warpgroup 0
-//   warp 10    lane 0 issues the tcgen05 MMAs of softmax warpgroup 1
-//   warp 11    idle: it completes the third warpgroup, whose registers the softmax
+//   warp 9     TMEM allocator and, on lane 0, the tcgen05 MMA issuer
+//   warps 10-11 idle: they complete the third warpgroup, whose registers the softmax
 //              warpgroups take over (setmaxnreg)
-// Tensor memory (512 columns): S buffer of warpgroup 0 [0,128), of warpgroup 1 [128,256),
-// then one CP-column fp32 O accumulator per slot of the chunk.
-//
-// Per step a softmax warpgroup loads its S tile from TMEM and at once hands the buffer
-// back, so the next Q K^T of that warpgroup runs while it computes exp(); it then writes
-// P (bf16) to a shared-memory tile, from which the P V product reads.  Neither MMA is on
-// the warpgroup's critical path.
+// Tensor memory (512 columns): S/P buffer of warpgroup 0 [0,128), of warpgroup 1
+// [128,256), then one CP-column fp32 O accumulator per slot of the chunk.
+// The two warpgroups alternate: while one computes exp() of its S tile the MMA issuer
+// runs the other's Q K^T and P V products.
 #pragma once
 
 #include "pba_device.cuh"
@@ -45,26 +40,22 @@ struct FwdArgs {
     __nv_bfloat16 *out;
     long long so0, so1, so2;
     float *lse;
-    int skip_step;   // test hook: the producer skips this step's Q/K load (-1: never)
+    int skip_step;   // test hook: the producer skips this step's K/V load (-1: never)
 };
 
 template <int CP>
 struct FwdTraits {
     static constexpr int BCMAX = (CP == 64) ? 4 : 8;           // O slots in TMEM
-    static constexpr int QKS = (CP == 64) ? 2 : (CP == 32 ? 3 : 4);  // Q+K stages
-    static constexpr int VS = (CP == 64) ? 3 : (CP == 32 ? 5 : 6);   // V stages
-    static constexpr int BS = (CP == 64) ? 1 : 2;              // bias stages
+    static constexpr int KV_STAGES = (CP == 64) ? 2 : 3;
     static constexpr int TILE_BYTES = 128 * CP * 2;            // Q, K or V tile
     static constexpr int BIAS_BYTES = 128 * 128 * 2;           // two 64-key halves
-    static constexpr int P_BYTES = 128 * 128 * 2;              // P tile, two 64-key halves
-    static constexpr int OFF_QK = 0;                           // [QKS] x (Q, K)
-    static constexpr int OFF_V = OFF_QK + QKS * 2 * TILE_BYTES; // [VS] x V
-    static constexpr int OFF_BIAS = OFF_V + VS * TILE_BYTES;
-    static constexpr int OFF_P = OFF_BIAS + BS * BIAS_BYTES;   // [2 warpgroups]
-    static constexpr int OFF_STATS = OFF_P + 2 * P_BYTES;      // float2 [BCMAX][128]
-    static constexpr int OFF_MASK = OFF_STATS + BCMAX * 128 * 8; // u32 [VS][8] (per row b)
-    static constexpr int OFF_BMASK = OFF_MASK + VS * 32;         // u32 [BS][8] (shared by all b)
-    static constexpr int SMEM_BYTES = OFF_BMASK + BS * 32 + 1024;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = OFF_Q + BCMAX * TILE_BYTES;
+    static constexpr int OFF_BIAS = OFF_KV + KV_STAGES * 2 * TILE_BYTES;
+    static constexpr int OFF_STATS = OFF_BIAS + 2 * BIAS_BYTES;  // float2 [BCMAX][128]
+    static constexpr int OFF_MASK = OFF_STATS + BCMAX * 128 * 8; // u32 [KV_STAGES][8] (per row b)
+    static constexpr int OFF_BMASK = OFF_MASK + KV_STAGES * 32;  // u32 [2][8] (shared by all b)
+    static constexpr int SMEM_BYTES = OFF_BMASK + 2 * 32 + 1024;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
     static constexpr uint32_t ROWB = CP * 2;                   // bytes per tile row
     static constexpr int THREADS = 384;
@@ -92,28 +83,22 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmBias, const FwdArgs a) {
     using T = FwdTraits<CP>;
-    constexpr int QKS = T::QKS, VS = T::VS, BS = T::BS;
+    constexpr int KVS = T::KV_STAGES;
     extern __shared__ uint8_t dsmem[];
-    __shared__ __align__(8) uint64_t bars[4 + 2 * QKS + 2 * VS + 2 * BS + 8 + T::BCMAX];
+    __shared__ __align__(8) uint64_t bars[6 + 2 * KVS + 2 + 2 + 2 + 2];
     __shared__ uint32_t s_tmem_base;
     __shared__ int s_abort;
 
     // barrier slots
-    const uint32_t b_ofinal = smem_u32(&bars[0]);
-    auto b_drain = [&](int w) { return smem_u32(&bars[1 + w]); };             // abort path
-    auto b_qk_full = [&](int st) { return smem_u32(&bars[4 + st]); };          // Q, K landed
-    auto b_qk_empty = [&](int st) { return smem_u32(&bars[4 + QKS + st]); };   // Q K^T done
-    auto b_v_full = [&](int st) { return smem_u32(&bars[4 + 2 * QKS + st]); }; // V landed
-    auto b_v_empty = [&](int st) { return smem_u32(&bars[4 + 2 * QKS + VS + st]); };  // P V done
-    constexpr int OBB = 4 + 2 * QKS + 2 * VS;
-    auto b_bias_full = [&](int x) { return smem_u32(&bars[OBB + x]); };
-    auto b_bias_empty = [&](int x) { return smem_u32(&bars[OBB + BS + x]); };
-    constexpr int OB = OBB + 2 * BS;
-    auto b_s_full = [&](int w) { return smem_u32(&bars[OB + w]); };        // S in TMEM
-    auto b_s_free = [&](int w) { return smem_u32(&bars[OB + 2 + w]); };    // S read out
-    auto b_p_full = [&](int w) { return smem_u32(&bars[OB + 4 + w]); };    // P in smem
-    auto b_p_free = [&](int w) { return smem_u32(&bars[OB + 6 + w]); };    // P V done reading P
-    auto b_o_ready = [&](int s) { return smem_u32(&bars[OB + 8 + s]); };   // P V into O[s] done
+    const uint32_t b_q = smem_u32(&bars[0]);
+    const uint32_t b_ofinal = smem_u32(&bars[1]);
+    const uint32_t b_drain = smem_u32(&bars[2]);
+    auto b_kv_full = [&](int st) { return smem_u32(&bars[6 + st]); };
+    auto b_kv_empty = [&](int st) { return smem_u32(&bars[6 + KVS + st]); };
+    auto b_bias_full = [&](int x) { return smem_u32(&bars[6 + 2 * KVS + x]); };
+    auto b_bias_empty = [&](int x) { return smem_u32(&bars[6 + 2 * KVS + 2 + x]); };
+    auto b_s_full = [&](int x) { return smem_u32(&bars[6 + 2 * KVS + 4 + x]); };
+    auto b_p_full = [&](int x) { return smem_u32(&bars[6 + 2 * KVS + 6 + x]); };
 
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -131,28 +116,19 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int nW = nb >= 2 ? 2 : 1;
 
     if (threadIdx.x == 0) {
-        mbar_init(b_ofinal, nW);  // one commit from each MMA issuer
-        mbar_init(b_drain(0), 1);
-        mbar_init(b_drain(1), 1);
-        for (int st = 0; st < QKS; ++st) {
-            mbar_init(b_qk_full(st), 1);
-            mbar_init(b_qk_empty(st), 1);
+        mbar_init(b_q, 1);
+        mbar_init(b_ofinal, 1);
+        mbar_init(b_drain, 1);
+        for (int st = 0; st < KVS; ++st) {
+            mbar_init(b_kv_full(st), 1);
+            mbar_init(b_kv_empty(st), 1);
         }
-        for (int st = 0; st < VS; ++st) {
-            mbar_init(b_v_full(st), 1);
-            mbar_init(b_v_empty(st), 1);
-        }
-        for (int x = 0; x < BS; ++x) {
+        for (int x = 0; x < 2; ++x) {
             mbar_init(b_bias_full(x), 1);
             mbar_init(b_bias_empty(x), 128 * nW);
+            mbar_init(b_s_full(x), 1);
+            mbar_init(b_p_full(x), 128);
         }
-        for (int w = 0; w < 2; ++w) {
-            mbar_init(b_s_full(w), 1);
-            mbar_init(b_s_free(w), 128);
-            mbar_init(b_p_full(w), 128);
-            mbar_init(b_p_free(w), 1);
-        }
-        for (int s = 0; s < T::BCMAX; ++s) mbar_init(b_o_ready(s), 1);
         s_abort = 0;
         fence_mbar_init();
     }
@@ -172,9 +148,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tbase = s_tmem_base;
     volatile int *abort_flag = &s_abort;
 
-    // steps whose Q/K (V) loads the producer issued are [0, qk_done) ([0, v_done)); bias
-    // tiles [0, n_bias): what has to land before the CTA may exit after an abort
-    int qk_done = 0, v_done = 0, n_bias = 0;
+    // K/V loads issued for steps [0, kv_done), bias tiles [0, n_bias): what has to land
+    // before the CTA may exit after an abort
+    int kv_done = 0, n_bias = 0;
 
     if (warp >= 8) reg_dealloc<T::REGS_OTHER>();   // the whole third warpgroup, same point
     if (warp == 8) {
@@ -184,6 +160,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             if (a.has_bias) tma_prefetch_desc(&tmBias);
+            mbar_arrive_tx(b_q, nb * T::TILE_BYTES);
+            for (int s = 0; s < nb; ++s)
+                tma_load_4d(sbase + T::OFF_Q + s * T::TILE_BYTES, &tmQ, b_q, 0, h, i0, b0 + s);
         }
         // mask bits of key tile j for row b: word q bit t <-> key 128 j + 32 q + t attended
         auto mask_words = [&](int b, int j, uint32_t (&w)[4]) {
@@ -205,8 +184,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         bool ok = true;
         int k = 0;
         for (int j = 0; j < nJ && ok; ++j) {
-            const int bs = j % BS;
-            if (j >= BS) ok = mbar_wait(b_bias_empty(bs), ((j / BS) - 1) & 1, abort_flag, SITE_FWD_PROD | 0x20 | (j << 12));
+            const int bs = j & 1;
+            if (j >= 2) ok = mbar_wait(b_bias_empty(bs), ((j >> 1) - 1) & 1, abort_flag, SITE_FWD_PROD | 0x20 | (j << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             uint32_t wj[4] = {0, 0, 0, 0};
@@ -223,105 +202,98 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     mbar_arrive(b_bias_full(bs));
                 }
             }
-            ++n_bias;
+            n_bias = j + 1;
             for (int s = 0; s < nb; ++s, ++k) {
-                const int sq = k % QKS, uq = k / QKS, sv = k % VS, uv = k / VS;
-                if (uq >= 1) ok = mbar_wait(b_qk_empty(sq), (uq - 1) & 1, abort_flag, SITE_FWD_PROD | (k << 12));
+                const int st = k % KVS, use = k / KVS;
+                if (use >= 1) ok = mbar_wait(b_kv_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | (k << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 const int b = b0 + s;
-                if (lane == 0 && k != a.skip_step) {
-                    const uint32_t dst = sbase + T::OFF_QK + sq * 2 * T::TILE_BYTES;
-                    mbar_arrive_tx(b_qk_full(sq), 2 * T::TILE_BYTES);
-                    tma_load_4d(dst, &tmQ, b_qk_full(sq), 0, h, i0, b);
-                    tma_load_4d(dst + T::TILE_BYTES, &tmK, b_qk_full(sq), 0, h, j * 128, b);
-                }
-                qk_done = k + 1;
-                if (uv >= 1) ok = mbar_wait(b_v_empty(sv), (uv - 1) & 1, abort_flag, SITE_FWD_PROD | 0x10 | (k << 12));
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                // a per-row mask travels with the V stage: it is released only after P V,
-                // i.e. after the softmax of this step has read the mask
                 uint32_t w[4] = {0, 0, 0, 0};
                 if (!a.mask_shared) mask_words(b, j, w);
-                if (lane == 0) {
+                if (lane == 0 && k != a.skip_step) {
                     if (!a.mask_shared)
-                        put_words(reinterpret_cast<uint32_t *>(gbase + T::OFF_MASK) + sv * 8, w);
-                    mbar_arrive_tx(b_v_full(sv), T::TILE_BYTES);
-                    tma_load_4d(sbase + T::OFF_V + sv * T::TILE_BYTES, &tmV, b_v_full(sv), 0, h, j * 128, b);
+                        put_words(reinterpret_cast<uint32_t *>(gbase + T::OFF_MASK) + st * 8, w);
+                    const uint32_t dst = sbase + T::OFF_KV + st * 2 * T::TILE_BYTES;
+                    mbar_arrive_tx(b_kv_full(st), 2 * T::TILE_BYTES);
+                    tma_load_4d(dst, &tmK, b_kv_full(st), 0, h, j * 128, b);
+                    tma_load_4d(dst + T::TILE_BYTES, &tmV, b_kv_full(st), 0, h, j * 128, b);
                 }
-                v_done = k + 1;
+                kv_done = k + 1;
             }
         }
-    } else if (warp == 9 || warp == 10) {
-        // ------------------------------------------------------------------ MMA issuers
-        // Lane 0 of warp 9 issues every MMA of softmax warpgroup 0, lane 0 of warp 10 those
-        // of warpgroup 1.  Each keeps the Q K^T of the warpgroup's next step one step ahead
-        // of its P V: S(k+1) as soon as S(k) was read out of TMEM, P V(k) once P(k) is in
-        // shared memory.  All waits suspend the thread.
-        const int w = warp - 9;
-        if (lane == 0 && w < nW) {
+    } else if (warp == 9) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, CP, false, true);
             constexpr uint32_t SBO = 8 * T::ROWB;
+            bool ok = mbar_wait(b_q, 0, abort_flag, SITE_FWD_MMA);
+            int pending[2] = {-1, -1};
+            int pcount[2] = {0, 0};
             const int K = nJ * nb;
-            // steps of warpgroup w: slots s = w, w + 2, ... of key tile j, j = 0, 1, ...
-            auto step_after = [&](int k) {
-                const int s = k % nb, j = k / nb;
-                const int n = (s + 2 < nb) ? k + 2 : (j + 1) * nb + (s & 1);
-                return n < K ? n : K;
-            };
-            auto issue_s = [&](int k, int n) -> bool {   // n = how many S this warpgroup issued
-                if (n > 0 && !mbar_wait(b_s_free(w), (n - 1) & 1, abort_flag, SITE_FWD_MMA | (k << 12))) return false;
-                if (!mbar_wait(b_qk_full(k % QKS), (k / QKS) & 1, abort_flag, SITE_FWD_MMA | 0x10 | (k << 12))) return false;
-                tc_fence_after();
-                const uint32_t qa = sbase + T::OFF_QK + (k % QKS) * 2 * T::TILE_BYTES;
-                const uint32_t ka = qa + T::TILE_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < CP / 16; ++kk)
-                    umma_ss(tbase + w * 128, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
-                umma_commit(b_s_full(w));
-                umma_commit(b_qk_empty(k % QKS));
-                return true;
-            };
-            auto issue_pv = [&](int k, int n) -> bool {  // n = how many P V this warpgroup issued
-                if (!mbar_wait(b_p_full(w), n & 1, abort_flag, SITE_FWD_MMA | 0x20 | (k << 12))) return false;
-                if (!mbar_wait(b_v_full(k % VS), (k / VS) & 1, abort_flag, SITE_FWD_MMA | 0x30 | (k << 12))) return false;
-                tc_fence_after();
-                const int jp = k / nb, sp = k % nb;
-                const uint32_t pa = sbase + T::OFF_P + w * T::P_BYTES;
-                const uint32_t va = sbase + T::OFF_V + (k % VS) * T::TILE_BYTES;
+            auto issue_pv = [&](int kp) {
+                const int jp = kp / nb, sp = kp % nb, wp = sp & 1, stp = kp % KVS;
+                const uint32_t va = sbase + T::OFF_KV + stp * 2 * T::TILE_BYTES + T::TILE_BYTES;
+                const uint32_t d = tbase + 256 + sp * CP;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ss(tbase + 256 + sp * CP,
-                            sdesc(pa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128),
+                    umma_ts(d, tbase + wp * 128 + kk * 8,
                             sdesc(va + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), idesc_pv,
                             (jp > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(b_v_empty(k % VS));
-                umma_commit(b_p_free(w));
-                umma_commit(b_o_ready(sp));
-                return true;
+                umma_commit(b_kv_empty(stp));
             };
-            bool ok = true;
-            int k = w;                 // this warpgroup's first step
-            int n = 0;
-            if (k < K) ok = issue_s(k, n);
-            while (ok && k < K) {
-                const int kn = step_after(k);
-                // The producer reaches step kn only after the P V of step kn - 1 - VS (the
-                // V ring).  When that is this warpgroup's step k, its P V has to go first.
-                if (kn < K && kn - 1 - VS >= k) {
-                    ok = issue_pv(k, n);
-                    if (ok) ok = issue_s(kn, n + 1);
-                } else {
-                    if (kn < K) ok = issue_s(kn, n + 1);
-                    if (ok) ok = issue_pv(k, n);
+            // Serve whichever softmax warpgroup is ready: issue its pending P V as soon as
+            // its P is in TMEM, then its next Q K^T as soon as that step's K/V tile landed.
+            // Steps of warpgroup w: slots s = w, w + 2, ... of key tile j, j = 0, 1, ...
+            int next[2] = {0, 1 < nb ? 1 : K};
+            if (next[1] >= K) next[1] = K;
+            auto step_after = [&](int k) {
+                const int s = k % nb, j = k / nb;
+                return (s + 2 < nb) ? k + 2 : (j + 1) * nb + (s & 1);
+            };
+            long long t_idle = 0;
+            while (ok && (next[0] < K || next[1] < K || pending[0] >= 0 || pending[1] >= 0)) {
+                bool progress = false;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    if (pending[w] >= 0 && mbar_test(b_p_full(w), pcount[w] & 1)) {
+                        ++pcount[w];
+                        tc_fence_after();
+                        issue_pv(pending[w]);
+                        pending[w] = -1;
+                        progress = true;
+                    }
+                    const int k = next[w];
+                    if (pending[w] < 0 && k < K && mbar_test(b_kv_full(k % KVS), (k / KVS) & 1)) {
+                        tc_fence_after();
+                        const int s = k % nb, st = k % KVS;
+                        const uint32_t qa = sbase + T::OFF_Q + s * T::TILE_BYTES;
+                        const uint32_t ka = sbase + T::OFF_KV + st * 2 * T::TILE_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < CP / 16; ++kk)
+                            umma_ss(tbase + w * 128, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
+                                    sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
+                        umma_commit(b_s_full(w));
+                        pending[w] = k;
+                        int n2 = step_after(k);
+                        next[w] = n2 < K ? n2 : K;
+                        progress = true;
+                    }
                 }
-                k = kn;
-                ++n;
+                if (progress) {
+                    t_idle = 0;
+                } else if (t_idle == 0) {
+                    t_idle = sm_cycles();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (sm_cycles() - t_idle > kWaitLimitCycles) {
+                    *abort_flag = 1;
+                    watchdog_fire(SITE_FWD_MMA | ((next[0] < next[1] ? next[0] : next[1]) << 12));
+                    ok = false;
+                }
             }
-            if (ok) umma_commit(b_ofinal);   // each issuer arrives once (count = nW)
+            if (ok) umma_commit(b_ofinal);
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------------ softmax
@@ -330,7 +302,6 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const uint32_t tS = tbase + w * 128 + lane_off;
-        const uint32_t prow = sbase + T::OFF_P + w * T::P_BYTES + row * 128;
         float2 *stats = reinterpret_cast<float2 *>(gbase + T::OFF_STATS);
         const float2 sc2 = make_float2(a.scale, a.scale);
         const float2 l2e2 = make_float2(kLog2e, kLog2e);
@@ -339,27 +310,24 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int j = 0; j < nJ && ok; ++j) {
             bool bias_ready = false;
             for (int s = w; s < nb; s += 2) {
-                const int k = j * nb + s, st = k % VS;
+                const int k = j * nb + s, st = k % KVS;
                 ok = mbar_wait(b_s_full(w), ns & 1, abort_flag, SITE_FWD_SOFTMAX | (k << 12));
+                ++ns;
                 if (ok && !a.mask_shared)
-                    ok = mbar_wait(b_v_full(st), (k / VS) & 1, abort_flag, SITE_FWD_SOFTMAX);
+                    ok = mbar_wait(b_kv_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_SOFTMAX);
                 if (ok && !bias_ready) {
-                    ok = mbar_wait(b_bias_full(j % BS), (j / BS) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x10 | (k << 12));
+                    ok = mbar_wait(b_bias_full(j & 1), (j >> 1) & 1, abort_flag, SITE_FWD_SOFTMAX);
                     bias_ready = true;
                 }
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
 
-                // S of this row, then the buffer goes back to the MMA issuer
+                // logits of this row, in place: x = scale * S + bias (natural-log units)
                 uint32_t xr[128];
                 tmem_ld128(tS, xr);
-                tc_fence_before();
-                mbar_arrive(b_s_free(w));
-
-                // logits in place: x = scale * S + bias (natural-log units)
                 {
-                    const uint32_t bias_row = sbase + T::OFF_BIAS + (j % BS) * T::BIAS_BYTES + row * 128;
+                    const uint32_t bias_row = sbase + T::OFF_BIAS + (j & 1) * T::BIAS_BYTES + row * 128;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {  // 16-byte chunk q holds keys 8q .. 8q+7
                         uint4 bw = make_uint4(0, 0, 0, 0);
@@ -378,7 +346,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
                 float *x = reinterpret_cast<float *>(xr);
                 const uint32_t *mw = a.mask_shared
-                                         ? reinterpret_cast<const uint32_t *>(gbase + T::OFF_BMASK) + (j % BS) * 8
+                                         ? reinterpret_cast<const uint32_t *>(gbase + T::OFF_BMASK) + (j & 1) * 8
                                          : reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
                 if (mw[4] == 0u) {
 #pragma unroll
@@ -414,47 +382,35 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const float nm = (m_use == -INFINITY) ? 0.f : -m_use * kLog2e;
                 const float2 nm2 = make_float2(nm, nm);
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-                // P = exp(x - m) in bf16, written over x as packed pairs
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float2 t = ffma2(make_float2(x[2 * c], x[2 * c + 1]), l2e2, nm2);
-                    const float2 pv = make_float2(ex2(t.x), ex2(t.y));
-                    if (c & 1) acc1 = fadd2(acc1, pv);
-                    else acc0 = fadd2(acc0, pv);
-                    xr[c] = pack_bf16x2(pv.x, pv.y);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t p[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int i2 = hf * 64 + 2 * c;
+                        const float2 t = ffma2(make_float2(x[i2], x[i2 + 1]), l2e2, nm2);
+                        const float2 pv = make_float2(ex2(t.x), ex2(t.y));
+                        if (c & 1) acc1 = fadd2(acc1, pv);
+                        else acc0 = fadd2(acc0, pv);
+                        p[c] = pack_bf16x2(pv.x, pv.y);
+                    }
+                    tmem_st32(tS + hf * 32, p);
                 }
                 const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-                // the previous P of this warpgroup must have been consumed by its P V
-                if (ns > 0) {
-                    ok = mbar_wait(b_p_free(w), (ns - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x20 | (k << 12));
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                }
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    sts128(prow + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4),
-                           make_uint4(xr[4 * q], xr[4 * q + 1], xr[4 * q + 2], xr[4 * q + 3]));
-                // generic-proxy writes -> visible to the tensor core's async proxy
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                // O[s] must be rescaled before this step's P V, after the previous one
+                // O must be rescaled before P V of this step is issued, i.e. before p_full
                 if (__any_sync(0xffffffffu, resc)) {
-                    ok = mbar_wait(b_o_ready(s), (j - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x30 | (k << 12));
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
                     const uint32_t tO = tbase + 256 + s * CP + lane_off;
                     uint32_t o[CP];
                     tmem_ld_cols<CP>(tO, o);
 #pragma unroll
                     for (int c = 0; c < CP; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
                     tmem_st_cols<CP>(tO, o);
-                    tmem_wait_st();
-                    tc_fence_before();
                 }
+                tmem_wait_st();
                 stats[s * 128 + row] = make_float2(m_use, l_prev * alpha + sum);
+                tc_fence_before();
                 mbar_arrive(b_p_full(w));
-                ++ns;
-                if (s + 2 >= nb) mbar_arrive(b_bias_empty(j % BS));
+                if (s + 2 >= nb) mbar_arrive(b_bias_empty(j & 1));
             }
         }
         // ------------------------------------------------------------------ epilogue
@@ -524,14 +480,14 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // Some wait ran out.  Every role has stopped; before shared memory and TMEM are
         // released, let the copies and MMAs already issued finish (bounded waits).
         if (warp == 8 && lane == 0) {
-            for (int kk = max(0, qk_done - QKS); kk < qk_done; ++kk)
-                if (kk != a.skip_step) mbar_wait_drain(b_qk_full(kk % QKS), (kk / QKS) & 1);
-            for (int kk = max(0, v_done - VS); kk < v_done; ++kk) mbar_wait_drain(b_v_full(kk % VS), (kk / VS) & 1);
-            for (int jj = max(0, n_bias - BS); jj < n_bias; ++jj) mbar_wait_drain(b_bias_full(jj % BS), (jj / BS) & 1);
+            mbar_wait_drain(b_q, 0);
+            for (int kk = max(0, kv_done - KVS); kk < kv_done; ++kk)
+                if (kk != a.skip_step) mbar_wait_drain(b_kv_full(kk % KVS), (kk / KVS) & 1);
+            for (int jj = max(0, n_bias - 2); jj < n_bias; ++jj) mbar_wait_drain(b_bias_full(jj & 1), (jj >> 1) & 1);
         }
-        if ((warp == 9 || warp == 10) && lane == 0 && warp - 9 < nW) {
-            umma_commit(b_drain(warp - 9));
-            mbar_wait_drain(b_drain(warp - 9), 0);
+        if (warp == 9 && lane == 0) {
+            umma_commit(b_drain);
+            mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
         __syncthreads();
