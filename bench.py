@@ -80,10 +80,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {"pba_fwd_kernel": "pba_fwd.cuh"}   # every other kernel lives in pba_bwd.cuh
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources one kernel is compiled from: its own file and the shared device
+    header (launch configuration in the API file is not covered)."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc")
-    for name in sorted(os.listdir(cdir)):
+    for name in (KERNEL_SOURCES.get(kernel, "pba_bwd.cuh"), "pba_device.cuh"):
         with open(os.path.join(cdir, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -97,10 +102,10 @@ def ncu_traffic(kernel: str, workload: str):
         return None
     with open(p) as fh:
         d = json.load(fh)
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     ent = d.get("kernels", {}).get(kernel, {}).get(workload)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    if ent is None or ent.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return ent.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------------------

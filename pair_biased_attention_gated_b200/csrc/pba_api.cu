@@ -221,12 +221,8 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.B = d->B; a.H = d->H; a.Nq = d->Nq; a.Nk = d->Nk; a.C = d->C;
     a.nI = (d->Nq + 127) / 128;
     a.nJ = (d->Nk + 127) / 128;
-    // rows per CTA: as many as TMEM holds, fewer when that would leave SMs idle
+    a.nChunks = (d->B + T::BC - 1) / T::BC;
     const long long tiles = (long long)a.nI * d->H;
-    int bc = T::BCMAX;
-    while (bc > 2 && tiles * ((d->B + bc - 1) / bc) < 2LL * 148) bc /= 2;
-    a.bc = bc;
-    a.nChunks = (d->B + bc - 1) / bc;
     a.scale = eff_scale(d);
     a.has_bias = bias != nullptr;
     a.mask = mask;
@@ -239,6 +235,11 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.lse = lse;
     a.skip_step = g_debug_skip_step;
     if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
+    // two CTAs per SM need (almost) all of the unified L1 / shared memory as shared memory
+    cudaError_t ce = cudaFuncSetAttribute(pba::pba_fwd_kernel<CP>,
+                                          cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          cudaSharedmemCarveoutMaxShared);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute (carveout)");
     const long long grid = tiles * a.nChunks;
     {
         ProfScope ps(K_FWD, stream);
@@ -577,6 +578,9 @@ pba_status pba_device_status(void *stream) {
         cudaMemcpyFromSymbol(&site, pba::g_pba_watchdog_site, sizeof(site));
         cudaMemcpyToSymbol(pba::g_pba_watchdog, &zero, sizeof(zero));
         cudaMemcpyToSymbol(pba::g_pba_watchdog_site, &zero, sizeof(zero));
+        if ((site & 0xFFFu) == pba::SITE_FWD_ALIGN)
+            return fail(PBA_ERR_UNSUPPORTED, "forward kernel refused: dynamic shared memory "
+                                             "is not 1024-byte aligned");
         return fail(PBA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (site 0x%x)", site);
     }
     return PBA_OK;

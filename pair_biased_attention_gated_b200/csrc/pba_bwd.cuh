@@ -471,7 +471,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                                              pack_bf16x2(ds[c8 * 8 + 6], ds[c8 * 8 + 7])));
             }
             // generic-proxy writes -> visible to the tensor core's async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_proxy_async();
             mbar_arrive(b_ps_full);
             if (t > 0) ok = flush_dq(t - 1);
         }
