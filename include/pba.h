@@ -161,7 +161,7 @@ int pba_profile_read(pba_kernel_stat *out, int max);
 
 /*
  * Test hook for the device watchdog (no production use).  With step >= 0, the next
- * pba_fwd calls make their TMA producer skip the K/V load of that step of every CTA, so
+ * pba_fwd calls make their TMA producer skip the K load of that step of every CTA, so
  * the barrier it would have completed never does: the MMA issuer's bounded wait runs
  * out (about one second), every role of the CTA drains what it issued and returns, and
  * pba_device_status() then reports PBA_ERR_TIMEOUT.  No GPU fault is raised and the

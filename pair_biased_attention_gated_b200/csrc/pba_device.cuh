@@ -62,6 +62,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same, but a thread whose phase is not complete is suspended (woken when the phase
+// completes) for up to `hint_ns` before the instruction gives up, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kSuspendHintNs = 20000;
+
 // Bounded wait for the phase with the given parity to complete.  Returns false (and
 // raises the CTA's abort flag and the device watchdog) if it does not complete within
 // kWaitLimitCycles, or if another role of the CTA has already aborted.
@@ -72,7 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = sm_cycles();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
         if (*abort_flag) return false;
         if (sm_cycles() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;

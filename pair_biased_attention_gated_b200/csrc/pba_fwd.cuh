@@ -9,14 +9,18 @@
 // SM, so one CTA's prologue and epilogue overlap the other's main loop.  The loop runs over
 // key tiles j (outer) and the chunk's rows b (inner): each 128x128 bias tile is moved into
 // shared memory once and reused by all rows of the chunk.  The chunk's Q tiles stay
-// resident; K/V tiles stream through a ring.
+// resident; K and V tiles stream through two rings: a K stage is refilled as soon as its
+// Q K^T is done, a V stage only after its P V.
 //
 // Warp roles (256 threads, two warpgroups):
 //   warps 0-3  softmax and epilogue: thread = query row = TMEM lane
 //   warp 4     TMA producer (Q, K, V, bias tiles) and per-row key-mask words
-//   warp 5     TMEM allocator and, on lane 0, the tcgen05 MMA issuer
-//   warps 6-7  fold the key mask into each bias tile (masked keys -> -inf), or build the
+//   warp 5     TMEM allocator and, on lane 0, the issuer of the Q K^T MMAs
+//   warp 6     lane 0 issues the P V MMAs
+//   warp 7     folds the key mask into each bias tile (masked keys -> -inf), or builds the
 //              tile when there is no bias, so the softmax never tests mask bits
+// A tcgen05.mma issue occupies the issuing thread about as long as the MMA runs, so the
+// two products have separate issuers: Q K^T of the next step never queues behind P V.
 // The second warpgroup hands registers to the first through setmaxnreg.
 //
 // Tensor memory (256 columns): S [0,128), P as packed bf16 [128,192), then one
@@ -42,21 +46,22 @@ struct FwdArgs {
     __nv_bfloat16 *out;
     long long so0, so1, so2;
     float *lse;
-    int skip_step;   // test hook: the producer skips this step's K/V load (-1: never)
+    int skip_step;   // test hook: the producer skips this step's K load (-1: never)
 };
 
 template <int CP>
 struct FwdTraits {
     static constexpr int BC = 64 / CP;                         // rows b per CTA (O slots)
-    static constexpr int KVS = (CP == 16) ? 3 : 2;             // K/V ring stages
+    static constexpr int KVS = (CP == 16) ? 3 : 2;             // stages of each of the K and V rings
     static constexpr int BS = (CP == 64) ? 1 : 2;              // bias tile buffers
     static constexpr int TILE_BYTES = 128 * CP * 2;            // Q, K or V tile
     static constexpr int BIAS_BYTES = 128 * 128 * 2;           // two 64-key halves
     static constexpr int OFF_BIAS = 0;                         // 1024-byte aligned (SW128)
     static constexpr int OFF_Q = OFF_BIAS + BS * BIAS_BYTES;
-    static constexpr int OFF_KV = OFF_Q + BC * TILE_BYTES;
-    static constexpr int OFF_MASK = OFF_KV + KVS * 2 * TILE_BYTES;  // u32 [KVS][8] per-row words
-    static constexpr int NBAR = 1 + 2 * KVS + 3 * BS + 6;
+    static constexpr int OFF_K = OFF_Q + BC * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KVS * TILE_BYTES;
+    static constexpr int OFF_MASK = OFF_V + KVS * TILE_BYTES;  // u32 [KVS][8] per-row words (V ring)
+    static constexpr int NBAR = 1 + 4 * KVS + 3 * BS + 6;
     static constexpr int OFF_BAR = OFF_MASK + KVS * 32;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // TMEM base, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -112,12 +117,15 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
     const uint32_t b_q = smem_u32(&bars[0]);
-    auto b_kv_full = [&](int st) { return smem_u32(&bars[1 + st]); };
-    auto b_kv_empty = [&](int st) { return smem_u32(&bars[1 + KVS + st]); };
-    auto b_bias_full = [&](int x) { return smem_u32(&bars[1 + 2 * KVS + x]); };    // landed
-    auto b_bias_ready = [&](int x) { return smem_u32(&bars[1 + 2 * KVS + BS + x]); }; // folded
-    auto b_bias_empty = [&](int x) { return smem_u32(&bars[1 + 2 * KVS + 2 * BS + x]); };
-    constexpr int OB = 1 + 2 * KVS + 3 * BS;
+    auto b_k_full = [&](int st) { return smem_u32(&bars[1 + st]); };
+    auto b_k_empty = [&](int st) { return smem_u32(&bars[1 + KVS + st]); };
+    auto b_v_full = [&](int st) { return smem_u32(&bars[1 + 2 * KVS + st]); };
+    auto b_v_empty = [&](int st) { return smem_u32(&bars[1 + 3 * KVS + st]); };
+    constexpr int OBB = 1 + 4 * KVS;
+    auto b_bias_full = [&](int x) { return smem_u32(&bars[OBB + x]); };            // landed
+    auto b_bias_ready = [&](int x) { return smem_u32(&bars[OBB + BS + x]); };      // folded
+    auto b_bias_empty = [&](int x) { return smem_u32(&bars[OBB + 2 * BS + x]); };
+    constexpr int OB = OBB + 3 * BS;
     const uint32_t b_s_full = smem_u32(&bars[OB + 0]);   // Q K^T in S
     const uint32_t b_s_free = smem_u32(&bars[OB + 1]);   // S read out
     const uint32_t b_p_full = smem_u32(&bars[OB + 2]);   // P in TMEM, O rescaled
@@ -142,12 +150,14 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (threadIdx.x == 0) {
         mbar_init(b_q, 1);
         for (int st = 0; st < KVS; ++st) {
-            mbar_init(b_kv_full(st), 1);
-            mbar_init(b_kv_empty(st), 1);
+            mbar_init(b_k_full(st), 1);
+            mbar_init(b_k_empty(st), 1);
+            mbar_init(b_v_full(st), 1);
+            mbar_init(b_v_empty(st), 1);
         }
         for (int x = 0; x < BS; ++x) {
             mbar_init(b_bias_full(x), 1);
-            mbar_init(b_bias_ready(x), 64);
+            mbar_init(b_bias_ready(x), 32);
             mbar_init(b_bias_empty(x), 128);
         }
         mbar_init(b_s_full, 1);
@@ -155,7 +165,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_init(b_p_full, 128);
         mbar_init(b_p_free, 1);
         mbar_init(b_ofinal, 1);
-        mbar_init(b_drain, 1);
+        mbar_init(b_drain, 2);   // one commit from each issuer
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -168,9 +178,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tbase = *s_tmem_base;
 
-    // K/V loads issued for steps [0, kv_done), bias tiles [0, n_bias): what has to land
-    // before the CTA may exit after an abort
-    int kv_done = 0, n_bias = 0;
+    // K loads issued for steps [0, k_done), V loads for [0, v_done), bias tiles
+    // [0, n_bias): what has to land before the CTA may exit after an abort
+    int k_done = 0, v_done = 0, n_bias = 0;
 
     if (warp >= 4) reg_dealloc<T::REGS_OTHER>();   // the whole second warpgroup, same point
     if (warp == 4) {
@@ -184,15 +194,18 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int s = 0; s < nb; ++s)
                 tma_load_4d(sbase + T::OFF_Q + s * T::TILE_BYTES, &tmQ, b_q, 0, h, i0, b0 + s);
         }
-        bool ok = true;
-        int k = 0;
-        for (int j = 0; j < nJ && ok; ++j) {
+        // Load order: B(0), K(0), then for every step k: K(k + 1), V(k), and the bias tile
+        // of the next key tile once step k + 1 starts one.  K runs a step ahead of V; a bias
+        // tile (which waits for the softmax to leave the buffer's previous tile) comes after
+        // the V loads whose mask words that softmax may be waiting for.
+        auto load_bias = [&](int j) -> bool {
             const int bs = j % BS;
+            bool ok = true;
             if (j >= BS)
                 ok = mbar_wait(b_bias_empty(bs), ((j / BS) - 1) & 1, abort_flag,
                                SITE_FWD_PROD | 0x20 | (j << 12));
             ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
+            if (!ok) return false;
             if (lane == 0) {
                 if (a.has_bias) {
                     const uint32_t dst = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
@@ -204,98 +217,113 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
             n_bias = j + 1;
-            for (int s = 0; s < nb; ++s, ++k) {
-                const int st = k % KVS, use = k / KVS;
-                if (use >= 1)
-                    ok = mbar_wait(b_kv_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | (k << 12));
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                if (row_mask) {
-                    // words of row b: word q bit t <-> key 128 j + 32 q + t attended
-                    uint32_t w[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int key = j * 128 + q * 32 + lane;
-                        const bool valid = key < a.Nk && a.mask[(long long)(b0 + s) * a.smask_b + key] != 0;
-                        w[q] = __ballot_sync(0xffffffffu, valid);
-                    }
-                    if (lane == 0) {
-                        uint32_t *mw = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MASK) + st * 8;
-                        mw[0] = w[0];
-                        mw[1] = w[1];
-                        mw[2] = w[2];
-                        mw[3] = w[3];
-                        mw[4] = (w[0] & w[1] & w[2] & w[3]) == 0xffffffffu;
-                    }
-                }
-                if (lane == 0 && k != a.skip_step) {
-                    const uint32_t dst = sbase + T::OFF_KV + st * 2 * T::TILE_BYTES;
-                    mbar_arrive_tx(b_kv_full(st), 2 * T::TILE_BYTES);
-                    tma_load_4d(dst, &tmK, b_kv_full(st), 0, h, j * 128, b0 + s);
-                    tma_load_4d(dst + T::TILE_BYTES, &tmV, b_kv_full(st), 0, h, j * 128, b0 + s);
-                }
-                kv_done = k + 1;
+            return true;
+        };
+        auto load_k = [&](int k) -> bool {
+            const int st = k % KVS, use = k / KVS;
+            bool ok = true;
+            if (use >= 1)
+                ok = mbar_wait(b_k_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | (k << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return false;
+            if (lane == 0 && k != a.skip_step) {
+                mbar_arrive_tx(b_k_full(st), T::TILE_BYTES);
+                tma_load_4d(sbase + T::OFF_K + st * T::TILE_BYTES, &tmK, b_k_full(st), 0, h,
+                            (k / nb) * 128, b0 + k % nb);
             }
+            k_done = k + 1;
+            return true;
+        };
+        auto load_v = [&](int k) -> bool {
+            const int st = k % KVS, use = k / KVS;
+            bool ok = true;
+            if (use >= 1)
+                ok = mbar_wait(b_v_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | 0x10 | (k << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return false;
+            const int j = k / nb, b = b0 + k % nb;
+            if (row_mask) {
+                // words of row b: word q bit t <-> key 128 j + 32 q + t attended
+                uint32_t w[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int key = j * 128 + q * 32 + lane;
+                    const bool valid = key < a.Nk && a.mask[(long long)b * a.smask_b + key] != 0;
+                    w[q] = __ballot_sync(0xffffffffu, valid);
+                }
+                if (lane == 0) {
+                    uint32_t *mw = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MASK) + st * 8;
+                    mw[0] = w[0];
+                    mw[1] = w[1];
+                    mw[2] = w[2];
+                    mw[3] = w[3];
+                    mw[4] = (w[0] & w[1] & w[2] & w[3]) == 0xffffffffu;
+                }
+            }
+            if (lane == 0) {
+                mbar_arrive_tx(b_v_full(st), T::TILE_BYTES);
+                tma_load_4d(sbase + T::OFF_V + st * T::TILE_BYTES, &tmV, b_v_full(st), 0, h, j * 128, b);
+            }
+            v_done = k + 1;
+            return true;
+        };
+        bool ok = K > 0 ? (load_bias(0) && load_k(0)) : true;
+        for (int k = 0; k < K && ok; ++k) {
+            if (k + 1 < K) ok = load_k(k + 1);
+            if (ok) ok = load_v(k);
+            if (ok && k + 1 < K && (k + 1) % nb == 0) ok = load_bias((k + 1) / nb);
         }
     } else if (warp == 5) {
-        // ------------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------------ Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, CP, false, true);
             constexpr uint32_t SBO = 8 * T::ROWB;
             bool ok = mbar_wait(b_q, 0, abort_flag, SITE_FWD_MMA);
-            // Q K^T of step kq needs its K/V tile and S read out by the softmax of step
-            // kq - 1; P V of step kp needs P of step kp.  Issue whichever is ready.
-            int kq = 0, kp = 0;
-            long long t_idle = 0;
-            while (ok && kp < K) {
-                bool progress = false;
-                if (kq < K && (kq == 0 || mbar_test(b_s_free, (kq - 1) & 1)) &&
-                    mbar_test(b_kv_full(kq % KVS), (kq / KVS) & 1)) {
-                    tc_fence_after();
-                    const int s = kq % nb, st = kq % KVS;
-                    const uint32_t qa = sbase + T::OFF_Q + s * T::TILE_BYTES;
-                    const uint32_t ka = sbase + T::OFF_KV + st * 2 * T::TILE_BYTES;
+            // step k: S must have been read out by the softmax of step k - 1
+            for (int k = 0; k < K && ok; ++k) {
+                const int s = k % nb, st = k % KVS;
+                if (k > 0) ok = mbar_wait(b_s_free, (k - 1) & 1, abort_flag, SITE_FWD_MMA | 0x20 | (k << 12));
+                if (ok) ok = mbar_wait(b_k_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x10 | (k << 12));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t qa = sbase + T::OFF_Q + s * T::TILE_BYTES;
+                const uint32_t ka = sbase + T::OFF_K + st * T::TILE_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < CP / 16; ++kk)
-                        umma_ss(tbase + T::T_S, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
-                                sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
-                    umma_commit(b_s_full);
-                    ++kq;
-                    progress = true;
-                }
-                if (kp < kq && mbar_test(b_p_full, kp & 1)) {
-                    tc_fence_after();
-                    const int jp = kp / nb, sp = kp % nb, stp = kp % KVS;
-                    const uint32_t va = sbase + T::OFF_KV + stp * 2 * T::TILE_BYTES + T::TILE_BYTES;
-                    const uint32_t d = tbase + T::T_O + sp * CP;
+                for (int kk = 0; kk < CP / 16; ++kk)
+                    umma_ss(tbase + T::T_S, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
+                            sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
+                umma_commit(b_s_full);
+                umma_commit(b_k_empty(st));
+            }
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------------ P V issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_pv = idesc_bf16(128, CP, false, true);
+            constexpr uint32_t SBO = 8 * T::ROWB;
+            bool ok = true;
+            // step k: P of step k written (and O[s] rescaled) by the softmax, V landed
+            for (int k = 0; k < K && ok; ++k) {
+                const int j = k / nb, s = k % nb, st = k % KVS;
+                ok = mbar_wait(b_p_full, k & 1, abort_flag, SITE_FWD_MMA | 0x30 | (k << 12));
+                if (ok) ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x40 | (k << 12));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t va = sbase + T::OFF_V + st * T::TILE_BYTES;
+                const uint32_t d = tbase + T::T_O + s * CP;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(d, tbase + T::T_P + kk * 8,
-                                sdesc(va + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), idesc_pv,
-                                (jp > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(b_p_free);
-                    umma_commit(b_kv_empty(stp));
-                    ++kp;
-                    progress = true;
-                }
-                if (progress) {
-                    t_idle = 0;
-                } else if (t_idle == 0) {
-                    t_idle = sm_cycles();
-                } else if (*abort_flag) {
-                    ok = false;
-                } else if (sm_cycles() - t_idle > kWaitLimitCycles) {
-                    *abort_flag = 1;
-                    watchdog_fire(SITE_FWD_MMA | (kp << 12));
-                    ok = false;
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(d, tbase + T::T_P + kk * 8,
+                            sdesc(va + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), idesc_pv,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(b_p_free);
+                umma_commit(b_v_empty(st));
             }
             if (ok) umma_commit(b_ofinal);
         }
-    } else if (warp >= 6) {
+    } else if (warp == 7) {
         // ------------------------------------------------------------------ mask fold
-        const int t = threadIdx.x - 192;   // rows t and t + 64 of every bias tile
+        const int t = lane;   // rows t, t + 32, t + 64, t + 96 of every bias tile
         bool ok = true;
         for (int j = 0; j < nJ && ok; ++j) {
             const int bs = j % BS;
@@ -320,8 +348,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         while (m) {
                             const int c = q * 32 + __ffs(m) - 1;
                             m &= m - 1;
-                            *reinterpret_cast<uint16_t *>(tile + bias_off(t, c)) = 0xFF80u;
-                            *reinterpret_cast<uint16_t *>(tile + bias_off(t + 64, c)) = 0xFF80u;
+#pragma unroll
+                            for (int r = t; r < 128; r += 32)
+                                *reinterpret_cast<uint16_t *>(tile + bias_off(r, c)) = 0xFF80u;
                         }
                     }
                 }
@@ -341,8 +370,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     }
                     const uint4 val = make_uint4(v4[0], v4[1], v4[2], v4[3]);
                     const uint32_t tb = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
-                    sts128(tb + bias_off(t, ch * 8), val);
-                    sts128(tb + bias_off(t + 64, ch * 8), val);
+#pragma unroll
+                    for (int r = t; r < 128; r += 32) sts128(tb + bias_off(r, ch * 8), val);
                 }
             }
             // these generic writes precede a later TMA refill of the same buffer
@@ -374,8 +403,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (ok && s == 0)
                     ok = mbar_wait(b_bias_ready(bs), (j / BS) & 1, abort_flag,
                                    SITE_FWD_SOFTMAX | 0x10 | (k << 12));
-                if (ok && row_mask)
-                    ok = mbar_wait(b_kv_full(st), (k / KVS) & 1, abort_flag,
+                if (ok && row_mask)   // this step's mask words come with its V tile
+                    ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag,
                                    SITE_FWD_SOFTMAX | 0x20 | (k << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -556,13 +585,15 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // released, let the copies and MMAs already issued finish (bounded waits).
         if (warp == 4 && lane == 0) {
             mbar_wait_drain(b_q, 0);
-            for (int kk = max(0, kv_done - KVS); kk < kv_done; ++kk)
-                if (kk != a.skip_step) mbar_wait_drain(b_kv_full(kk % KVS), (kk / KVS) & 1);
+            for (int kk = max(0, k_done - KVS); kk < k_done; ++kk)
+                if (kk != a.skip_step) mbar_wait_drain(b_k_full(kk % KVS), (kk / KVS) & 1);
+            for (int kk = max(0, v_done - KVS); kk < v_done; ++kk)
+                mbar_wait_drain(b_v_full(kk % KVS), (kk / KVS) & 1);
             for (int jj = max(0, n_bias - BS); jj < n_bias; ++jj)
                 mbar_wait_drain(b_bias_full(jj % BS), (jj / BS) & 1);
         }
-        if (warp == 5 && lane == 0) {
-            umma_commit(b_drain);
+        if ((warp == 5 || warp == 6) && lane == 0) {
+            umma_commit(b_drain);   // each issuer's own MMAs
             mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
