@@ -251,6 +251,8 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
 }
 
 // ---------------------------------------------------------------------------- backward
+constexpr long long kSmCount = 148;   // SMs of a B200
+
 struct BwdPlan {
     int nI, nJ, NqPad, NkPad, splits, rows_per_split;
     size_t off_rs, off_doa, off_dq, off_part, total;
@@ -265,14 +267,26 @@ BwdPlan plan_bwd(const pba_dims *d) {
     p.NqPad = p.nI * 128;
     p.NkPad = p.nJ * 128;
     // splits of the broadcast rows for the dbias kernel: a fixed function of the sizes,
-    // so the reduction order (and every bit of dbias) depends on nothing else
+    // so the reduction order (and every bit of dbias) depends on nothing else.  A CTA
+    // handles one (head, query tile, key tile, split); its time grows with the rows of its
+    // split plus a fixed cost (bias tile, pipeline fill, the partial tile's store) of about
+    // three rows, so pick the split count that minimises waves x (rows + 3) on 148 SMs.
     const long long tiles = (long long)d->H * p.nI * p.nJ;
-    long long splits = tiles > 0 ? (2LL * 148 + tiles - 1) / tiles : 1;
-    if (splits < 1) splits = 1;
-    if (splits > d->B) splits = d->B > 0 ? d->B : 1;
-    if (splits > 64) splits = 64;
-    p.rows_per_split = d->B > 0 ? (int)((d->B + splits - 1) / splits) : 1;
-    p.splits = d->B > 0 ? (d->B + p.rows_per_split - 1) / p.rows_per_split : 1;
+    const long long maxs = d->B < 64 ? (d->B > 0 ? d->B : 1) : 64;
+    long long best_cost = -1;
+    p.splits = 1;
+    p.rows_per_split = d->B > 0 ? d->B : 1;
+    for (long long sp = 1; sp <= maxs; ++sp) {
+        const long long rows = d->B > 0 ? (d->B + sp - 1) / sp : 1;
+        const long long actual = d->B > 0 ? (d->B + rows - 1) / rows : 1;
+        const long long waves = (tiles * actual + kSmCount - 1) / kSmCount;
+        const long long cost = waves * (rows + 3);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            p.splits = (int)actual;
+            p.rows_per_split = (int)rows;
+        }
+    }
     const size_t rows = (size_t)d->B * d->H * p.NqPad;
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
     p.off_rs = 0;
@@ -297,6 +311,15 @@ __global__ void zero_rows_kernel(__nv_bfloat16 *dk, __nv_bfloat16 *dv, pba::BwdA
         *reinterpret_cast<uint4 *>(dk + b * a.sk0 + (long long)j * a.sk1 + h * a.sk2 + c8 * 8) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4 *>(dv + b * a.sv0 + (long long)j * a.sv1 + h * a.sv2 + c8 * 8) = make_uint4(0, 0, 0, 0);
     }
+}
+
+// SMs of the current device (one CTA each for the persistent kernels)
+long long num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return kSmCount;
+    return n;
 }
 
 unsigned grid_for(long long n, int threads) {
@@ -387,7 +410,9 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_pre_kernel launch");
     if (pl.nJ > 0) {
         if ((st = set_smem(pba::pba_bwd_main_kernel<CP>, MT::SMEM_BYTES)) != PBA_OK) return st;
-        const long long grid = (long long)d->B * d->H * pl.nJ;
+        // persistent: one CTA per SM (at most one per item)
+        const long long items = (long long)d->B * d->H * pl.nJ;
+        const long long grid = items < num_sms() ? items : num_sms();
         {
             ProfScope ps(K_BWD_MAIN, s);
             pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 320, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);

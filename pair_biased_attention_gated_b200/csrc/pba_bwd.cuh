@@ -178,28 +178,40 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
 
 // ---------------------------------------------------------------------------------------
 // main backward kernel: dQ, dK, dV
+//
+// Persistent: one CTA per SM walks the items (b, h, 128-key tile) n = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; an item's steps are its query tiles.  The step pipeline
+// (S/dP -> P/dS -> dV, dK, dQ) runs on across item boundaries: the next item's K/V tiles
+// load into the other stage while the current item finishes, and dK/dV accumulate in one
+// of two TMEM buffers, so an item's dK/dV epilogue (written by the element-wise warps right
+// after the next item's first step) overlaps the next item's MMAs.
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct BwdTraits {
     static constexpr int QS = 2;                                // Q/dOa/row-stat stages
     static constexpr int BS = (CP == 64) ? 1 : 2;               // bias stages
+    static constexpr int KVB = (CP == 64) ? 1 : 2;              // K/V stages (items)
+    static constexpr int DKB = (CP == 64) ? 1 : 2;              // dK/dV TMEM buffers (items)
     static constexpr int TILE_BYTES = 128 * CP * 2;
     static constexpr int BIAS_BYTES = 128 * 128 * 2;
     static constexpr int PS_BYTES = 128 * 128 * 2;              // P or dS tile (bf16)
-    static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = OFF_K + TILE_BYTES;
-    static constexpr int OFF_Q = OFF_V + TILE_BYTES;            // + st * 2 * TILE_BYTES
+    static constexpr int OFF_K = 0;                             // + x * TILE_BYTES
+    static constexpr int OFF_V = OFF_K + KVB * TILE_BYTES;      // + x * TILE_BYTES
+    static constexpr int OFF_Q = OFF_V + KVB * TILE_BYTES;      // + st * 2 * TILE_BYTES
     static constexpr int OFF_P = OFF_Q + QS * 2 * TILE_BYTES;
     static constexpr int OFF_DS = OFF_P + PS_BYTES;
     static constexpr int OFF_BIAS = OFF_DS + PS_BYTES;          // + bs * BIAS_BYTES
     static constexpr int OFF_RS = OFF_BIAS + BS * BIAS_BYTES;   // float2 [QS][128]
-    static constexpr int OFF_MASK = OFF_RS + QS * 1024;         // u32 [8]
-    static constexpr int SMEM_BYTES = OFF_MASK + 64 + 1024;
+    static constexpr int OFF_MASK = OFF_RS + QS * 1024;         // u32 [KVB][8]
+    static constexpr int SMEM_BYTES = OFF_MASK + KVB * 32 + 1024;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
     static constexpr uint32_t ROWB = CP * 2;
-    // TMEM columns
-    static constexpr int T_S = 0, T_DP = 128, T_DK = 256, T_DV = 256 + CP, T_DQ = 256 + 2 * CP;
+    // TMEM columns: S, dP, then per dK/dV buffer x: dK at T_DK + 2 CP x, dV after it, then
+    // the two dQ buffers
+    static constexpr int T_S = 0, T_DP = 128, T_DK = 256, T_DQ = 256 + DKB * 2 * CP;
+    static_assert(T_DQ + 2 * CP <= 512, "TMEM");
 };
+static_assert(BwdTraits<64>::SMEM_BYTES <= 232448 && BwdTraits<32>::SMEM_BYTES <= 232448, "smem");
 
 template <int CP>
 __global__ void __launch_bounds__(320, 1)
@@ -207,18 +219,16 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
     using T = BwdTraits<CP>;
-    constexpr int QS = T::QS, BS = T::BS;
+    constexpr int QS = T::QS, BS = T::BS, KVB = T::KVB, DKB = T::DKB;
     extern __shared__ uint8_t dsmem[];
-    __shared__ __align__(8) uint64_t bars[16 + 2 * QS + 2 * BS];
+    __shared__ __align__(8) uint64_t bars[16 + 2 * QS + 2 * BS + 2 * KVB + 2 * DKB];
     __shared__ uint32_t s_tmem_base;
     __shared__ int s_abort;
 
-    const uint32_t b_kv = smem_u32(&bars[0]);
     const uint32_t b_sd_full = smem_u32(&bars[1]);
     const uint32_t b_sd_free = smem_u32(&bars[2]);
     const uint32_t b_ps_full = smem_u32(&bars[3]);
     const uint32_t b_ps_free = smem_u32(&bars[4]);
-    const uint32_t b_done = smem_u32(&bars[5]);
     const uint32_t b_drain = smem_u32(&bars[6]);
     auto b_dq_full = [&](int x) { return smem_u32(&bars[8 + x]); };
     auto b_dq_free = [&](int x) { return smem_u32(&bars[10 + x]); };
@@ -226,27 +236,38 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     auto b_q_empty = [&](int x) { return smem_u32(&bars[16 + QS + x]); };
     auto b_bias_full = [&](int x) { return smem_u32(&bars[16 + 2 * QS + x]); };
     auto b_bias_empty = [&](int x) { return smem_u32(&bars[16 + 2 * QS + BS + x]); };
+    constexpr int OK_ = 16 + 2 * QS + 2 * BS;
+    auto b_kv_full = [&](int x) { return smem_u32(&bars[OK_ + x]); };          // K, V, mask words
+    auto b_kv_empty = [&](int x) { return smem_u32(&bars[OK_ + KVB + x]); };   // item's MMAs done
+    auto b_dkv_full = [&](int x) { return smem_u32(&bars[OK_ + 2 * KVB + x]); };        // dK/dV final
+    auto b_dkv_free = [&](int x) { return smem_u32(&bars[OK_ + 2 * KVB + DKB + x]); };  // read out
 
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *gbase = dsmem + (sbase - raw);
 
     const int warp = warp_id(), lane = lane_id();
-    int idx = blockIdx.x;
-    const int jt = idx % a.nJ;
-    idx /= a.nJ;
-    const int h = idx % a.H;
-    const int b = idx / a.H;
-    const int j0 = jt * 128;
     const int nI = a.nI;
+    const long long n_items = (long long)a.B * a.H * a.nJ;
+    // items of this CTA: blockIdx.x + m * gridDim.x, m < M; steps t = m * nI + i
+    const int M = blockIdx.x < n_items ? (int)((n_items - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+    const int Tn = M * nI;
+    struct Item { int b, h, jt; };
+    auto item = [&](int m) {
+        long long n = blockIdx.x + (long long)m * gridDim.x;
+        Item it;
+        it.jt = (int)(n % a.nJ);
+        n /= a.nJ;
+        it.h = (int)(n % a.H);
+        it.b = (int)(n / a.H);
+        return it;
+    };
 
     if (threadIdx.x == 0) {
-        mbar_init(b_kv, 1);
         mbar_init(b_sd_full, 1);
         mbar_init(b_sd_free, 256);
         mbar_init(b_ps_full, 256);
         mbar_init(b_ps_free, 1);
-        mbar_init(b_done, 1);
         mbar_init(b_drain, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_dq_full(x), 1);
@@ -260,6 +281,14 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_init(b_bias_full(x), 1);
             mbar_init(b_bias_empty(x), 256);
         }
+        for (int x = 0; x < KVB; ++x) {
+            mbar_init(b_kv_full(x), 1);
+            mbar_init(b_kv_empty(x), 1);
+        }
+        for (int x = 0; x < DKB; ++x) {
+            mbar_init(b_dkv_full(x), 1);
+            mbar_init(b_dkv_free(x), 256);
+        }
         s_abort = 0;
         fence_mbar_init();
     }
@@ -272,48 +301,64 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tc_fence_after();
     const uint32_t tbase = s_tmem_base;
     volatile int *abort_flag = &s_abort;
-    // query tiles whose Q/dOa/row-stat (bias) loads were issued: [0, q_done) ([0, bias_done))
-    int q_done = 0, bias_done = 0;
+    // loads issued: items [0, kv_done), steps [0, q_done) (Q/dOa/row stats), [0, bias_done)
+    int kv_done = 0, q_done = 0, bias_done = 0;
 
     if (warp == 8) {
         // ------------------------------------------------------------------ producer
-        uint32_t w[4];
-        mask_words(a, b, j0, w);
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
             if (a.has_bias) tma_prefetch_desc(&tmBias);
-            uint32_t *mw = reinterpret_cast<uint32_t *>(gbase + T::OFF_MASK);
-            mw[0] = w[0]; mw[1] = w[1]; mw[2] = w[2]; mw[3] = w[3];
-            mw[4] = (w[0] & w[1]) == 0xffffffffu;
-            mw[5] = (w[2] & w[3]) == 0xffffffffu;
-            mbar_arrive_tx(b_kv, 2 * T::TILE_BYTES);
-            tma_load_4d(sbase + T::OFF_K, &tmK, b_kv, 0, h, j0, b);
-            tma_load_4d(sbase + T::OFF_V, &tmV, b_kv, 0, h, j0, b);
-            bool ok = true;
-            int t = 0;
-            for (; t < nI && ok; ++t) {
-                const int st = t % QS, bs = t % BS, i0 = t * 128;
-                if (t >= QS) ok = mbar_wait(b_q_empty(st), ((t / QS) - 1) & 1, abort_flag, SITE_BWD_PROD);
+        }
+        bool ok = true;
+        for (int m = 0; m < M && ok; ++m) {
+            const Item it = item(m);
+            const int x = m % KVB, j0 = it.jt * 128;
+            if (m >= KVB)
+                ok = mbar_wait(b_kv_empty(x), ((m / KVB) - 1) & 1, abort_flag, SITE_BWD_PROD | 0x10 | (m << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            uint32_t w[4];
+            mask_words(a, it.b, j0, w);
+            if (lane == 0) {
+                uint32_t *mw = reinterpret_cast<uint32_t *>(gbase + T::OFF_MASK) + x * 8;
+                mw[0] = w[0]; mw[1] = w[1]; mw[2] = w[2]; mw[3] = w[3];
+                mw[4] = (w[0] & w[1]) == 0xffffffffu;
+                mw[5] = (w[2] & w[3]) == 0xffffffffu;
+                mbar_arrive_tx(b_kv_full(x), 2 * T::TILE_BYTES);
+                tma_load_4d(sbase + T::OFF_K + x * T::TILE_BYTES, &tmK, b_kv_full(x), 0, it.h, j0, it.b);
+                tma_load_4d(sbase + T::OFF_V + x * T::TILE_BYTES, &tmV, b_kv_full(x), 0, it.h, j0, it.b);
+            }
+            kv_done = m + 1;
+            for (int i = 0; i < nI && ok; ++i) {
+                const int t = m * nI + i, st = t % QS, bs = t % BS, i0 = i * 128;
+                if (t >= QS) ok = mbar_wait(b_q_empty(st), ((t / QS) - 1) & 1, abort_flag, SITE_BWD_PROD | (t << 12));
+                ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                const uint32_t qdst = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                mbar_arrive_tx(b_q_full(st), 2 * T::TILE_BYTES + 1024);
-                tma_load_4d(qdst, &tmQ, b_q_full(st), 0, h, i0, b);
-                tma_load_4d(qdst + T::TILE_BYTES, &tmDO, b_q_full(st), 0, h, i0, b);
-                bulk_load(sbase + T::OFF_RS + st * 1024,
-                          a.rowstats + ((long long)b * a.H + h) * a.NqPad + i0, 1024, b_q_full(st));
+                if (lane == 0) {
+                    const uint32_t qdst = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
+                    mbar_arrive_tx(b_q_full(st), 2 * T::TILE_BYTES + 1024);
+                    tma_load_4d(qdst, &tmQ, b_q_full(st), 0, it.h, i0, it.b);
+                    tma_load_4d(qdst + T::TILE_BYTES, &tmDO, b_q_full(st), 0, it.h, i0, it.b);
+                    bulk_load(sbase + T::OFF_RS + st * 1024,
+                              a.rowstats + ((long long)it.b * a.H + it.h) * a.NqPad + i0, 1024, b_q_full(st));
+                }
                 q_done = t + 1;
-                if (t >= BS) ok = mbar_wait(b_bias_empty(bs), ((t / BS) - 1) & 1, abort_flag, SITE_BWD_PROD);
+                if (t >= BS) ok = mbar_wait(b_bias_empty(bs), ((t / BS) - 1) & 1, abort_flag, SITE_BWD_PROD | 0x20 | (t << 12));
+                ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                if (a.has_bias) {
-                    const uint32_t dst = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
-                    mbar_arrive_tx(b_bias_full(bs), T::BIAS_BYTES);
-                    tma_load_3d(dst, &tmBias, b_bias_full(bs), j0, i0, h);
-                    tma_load_3d(dst + 16384, &tmBias, b_bias_full(bs), j0 + 64, i0, h);
-                } else {
-                    mbar_arrive(b_bias_full(bs));
+                if (lane == 0) {
+                    if (a.has_bias) {
+                        const uint32_t dst = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
+                        mbar_arrive_tx(b_bias_full(bs), T::BIAS_BYTES);
+                        tma_load_3d(dst, &tmBias, b_bias_full(bs), j0, i0, it.h);
+                        tma_load_3d(dst + 16384, &tmBias, b_bias_full(bs), j0 + 64, i0, it.h);
+                    } else {
+                        mbar_arrive(b_bias_full(bs));
+                    }
                 }
                 bias_done = t + 1;
             }
@@ -325,13 +370,13 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);   // S = Q K^T, dP = dOa V^T
             constexpr uint32_t id_kv = idesc_bf16(128, CP, true, true);     // dV = P^T dOa, dK = dS^T Q
             constexpr uint32_t id_q = idesc_bf16(128, CP, false, true);     // dQ = dS K
-            const uint32_t sK = sbase + T::OFF_K, sV = sbase + T::OFF_V;
             const uint32_t sP = sbase + T::OFF_P, sDS = sbase + T::OFF_DS;
-            bool ok = mbar_wait(b_kv, 0, abort_flag, SITE_BWD_MMA);
             auto issue_sdp = [&](int t) {
-                const int st = t % QS;
+                const int st = t % QS, x = (t / nI) % KVB;
                 const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
                 const uint32_t sDO = sQ + T::TILE_BYTES;
+                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < CP / 16; ++kk) {
                     umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
@@ -341,37 +386,62 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 umma_commit(b_sd_full);
             };
-            if (ok) ok = mbar_wait(b_q_full(0), 0, abort_flag, SITE_BWD_MMA);
-            if (ok) {
-                tc_fence_after();
-                issue_sdp(0);
+            bool ok = true;
+            if (Tn > 0) {
+                ok = mbar_wait(b_kv_full(0), 0, abort_flag, SITE_BWD_MMA | 0x10);
+                if (ok) ok = mbar_wait(b_q_full(0), 0, abort_flag, SITE_BWD_MMA);
+                if (ok) {
+                    tc_fence_after();
+                    issue_sdp(0);
+                }
             }
-            for (int t = 0; t < nI && ok; ++t) {
-                const int st = t % QS;
-                ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA);
+            for (int t = 0; t < Tn && ok; ++t) {
+                const int m = t / nI, i = t % nI, st = t % QS;
+                const int x = m % KVB, d = m % DKB;
+                ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
                 if (!ok) break;
-                if (t + 1 < nI) {
-                    ok = mbar_wait(b_q_full((t + 1) % QS), ((t + 1) / QS) & 1, abort_flag, SITE_BWD_MMA);
-                    if (ok) ok = mbar_wait(b_sd_free, t & 1, abort_flag, SITE_BWD_MMA);
-                    if (!ok) break;
+                // S/dP of the next step go ahead of this step's products, except when the
+                // next step starts an item whose K/V reuse this item's stage: those tiles
+                // only load once this item's MMAs are done, so they follow them.
+                const int m1 = (t + 1) / nI;
+                const bool late = t + 1 < Tn && m1 != m && m1 % KVB == x;
+                auto next_sdp = [&]() -> bool {
+                    bool okn = true;
+                    if (m1 != m)
+                        okn = mbar_wait(b_kv_full(m1 % KVB), (m1 / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x30 | (t << 12));
+                    if (okn) okn = mbar_wait(b_q_full((t + 1) % QS), ((t + 1) / QS) & 1, abort_flag, SITE_BWD_MMA | 0x40 | (t << 12));
+                    if (okn) okn = mbar_wait(b_sd_free, t & 1, abort_flag, SITE_BWD_MMA | 0x50 | (t << 12));
+                    if (!okn) return false;
                     tc_fence_after();
                     issue_sdp(t + 1);
+                    return true;
+                };
+                if (t + 1 < Tn && !late) {
+                    ok = next_sdp();
+                    if (!ok) break;
+                }
+                if (i == 0 && m >= DKB) {
+                    // this item's dK/dV buffer: the epilogue of item m - DKB has read it
+                    ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
+                    if (!ok) break;
                 }
                 if (t >= 2) {
-                    ok = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA);
+                    ok = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
                     if (!ok) break;
                 }
                 tc_fence_after();
                 const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
                 const uint32_t sDO = sQ + T::TILE_BYTES;
+                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                const uint32_t tDK = tbase + T::T_DK + d * 2 * CP, tDV = tDK + CP;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
                     // B (dOa / Q, MN-major) rows advance 16 rows
-                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                    umma_ss(tbase + T::T_DV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
+                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                    umma_ss(tDV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
                             sdesc(sDO + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                    umma_ss(tbase + T::T_DK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
+                    umma_ss(tDK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
                             sdesc(sQ + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
                 }
 #pragma unroll
@@ -384,8 +454,12 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 umma_commit(b_ps_free);
                 umma_commit(b_q_empty(st));
                 umma_commit(b_dq_full(t & 1));
+                if (i == nI - 1) {
+                    umma_commit(b_dkv_full(d));
+                    umma_commit(b_kv_empty(x));
+                }
+                if (late) ok = next_sdp();
             }
-            if (ok) umma_commit(b_done);
         }
     } else {
         // ------------------------------------------------------------------ elementwise
@@ -393,15 +467,11 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int e = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
-        const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK);
-        bool ok = mbar_wait(b_kv, 0, abort_flag, SITE_BWD_EW);
-        ok = __all_sync(0xffffffffu, ok);
-        const uint32_t mw0 = mw[2 * e], mw1 = mw[2 * e + 1];
-        const bool full = mw[4 + e] != 0;
         const float scale = a.scale;
+        bool ok = true;
         auto flush_dq = [&](int t) -> bool {
             // dQ(t): this thread's query row, channels [e CP/2, (e+1) CP/2), added to dqacc
-            bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EW);
+            bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EW | 0x10 | (t << 12));
             okf = __all_sync(0xffffffffu, okf);
             if (!okf) return false;
             tc_fence_after();
@@ -419,9 +489,10 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             tc_fence_before();
             mbar_arrive(b_dq_free(t & 1));
-            const int i = t * 128 + row;
+            const Item it = item(t / nI);
+            const int i = (t % nI) * 128 + row;
             if (i < a.Nq) {
-                float *dst = a.dqacc + (((long long)b * a.Nq + i) * a.H + h) * a.C;
+                float *dst = a.dqacc + (((long long)it.b * a.Nq + i) * a.H + it.h) * a.C;
 #pragma unroll
                 for (int c4 = 0; c4 < CP / 8; ++c4) {
                     const int c = e * (CP / 2) + c4 * 4;
@@ -433,11 +504,53 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             return true;
         };
-        for (int t = 0; t < nI && ok; ++t) {
-            const int st = t % QS, bs = t % BS;
-            ok = mbar_wait(b_sd_full, t & 1, abort_flag, SITE_BWD_EW);
-            if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_EW);
-            if (ok) ok = mbar_wait(b_bias_full(bs), (t / BS) & 1, abort_flag, SITE_BWD_EW);
+        auto epilogue = [&](int m) -> bool {
+            // dK/dV of item m: warpgroup 0 writes dK (times scale), warpgroup 1 dV; lane = key
+            bool oke = mbar_wait(b_dkv_full(m % DKB), (m / DKB) & 1, abort_flag, SITE_BWD_EW | 0x20 | (m << 12));
+            oke = __all_sync(0xffffffffu, oke);
+            if (!oke) return false;
+            tc_fence_after();
+            uint32_t r[CP];
+            tmem_ld_cols<CP>(tbase + T::T_DK + (m % DKB) * 2 * CP + e * CP + lane_off, r);
+            tc_fence_before();
+            mbar_arrive(b_dkv_free(m % DKB));
+            const Item it = item(m);
+            const int j = it.jt * 128 + row;
+            if (j < a.Nk) {
+                __nv_bfloat16 *dst = e == 0 ? a.dk + it.b * a.sk0 + (long long)j * a.sk1 + it.h * a.sk2
+                                            : a.dv + it.b * a.sv0 + (long long)j * a.sv1 + it.h * a.sv2;
+                const float mul = e == 0 ? a.scale : 1.f;
+#pragma unroll
+                for (int c8 = 0; c8 < CP / 8; ++c8) {
+                    if (c8 * 8 < a.C) {
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            ow[q] = pack_bf16x2(__uint_as_float(r[c8 * 8 + 2 * q]) * mul,
+                                                __uint_as_float(r[c8 * 8 + 2 * q + 1]) * mul);
+                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+            }
+            return true;
+        };
+        uint32_t mw0 = 0, mw1 = 0;
+        bool full = true;
+        for (int t = 0; t < Tn && ok; ++t) {
+            const int m = t / nI, i = t % nI, st = t % QS, bs = t % BS;
+            if (i == 0) {
+                // this item's mask words come with its K/V tiles
+                ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + (m % KVB) * 8;
+                mw0 = mw[2 * e];
+                mw1 = mw[2 * e + 1];
+                full = mw[4 + e] != 0;
+            }
+            ok = mbar_wait(b_sd_full, t & 1, abort_flag, SITE_BWD_EW | (t << 12));
+            if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_EW | 0x40 | (t << 12));
+            if (ok) ok = mbar_wait(b_bias_full(bs), (t / BS) & 1, abort_flag, SITE_BWD_EW | 0x50 | (t << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -451,7 +564,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_arrive(b_bias_empty(bs));
             mbar_arrive(b_q_empty(st));
             if (t > 0) {
-                ok = mbar_wait(b_ps_free, (t - 1) & 1, abort_flag, SITE_BWD_EW);
+                ok = mbar_wait(b_ps_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x60 | (t << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
@@ -474,36 +587,10 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             fence_proxy_async();
             mbar_arrive(b_ps_full);
             if (t > 0) ok = flush_dq(t - 1);
+            if (ok && i == 0 && m > 0) ok = epilogue(m - 1);
         }
-        if (ok && nI > 0) ok = flush_dq(nI - 1);
-        // ------------------------------------------------------------------ epilogue
-        if (ok) {
-            ok = mbar_wait(b_done, 0, abort_flag, SITE_BWD_EW);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        if (ok) {
-            tc_fence_after();
-            // warpgroup 0 writes dK (times scale), warpgroup 1 writes dV; lane = key row
-            uint32_t r[CP];
-            tmem_ld_cols<CP>(tbase + (e == 0 ? T::T_DK : T::T_DV) + lane_off, r);
-            const int j = j0 + row;
-            if (j < a.Nk) {
-                __nv_bfloat16 *dst = e == 0 ? a.dk + b * a.sk0 + (long long)j * a.sk1 + h * a.sk2
-                                            : a.dv + b * a.sv0 + (long long)j * a.sv1 + h * a.sv2;
-                const float mul = e == 0 ? a.scale : 1.f;
-#pragma unroll
-                for (int c8 = 0; c8 < CP / 8; ++c8) {
-                    if (c8 * 8 < a.C) {
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            ow[q] = pack_bf16x2(__uint_as_float(r[c8 * 8 + 2 * q]) * mul,
-                                                __uint_as_float(r[c8 * 8 + 2 * q + 1]) * mul);
-                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
-                }
-            }
-        }
+        if (ok && Tn > 0) ok = flush_dq(Tn - 1);
+        if (ok && M > 0) ok = epilogue(M - 1);
     }
 
     tc_fence_before();
@@ -512,7 +599,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // a wait ran out: let the copies and MMAs already issued finish before shared memory
         // and TMEM are released (bounded waits)
         if (warp == 8 && lane == 0) {
-            mbar_wait_drain(b_kv, 0);
+            for (int mm = max(0, kv_done - KVB); mm < kv_done; ++mm)
+                mbar_wait_drain(b_kv_full(mm % KVB), (mm / KVB) & 1);
             for (int tt = max(0, q_done - QS); tt < q_done; ++tt) mbar_wait_drain(b_q_full(tt % QS), (tt / QS) & 1);
             for (int tt = max(0, bias_done - BS); tt < bias_done; ++tt)
                 mbar_wait_drain(b_bias_full(tt % BS), (tt / BS) & 1);

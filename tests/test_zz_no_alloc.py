@@ -57,9 +57,9 @@ def test_noalloc_matches_workspace_entry_point_twice(pba):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(pba):
-    # the MSA row attention workload needs more than 64 MiB of scratch: refused on the
-    # host, before any launch
-    d = pba.dims_dense(128, 8, 256, 256, 32)
+    # the triangle attention workload (384 rows of 384 tokens, 4 heads) needs more than
+    # 64 MiB of scratch: refused on the host, before any launch
+    d = pba.dims_dense(384, 4, 384, 384, 32)
     assert pba.pba_bwd_workspace_size(d) > (64 << 20)
     st = pba.lib.pba_bwd_noalloc(*([16] * 14), ctypes.byref(d), None)
     assert st == 2
