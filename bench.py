@@ -61,11 +61,10 @@ def work(cfg: pi.Config, B=None):
         "pba_fwd_kernel": (4 * unit, 5 * e * 2 + lse_b + bias_b + mask_b),
         # q, k, v, dOa, (lse, D) in; dq, dk, dv out; bias; mask
         "pba_bwd_main_kernel": (10 * unit, 7 * e * 2 + B * H * N * 8 + bias_b + mask_b),
-        # q, k, v, dOa, (lse, D) in; bias; dbias out
+        # q, k, v, dOa, (lse, D) in; bias; dbias out (the split partials are workspace)
         "pba_dbias_kernel": (0, 4 * e * 2 + B * H * N * 8 + bias_b + H * N * N * 4),
         # out, dout, g, lse in; dOa, dg, (lse, D) out
         "pba_bwd_pre_kernel": (0, 5 * e * 2 + lse_b + B * H * N * 8),
-        "pba_dbias_reduce_kernel": (0, 2 * H * N * N * 4),
         "pba_dq_convert_kernel": (0, e * 4 + e * 2),
     }
     return f

@@ -39,9 +39,9 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 // ---------------------------------------------------------------------------- profiling
-enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DBIAS_REDUCE, K_DQ_CONVERT, K_ZERO_ROWS, K_COUNT };
+enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS, K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
-                                           "pba_dbias_kernel", "pba_dbias_reduce_kernel",
+                                           "pba_dbias_kernel",
                                            "pba_dq_convert_kernel", "zero_rows_kernel"};
 struct ProfRec {
     int kid;
@@ -255,7 +255,7 @@ constexpr long long kSmCount = 148;   // SMs of a B200
 
 struct BwdPlan {
     int nI, nJ, NqPad, NkPad, splits, rows_per_split;
-    size_t off_rs, off_doa, off_dq, off_part, total;
+    size_t off_rs, off_doa, off_dq, off_cnt, off_part, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -292,7 +292,10 @@ BwdPlan plan_bwd(const pba_dims *d) {
     p.off_rs = 0;
     p.off_doa = align256(p.off_rs + rows * sizeof(float2));
     p.off_dq = align256(p.off_doa + elems * 2);
-    p.off_part = align256(p.off_dq + elems * 4);
+    // per-tile counters of the dbias kernel right after the dQ accumulator: one memset
+    // clears both
+    p.off_cnt = align256(p.off_dq + elems * 4);
+    p.off_part = align256(p.off_cnt + (size_t)d->H * p.nI * p.nJ * sizeof(int));
     p.total = align256(p.off_part + (size_t)p.splits * d->H * p.NqPad * p.NkPad * 4);
     return p;
 }
@@ -382,6 +385,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.doa = reinterpret_cast<__nv_bfloat16 *>(w + pl.off_doa);
     a.dqacc = reinterpret_cast<float *>(w + pl.off_dq);
     a.dbias_part = reinterpret_cast<float *>(w + pl.off_part);
+    a.tile_count = reinterpret_cast<int *>(w + pl.off_cnt);
 
     pba_status st;
     CUtensorMap tq, tk, tv, tdo, tb;
@@ -401,21 +405,23 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     }
     cudaError_t e;
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
-    if ((e = cudaMemsetAsync(a.dqacc, 0, elems * 4, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if ((e = cudaMemsetAsync(a.dqacc, 0, pl.off_part - pl.off_dq, s)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync");
     const long long pre_rows = (long long)d->B * pl.NqPad * d->H;
     {
         ProfScope ps(K_BWD_PRE, s);
-        pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows, 256), 256, 0, s>>>(a);
+        pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows * (CP / 8), 256), 256, 0, s>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_pre_kernel launch");
     if (pl.nJ > 0) {
         if ((st = set_smem(pba::pba_bwd_main_kernel<CP>, MT::SMEM_BYTES)) != PBA_OK) return st;
         // persistent: one CTA per SM (at most one per item)
         const long long items = (long long)d->B * d->H * pl.nJ;
+        if (items >= (1LL << 31)) return fail(PBA_ERR_UNSUPPORTED, "B * H * key tiles must be below 2^31");
         const long long grid = items < num_sms() ? items : num_sms();
         {
             ProfScope ps(K_BWD_MAIN, s);
-            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 320, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 352, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {
@@ -426,12 +432,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                 pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
-            const long long n = (long long)d->H * d->Nq * d->Nk;
-            {
-                ProfScope ps(K_DBIAS_REDUCE, s);
-                pba::pba_dbias_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(a);
-            }
-            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_reduce_kernel launch");
+            // (the last CTA of every tile sums the split partials in split order)
         }
     }
     {

@@ -17,8 +17,8 @@
 //                           accumulator in global memory
 //   pba_dbias_kernel        CTA = (h, query tile, key tile, split of b): loops over its rows
 //                           b with the bias tile resident; dS summed in registers; one fp32
-//                           partial tile per split
-//   pba_dbias_reduce_kernel sums the split partials in split order (bit-stable dbias)
+//                           partial tile per split; the tile's last CTA to finish sums the
+//                           partials in split order (bit-stable dbias)
 //   pba_dq_convert_kernel   fp32 dQ accumulator -> bf16 dq (times scale)
 #pragma once
 
@@ -47,6 +47,7 @@ struct BwdArgs {
     __nv_bfloat16 *doa;        // [B][Nq][H][C] (only with a gate)
     float *dqacc;              // [B][Nq][H][C]
     float *dbias_part;         // [splits][H][NqPad][NkPad]
+    int *tile_count;           // [H][nI][nJ]: splits done (zeroed before the launch)
 };
 
 enum : unsigned {
@@ -57,37 +58,40 @@ enum : unsigned {
 constexpr float kLog2eB = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------------------
-// pre: one thread per (b, i, h) query row, i < NqPad (padded rows only get row stats)
+// pre: CP/8 lanes per query row (16 bytes of each tensor per lane), rows r = (b, h, i) with
+// i < NqPad fastest, so row stats and lse are read and written contiguously; padded rows
+// only get row stats
 // ---------------------------------------------------------------------------------------
 template <int CP>
 __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
-    const long long n = (long long)a.B * a.NqPad * a.H;
-    for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
-         r += (long long)gridDim.x * blockDim.x) {
-        const int h = (int)(r % a.H);
-        const long long bi = r / a.H;
-        const int i = (int)(bi % a.NqPad);
-        const int b = (int)(bi / a.NqPad);
-        float2 rs = make_float2(INFINITY, 0.f);
-        if (i < a.Nq) {
-            const __nv_bfloat16 *op = a.out + b * a.so0 + (long long)i * a.so1 + h * a.so2;
-            const __nv_bfloat16 *dp = a.dout + b * a.so0 + (long long)i * a.so1 + h * a.so2;
-            const __nv_bfloat16 *gp = a.has_gate ? a.gate + b * a.sg0 + (long long)i * a.sg1 + h * a.sg2 : nullptr;
-            __nv_bfloat16 *dgp = a.has_gate ? a.dgate + b * a.sg0 + (long long)i * a.sg1 + h * a.sg2 : nullptr;
-            __nv_bfloat16 *dap = a.has_gate ? a.doa + (((long long)b * a.Nq + i) * a.H + h) * a.C : nullptr;
-            float D = 0.f;
-#pragma unroll
-            for (int c8 = 0; c8 < CP / 8; ++c8) {
-                if (c8 * 8 >= a.C) break;
-                const uint4 o4 = *reinterpret_cast<const uint4 *>(op + c8 * 8);
-                const uint4 d4 = *reinterpret_cast<const uint4 *>(dp + c8 * 8);
-                const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
-                const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
-                uint32_t gw[4] = {0, 0, 0, 0};
-                if (gp) {
-                    const uint4 g4 = *reinterpret_cast<const uint4 *>(gp + c8 * 8);
-                    gw[0] = g4.x; gw[1] = g4.y; gw[2] = g4.z; gw[3] = g4.w;
-                }
+    constexpr int LPR = CP / 8;        // lanes per row
+    constexpr int RPW = 32 / LPR;      // rows per warp
+    const int lane = threadIdx.x & 31, sub = lane % LPR, rw = lane / LPR;
+    const long long nrows = (long long)a.B * a.H * a.NqPad;
+    const long long wstride = (long long)gridDim.x * (blockDim.x >> 5) * RPW;
+    for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW; r0 < nrows;
+         r0 += wstride) {
+        const long long r = r0 + rw;
+        const bool in = r < nrows;
+        int i = 0, h = 0, b = 0;
+        if (in) {
+            i = (int)(r % a.NqPad);
+            const long long bh = r / a.NqPad;
+            h = (int)(bh % a.H);
+            b = (int)(bh / a.H);
+        }
+        float D = 0.f;
+        const int c0 = sub * 8;
+        if (in && i < a.Nq && c0 < a.C) {
+            const long long orow = b * a.so0 + (long long)i * a.so1 + h * a.so2 + c0;
+            const uint4 o4 = *reinterpret_cast<const uint4 *>(a.out + orow);
+            const uint4 d4 = *reinterpret_cast<const uint4 *>(a.dout + orow);
+            const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+            const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+            if (a.has_gate) {
+                const long long grow = b * a.sg0 + (long long)i * a.sg1 + h * a.sg2 + c0;
+                const uint4 g4 = *reinterpret_cast<const uint4 *>(a.gate + grow);
+                const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
                 uint32_t dgw[4], daw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -95,23 +99,33 @@ __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
                     const float d0 = bf16lo(dw[e]), d1 = bf16hi(dw[e]);
                     D = fmaf(d0, o0, D);
                     D = fmaf(d1, o1, D);
-                    if (gp) {
-                        const float s0 = 1.f / (1.f + __expf(-bf16lo(gw[e])));
-                        const float s1 = 1.f / (1.f + __expf(-bf16hi(gw[e])));
-                        daw[e] = pack_bf16x2(d0 * s0, d1 * s1);
-                        dgw[e] = pack_bf16x2(d0 * o0 * (1.f - s0), d1 * o1 * (1.f - s1));
-                    }
+                    const float s0 = 1.f / (1.f + __expf(-bf16lo(gw[e])));
+                    const float s1 = 1.f / (1.f + __expf(-bf16hi(gw[e])));
+                    daw[e] = pack_bf16x2(d0 * s0, d1 * s1);
+                    dgw[e] = pack_bf16x2(d0 * o0 * (1.f - s0), d1 * o1 * (1.f - s1));
                 }
-                if (gp) {
-                    *reinterpret_cast<uint4 *>(dap + c8 * 8) = make_uint4(daw[0], daw[1], daw[2], daw[3]);
-                    *reinterpret_cast<uint4 *>(dgp + c8 * 8) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                *reinterpret_cast<uint4 *>(a.doa + (((long long)b * a.Nq + i) * a.H + h) * a.C + c0) =
+                    make_uint4(daw[0], daw[1], daw[2], daw[3]);
+                *reinterpret_cast<uint4 *>(a.dgate + grow) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    D = fmaf(bf16lo(dw[e]), bf16lo(ow[e]), D);
+                    D = fmaf(bf16hi(dw[e]), bf16hi(ow[e]), D);
                 }
             }
-            const float l = a.lse[((long long)b * a.H + h) * a.Nq + i];
-            rs.x = (l == -INFINITY) ? INFINITY : l * kLog2eB;
-            rs.y = D;
         }
-        a.rowstats[((long long)b * a.H + h) * a.NqPad + i] = rs;
+#pragma unroll
+        for (int x = 1; x < LPR; x <<= 1) D += __shfl_xor_sync(0xffffffffu, D, x);
+        if (in && sub == 0) {
+            float2 rs = make_float2(INFINITY, 0.f);
+            if (i < a.Nq) {
+                const float l = a.lse[((long long)b * a.H + h) * a.Nq + i];
+                rs.x = (l == -INFINITY) ? INFINITY : l * kLog2eB;
+                rs.y = D;
+            }
+            a.rowstats[r] = rs;   // [B][H][NqPad]
+        }
     }
 }
 
@@ -132,18 +146,23 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
     }
 }
 
-// P and dS of 64 keys (one half of a 128-key tile) for one query row.
-//   S, dP: this lane's 64 fp32 values from TMEM; bias: the row's 64 bf16 in a 128-byte
-//   swizzled shared-memory row; mask: two 32-bit words for those 64 keys.
-// Returns P (fp32) in p[], dS (fp32) in ds[].
+// P and dS of 64 keys (one half of a 128-key tile) for one query row, in 32-key chunks.
+//   tS, tdP: this lane's S and dP columns in TMEM; bias_row: the row's 64 bf16 bias values
+//   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
+//   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
+//   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
+// For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS.
+template <typename Use>
 __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
                                           bool has_bias, uint32_t mw0, uint32_t mw1, bool full,
-                                          float scale, float lse2, float D, float (&p)[64],
-                                          float (&ds)[64]) {
+                                          float sl2e, float lse2, float D, Use &&use) {
+    const float2 sl2 = make_float2(sl2e, sl2e), l2e2 = make_float2(kLog2eB, kLog2eB);
+    const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tS + q * 32, r);
+        uint32_t r[64];   // S of keys 32 q .. 32 q + 31 in r[0..31], dP in r[32..63]
+        tmem_ld32x2(tS + q * 32, tdP + q * 32, r);
+        const uint32_t mw = q == 0 ? mw0 : mw1;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
             const int c8 = q * 4 + c4;
@@ -152,27 +171,18 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int c = q * 32 + c4 * 8 + 2 * e;
-                const float t0 = fmaf(__uint_as_float(r[c4 * 8 + 2 * e]), scale, bf16lo(bb[e]));
-                const float t1 = fmaf(__uint_as_float(r[c4 * 8 + 2 * e + 1]), scale, bf16hi(bb[e]));
-                p[c] = ex2(fmaf(t0, kLog2eB, -lse2));
-                p[c + 1] = ex2(fmaf(t1, kLog2eB, -lse2));
+                const int k = c4 * 8 + 2 * e;   // key within the chunk
+                float2 u = ffma2(make_float2(bf16lo(bb[e]), bf16hi(bb[e])), l2e2, nl2);
+                u = ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, u);
+                float2 p = make_float2(ex2(u.x), ex2(u.y));
+                if (!full) {
+                    p.x = ((mw >> k) & 1u) ? p.x : 0.f;
+                    p.y = ((mw >> (k + 1)) & 1u) ? p.y : 0.f;
+                }
+                const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(r[32 + k]), __uint_as_float(r[33 + k])), nD2));
+                use(q * 32 + k, p, ds);
             }
         }
-    }
-    if (!full) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-            const uint32_t wd = c < 32 ? mw0 : mw1;
-            if (!((wd >> (c & 31)) & 1u)) p[c] = 0.f;
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tdP + q * 32, r);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) ds[q * 32 + c] = p[q * 32 + c] * (__uint_as_float(r[c]) - D);
     }
 }
 
@@ -188,7 +198,7 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct BwdTraits {
-    static constexpr int QS = 2;                                // Q/dOa/row-stat stages
+    static constexpr int QS = (CP == 64) ? 2 : 3;               // Q/dOa/row-stat stages
     static constexpr int BS = (CP == 64) ? 1 : 2;               // bias stages
     static constexpr int KVB = (CP == 64) ? 1 : 2;              // K/V stages (items)
     static constexpr int DKB = (CP == 64) ? 1 : 2;              // dK/dV TMEM buffers (items)
@@ -213,8 +223,13 @@ struct BwdTraits {
 };
 static_assert(BwdTraits<64>::SMEM_BYTES <= 232448 && BwdTraits<32>::SMEM_BYTES <= 232448, "smem");
 
+// Warp roles (352 threads): warps 0-7 element-wise (two warpgroups, one 64-key half each),
+// warp 8 TMA producer, warp 9 TMEM allocator and (lane 0) issuer of the dV, dK, dQ
+// products, warp 10 (lane 0) issuer of S = Q K^T and dP = dOa V^T.  A tcgen05.mma issue
+// holds its thread about as long as the MMA runs, so S/dP of the next step do not wait
+// behind this step's 24 products.
 template <int CP>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
@@ -253,13 +268,13 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int M = blockIdx.x < n_items ? (int)((n_items - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
     const int Tn = M * nI;
     struct Item { int b, h, jt; };
-    auto item = [&](int m) {
-        long long n = blockIdx.x + (long long)m * gridDim.x;
+    auto item = [&](int m) {   // n_items < 2^31 (checked on the host)
+        int n = (int)blockIdx.x + m * (int)gridDim.x;
         Item it;
-        it.jt = (int)(n % a.nJ);
+        it.jt = n % a.nJ;
         n /= a.nJ;
-        it.h = (int)(n % a.H);
-        it.b = (int)(n / a.H);
+        it.h = n % a.H;
+        it.b = n / a.H;
         return it;
     };
 
@@ -268,7 +283,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(b_sd_free, 256);
         mbar_init(b_ps_full, 256);
         mbar_init(b_ps_free, 1);
-        mbar_init(b_drain, 1);
+        mbar_init(b_drain, 2);   // one commit from each issuer
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_dq_full(x), 1);
             mbar_init(b_dq_free(x), 256);
@@ -363,16 +378,21 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 bias_done = t + 1;
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 10) {
+        // ------------------------------------------------------------------ S/dP issuer
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);   // S = Q K^T, dP = dOa V^T
-            constexpr uint32_t id_kv = idesc_bf16(128, CP, true, true);     // dV = P^T dOa, dK = dS^T Q
-            constexpr uint32_t id_q = idesc_bf16(128, CP, false, true);     // dQ = dS K
-            const uint32_t sP = sbase + T::OFF_P, sDS = sbase + T::OFF_DS;
-            auto issue_sdp = [&](int t) {
-                const int st = t % QS, x = (t / nI) % KVB;
+            bool ok = true;
+            // step t: its item's K/V, its Q/dOa, and S/dP of step t - 1 read out
+            for (int t = 0; t < Tn && ok; ++t) {
+                const int m = t / nI, st = t % QS, x = m % KVB;
+                if (t % nI == 0)
+                    ok = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
+                if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
+                if (ok && t > 0) ok = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
+                if (!ok) break;
+                tc_fence_after();
                 const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
                 const uint32_t sDO = sQ + T::TILE_BYTES;
                 const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
@@ -385,41 +405,23 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                             sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
                 }
                 umma_commit(b_sd_full);
-            };
-            bool ok = true;
-            if (Tn > 0) {
-                ok = mbar_wait(b_kv_full(0), 0, abort_flag, SITE_BWD_MMA | 0x10);
-                if (ok) ok = mbar_wait(b_q_full(0), 0, abort_flag, SITE_BWD_MMA);
-                if (ok) {
-                    tc_fence_after();
-                    issue_sdp(0);
-                }
             }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------------ products issuer
+        if (lane == 0) {
+            constexpr uint32_t SBO = 8 * T::ROWB;
+            constexpr uint32_t id_kv = idesc_bf16(128, CP, true, true);     // dV = P^T dOa, dK = dS^T Q
+            constexpr uint32_t id_q = idesc_bf16(128, CP, false, true);     // dQ = dS K
+            const uint32_t sP = sbase + T::OFF_P, sDS = sbase + T::OFF_DS;
+            bool ok = true;
+            // step t: P/dS written (S/dP of the step were read out before that, so its
+            // S/dP MMAs are complete); this item's dK/dV buffer and the dQ buffer free
             for (int t = 0; t < Tn && ok; ++t) {
                 const int m = t / nI, i = t % nI, st = t % QS;
                 const int x = m % KVB, d = m % DKB;
                 ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
                 if (!ok) break;
-                // S/dP of the next step go ahead of this step's products, except when the
-                // next step starts an item whose K/V reuse this item's stage: those tiles
-                // only load once this item's MMAs are done, so they follow them.
-                const int m1 = (t + 1) / nI;
-                const bool late = t + 1 < Tn && m1 != m && m1 % KVB == x;
-                auto next_sdp = [&]() -> bool {
-                    bool okn = true;
-                    if (m1 != m)
-                        okn = mbar_wait(b_kv_full(m1 % KVB), (m1 / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x30 | (t << 12));
-                    if (okn) okn = mbar_wait(b_q_full((t + 1) % QS), ((t + 1) / QS) & 1, abort_flag, SITE_BWD_MMA | 0x40 | (t << 12));
-                    if (okn) okn = mbar_wait(b_sd_free, t & 1, abort_flag, SITE_BWD_MMA | 0x50 | (t << 12));
-                    if (!okn) return false;
-                    tc_fence_after();
-                    issue_sdp(t + 1);
-                    return true;
-                };
-                if (t + 1 < Tn && !late) {
-                    ok = next_sdp();
-                    if (!ok) break;
-                }
                 if (i == 0 && m >= DKB) {
                     // this item's dK/dV buffer: the epilogue of item m - DKB has read it
                     ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
@@ -458,7 +460,6 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     umma_commit(b_dkv_full(d));
                     umma_commit(b_kv_empty(x));
                 }
-                if (late) ok = next_sdp();
             }
         }
     } else {
@@ -467,9 +468,11 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int e = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
-        const float scale = a.scale;
+        const float sl2e = a.scale * kLog2eB;
         bool ok = true;
-        auto flush_dq = [&](int t) -> bool {
+        // items of the current and the previous step (decoded once per item)
+        Item cur = {0, 0, 0}, last = {0, 0, 0};
+        auto flush_dq = [&](int t, const Item &it) -> bool {
             // dQ(t): this thread's query row, channels [e CP/2, (e+1) CP/2), added to dqacc
             bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EW | 0x10 | (t << 12));
             okf = __all_sync(0xffffffffu, okf);
@@ -489,7 +492,6 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             tc_fence_before();
             mbar_arrive(b_dq_free(t & 1));
-            const Item it = item(t / nI);
             const int i = (t % nI) * 128 + row;
             if (i < a.Nq) {
                 float *dst = a.dqacc + (((long long)it.b * a.Nq + i) * a.H + it.h) * a.C;
@@ -497,14 +499,13 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 for (int c4 = 0; c4 < CP / 8; ++c4) {
                     const int c = e * (CP / 2) + c4 * 4;
                     if (c < a.C)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + c),
-                                  make_float4(__uint_as_float(r[c4 * 4]), __uint_as_float(r[c4 * 4 + 1]),
-                                              __uint_as_float(r[c4 * 4 + 2]), __uint_as_float(r[c4 * 4 + 3])));
+                        red_add_v4(dst + c, __uint_as_float(r[c4 * 4]), __uint_as_float(r[c4 * 4 + 1]),
+                                   __uint_as_float(r[c4 * 4 + 2]), __uint_as_float(r[c4 * 4 + 3]));
                 }
             }
             return true;
         };
-        auto epilogue = [&](int m) -> bool {
+        auto epilogue = [&](int m, const Item &it) -> bool {
             // dK/dV of item m: warpgroup 0 writes dK (times scale), warpgroup 1 dV; lane = key
             bool oke = mbar_wait(b_dkv_full(m % DKB), (m / DKB) & 1, abort_flag, SITE_BWD_EW | 0x20 | (m << 12));
             oke = __all_sync(0xffffffffu, oke);
@@ -514,7 +515,6 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_ld_cols<CP>(tbase + T::T_DK + (m % DKB) * 2 * CP + e * CP + lane_off, r);
             tc_fence_before();
             mbar_arrive(b_dkv_free(m % DKB));
-            const Item it = item(m);
             const int j = it.jt * 128 + row;
             if (j < a.Nk) {
                 __nv_bfloat16 *dst = e == 0 ? a.dk + it.b * a.sk0 + (long long)j * a.sk1 + it.h * a.sk2
@@ -539,6 +539,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int t = 0; t < Tn && ok; ++t) {
             const int m = t / nI, i = t % nI, st = t % QS, bs = t % BS;
             if (i == 0) {
+                last = cur;
+                cur = item(m);
                 // this item's mask words come with its K/V tiles
                 ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
                 ok = __all_sync(0xffffffffu, ok);
@@ -555,10 +557,14 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (!ok) break;
             tc_fence_after();
             const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
-            float p[64], ds[64];
+            uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
             const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
             p_ds_half(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
-                      row, a.has_bias != 0, mw0, mw1, full, scale, rs.x, rs.y, p, ds);
+                      row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
+                      [&](int c, float2 p, float2 ds) {
+                          pp[c >> 1] = pack_bf16x2(p.x, p.y);
+                          dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
+                      });
             tc_fence_before();
             mbar_arrive(b_sd_free);
             mbar_arrive(b_bias_empty(bs));
@@ -574,23 +580,17 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
                 const uint32_t sw = (uint32_t)((c8 ^ (row & 7)) << 4);
-                sts128(prow + sw, make_uint4(pack_bf16x2(p[c8 * 8 + 0], p[c8 * 8 + 1]),
-                                             pack_bf16x2(p[c8 * 8 + 2], p[c8 * 8 + 3]),
-                                             pack_bf16x2(p[c8 * 8 + 4], p[c8 * 8 + 5]),
-                                             pack_bf16x2(p[c8 * 8 + 6], p[c8 * 8 + 7])));
-                sts128(drow + sw, make_uint4(pack_bf16x2(ds[c8 * 8 + 0], ds[c8 * 8 + 1]),
-                                             pack_bf16x2(ds[c8 * 8 + 2], ds[c8 * 8 + 3]),
-                                             pack_bf16x2(ds[c8 * 8 + 4], ds[c8 * 8 + 5]),
-                                             pack_bf16x2(ds[c8 * 8 + 6], ds[c8 * 8 + 7])));
+                sts128(prow + sw, make_uint4(pp[c8 * 4], pp[c8 * 4 + 1], pp[c8 * 4 + 2], pp[c8 * 4 + 3]));
+                sts128(drow + sw, make_uint4(dsp[c8 * 4], dsp[c8 * 4 + 1], dsp[c8 * 4 + 2], dsp[c8 * 4 + 3]));
             }
             // generic-proxy writes -> visible to the tensor core's async proxy
             fence_proxy_async();
             mbar_arrive(b_ps_full);
-            if (t > 0) ok = flush_dq(t - 1);
-            if (ok && i == 0 && m > 0) ok = epilogue(m - 1);
+            if (t > 0) ok = flush_dq(t - 1, i == 0 ? last : cur);
+            if (ok && i == 0 && m > 0) ok = epilogue(m - 1, last);
         }
-        if (ok && Tn > 0) ok = flush_dq(Tn - 1);
-        if (ok && M > 0) ok = epilogue(M - 1);
+        if (ok && Tn > 0) ok = flush_dq(Tn - 1, cur);
+        if (ok && M > 0) ok = epilogue(M - 1, cur);
     }
 
     tc_fence_before();
@@ -605,8 +605,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int tt = max(0, bias_done - BS); tt < bias_done; ++tt)
                 mbar_wait_drain(b_bias_full(tt % BS), (tt / BS) & 1);
         }
-        if (warp == 9 && lane == 0) {
-            umma_commit(b_drain);
+        if ((warp == 9 || warp == 10) && lane == 0) {
+            umma_commit(b_drain);   // each issuer's own MMAs
             mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
@@ -767,10 +767,10 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int e = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
-        const float scale = a.scale;
-        float acc[64];
+        const float sl2e = a.scale * kLog2eB;
+        float2 acc[32];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
         bool ok = mbar_wait(b_bias, 0, abort_flag, SITE_DB_EW);
         ok = __all_sync(0xffffffffu, ok);
         const uint32_t bias_row = sbase + T::OFF_BIAS + e * 16384 + row * 128;
@@ -784,23 +784,21 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
             const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
             const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
-            float p[64], ds[64];
             p_ds_half(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
-                      bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, scale,
-                      rs.x, rs.y, p, ds);
+                      bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
+                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
             tc_fence_before();
             mbar_arrive(b_sd_free(x));
             mbar_arrive(b_empty(st));
-#pragma unroll
-            for (int c = 0; c < 64; ++c) acc[c] += ds[c];
         }
         if (ok) {
             // this split's partial tile, padded layout: [split][h][NqPad][NkPad]
             float *dst = a.dbias_part +
                          ((((long long)sp * a.H + h) * a.NqPad + i0 + row) * a.NkPad + j0 + e * 64);
 #pragma unroll
-            for (int c = 0; c < 64; c += 4)
-                *reinterpret_cast<float4 *>(dst + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+            for (int c = 0; c < 32; c += 2)
+                *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
+            __threadfence();   // this thread's partial row, before the tile counter moves
         }
     }
 
@@ -823,22 +821,36 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tbase, 512);
     }
-}
-
-// dbias[h][i][j] = sum over splits s = 0, 1, ... of the partial tiles, in that order.
-__global__ void __launch_bounds__(256) pba_dbias_reduce_kernel(const BwdArgs a) {
-    const long long n = (long long)a.H * a.Nq * a.Nk;
+    if (*abort_flag) return;
+    // Every partial of this CTA is written and fenced.  The tile's last CTA to get here sums
+    // the partials of all splits, in split order, into dbias.
+    __shared__ int s_last;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int tile = (h * a.nI + it) * a.nJ + jt;
+        s_last = atomicAdd(a.tile_count + tile, 1) == a.splits - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
     const long long plane = (long long)a.H * a.NqPad * a.NkPad;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
-         e += (long long)gridDim.x * blockDim.x) {
-        const int j = (int)(e % a.Nk);
-        const long long hi = e / a.Nk;
-        const int i = (int)(hi % a.Nq);
-        const int h = (int)(hi / a.Nq);
+    for (int v = threadIdx.x; v < 128 * 32; v += blockDim.x) {
+        const int i = i0 + (v >> 5), j = j0 + (v & 31) * 4;
+        if (i >= a.Nq || j >= a.Nk) continue;
         const float *src = a.dbias_part + ((long long)h * a.NqPad + i) * a.NkPad + j;
-        float s = 0.f;
-        for (int sp = 0; sp < a.splits; ++sp) s += src[sp * plane];
-        a.dbias[e] = s;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < a.splits; ++q) {
+            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + q * plane));
+            sum.x += v4.x;
+            sum.y += v4.y;
+            sum.z += v4.z;
+            sum.w += v4.w;
+        }
+        float *dst = a.dbias + ((long long)h * a.Nq + i) * a.Nk + j;
+        dst[0] = sum.x;
+        if (j + 1 < a.Nk) dst[1] = sum.y;
+        if (j + 2 < a.Nk) dst[2] = sum.z;
+        if (j + 3 < a.Nk) dst[3] = sum.w;
     }
 }
 
