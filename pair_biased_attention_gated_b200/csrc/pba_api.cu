@@ -292,8 +292,7 @@ BwdPlan plan_bwd(const pba_dims *d) {
     p.off_rs = 0;
     p.off_doa = align256(p.off_rs + rows * sizeof(float2));
     p.off_dq = align256(p.off_doa + elems * 2);
-    // per-tile counters of the dbias kernel right after the dQ accumulator: one memset
-    // clears both
+    // per-tile counters of the dbias kernel (cleared by the pre kernel)
     p.off_cnt = align256(p.off_dq + elems * 4);
     p.off_part = align256(p.off_cnt + (size_t)d->H * p.nI * p.nJ * sizeof(int));
     p.total = align256(p.off_part + (size_t)p.splits * d->H * p.NqPad * p.NkPad * 4);
@@ -405,8 +404,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     }
     cudaError_t e;
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
-    if ((e = cudaMemsetAsync(a.dqacc, 0, pl.off_part - pl.off_dq, s)) != cudaSuccess)
-        return cuda_fail(e, "cudaMemsetAsync");
+    // (the pre kernel clears the dQ accumulator and the dbias tile counters)
     const long long pre_rows = (long long)d->B * pl.NqPad * d->H;
     {
         ProfScope ps(K_BWD_PRE, s);

@@ -58,12 +58,18 @@ enum : unsigned {
 constexpr float kLog2eB = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------------------
-// pre: CP/8 lanes per query row (16 bytes of each tensor per lane), rows r = (b, h, i) with
-// i < NqPad fastest, so row stats and lse are read and written contiguously; padded rows
-// only get row stats
+// pre: CP/8 lanes per query row (16 bytes of each tensor per lane), rows r = (b, i, h) with
+// h fastest, so a warp's rows are contiguous in the [B][N][H][C] tensors; padded rows
+// (i >= Nq) only get row stats
 // ---------------------------------------------------------------------------------------
+// It also clears the dQ accumulator and the dbias tile counters for the kernels after it.
 template <int CP>
 __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
+    {
+        const int ntiles = a.H * a.nI * a.nJ;
+        for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < ntiles; x += gridDim.x * blockDim.x)
+            a.tile_count[x] = 0;
+    }
     constexpr int LPR = CP / 8;        // lanes per row
     constexpr int RPW = 32 / LPR;      // rows per warp
     const int lane = threadIdx.x & 31, sub = lane % LPR, rw = lane / LPR;
@@ -75,14 +81,17 @@ __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
         const bool in = r < nrows;
         int i = 0, h = 0, b = 0;
         if (in) {
-            i = (int)(r % a.NqPad);
-            const long long bh = r / a.NqPad;
-            h = (int)(bh % a.H);
-            b = (int)(bh / a.H);
+            h = (int)(r % a.H);
+            const long long bi = r / a.H;
+            i = (int)(bi % a.NqPad);
+            b = (int)(bi / a.NqPad);
         }
         float D = 0.f;
         const int c0 = sub * 8;
         if (in && i < a.Nq && c0 < a.C) {
+            float4 *acc = reinterpret_cast<float4 *>(a.dqacc + (((long long)b * a.Nq + i) * a.H + h) * a.C + c0);
+            acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
             const long long orow = b * a.so0 + (long long)i * a.so1 + h * a.so2 + c0;
             const uint4 o4 = *reinterpret_cast<const uint4 *>(a.out + orow);
             const uint4 d4 = *reinterpret_cast<const uint4 *>(a.dout + orow);
@@ -124,7 +133,7 @@ __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
                 rs.x = (l == -INFINITY) ? INFINITY : l * kLog2eB;
                 rs.y = D;
             }
-            a.rowstats[r] = rs;   // [B][H][NqPad]
+            a.rowstats[((long long)b * a.H + h) * a.NqPad + i] = rs;   // [B][H][NqPad]
         }
     }
 }
