@@ -127,6 +127,20 @@ pba_status map_bnhc(CUtensorMap *m, const void *base, int B, int N, int H, int C
     return PBA_OK;
 }
 
+// The dense fp32 [B, Nq, H, C] dQ accumulator as a 4-D map (C, H, Nq, B), box (32, 1, 128, 1),
+// 128-byte swizzle (rows of 32 fp32), for the backward's TMA reductions.
+pba_status map_dqacc(CUtensorMap *m, void *base, int B, int Nq, int H, int C) {
+    cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)(Nq > 0 ? Nq : 1), (cuuint64_t)(B > 0 ? B : 1)};
+    cuuint64_t strides[3] = {(cuuint64_t)C * 4, (cuuint64_t)H * C * 4, (cuuint64_t)Nq * H * C * 4};
+    cuuint32_t box[4] = {32, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "tensor map for the dQ accumulator failed (CUresult %d)", (int)r);
+    return PBA_OK;
+}
+
 // The [H, Nq, Nk] bias as a 3-D map (Nk, Nq, H), box (64, 128, 1), 128-byte swizzle.
 pba_status map_bias(CUtensorMap *m, const void *base, int H, int Nq, int Nk, const int64_t s[2]) {
     cuuint64_t dims[3] = {(cuuint64_t)(Nk > 0 ? Nk : 1), (cuuint64_t)(Nq > 0 ? Nq : 1), (cuuint64_t)H};
@@ -387,7 +401,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.tile_count = reinterpret_cast<int *>(w + pl.off_cnt);
 
     pba_status st;
-    CUtensorMap tq, tk, tv, tdo, tb;
+    CUtensorMap tq, tk, tv, tdo, tb, tdq;
     if ((st = map_bnhc(&tq, q, d->B, d->Nq, d->H, d->C, d->sq, CP, "q")) != PBA_OK) return st;
     if ((st = map_bnhc(&tk, k, d->B, d->Nk, d->H, d->C, d->sk, CP, "k")) != PBA_OK) return st;
     if ((st = map_bnhc(&tv, v, d->B, d->Nk, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
@@ -402,10 +416,16 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     } else {
         std::memset(&tb, 0, sizeof(tb));
     }
+    if (MT::DQ_TMA) {
+        if ((st = map_dqacc(&tdq, a.dqacc, d->B, d->Nq, d->H, d->C)) != PBA_OK) return st;
+    } else {
+        std::memset(&tdq, 0, sizeof(tdq));
+    }
     cudaError_t e;
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
     // (the pre kernel clears the dQ accumulator and the dbias tile counters)
     const long long pre_rows = (long long)d->B * pl.NqPad * d->H;
+    if (pre_rows >= (1LL << 31)) return fail(PBA_ERR_UNSUPPORTED, "B * Nq * H must be below 2^31");
     {
         ProfScope ps(K_BWD_PRE, s);
         pba::pba_bwd_pre_kernel<CP><<<grid_for(pre_rows * (CP / 8), 256), 256, 0, s>>>(a);
@@ -419,7 +439,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         const long long grid = items < num_sms() ? items : num_sms();
         {
             ProfScope ps(K_BWD_MAIN, s);
-            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 352, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 352, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, tdq, a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {

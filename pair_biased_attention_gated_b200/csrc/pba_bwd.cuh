@@ -80,11 +80,12 @@ __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
         const long long r = r0 + rw;
         const bool in = r < nrows;
         int i = 0, h = 0, b = 0;
-        if (in) {
-            h = (int)(r % a.H);
-            const long long bi = r / a.H;
-            i = (int)(bi % a.NqPad);
-            b = (int)(bi / a.NqPad);
+        if (in) {   // nrows < 2^31 (checked on the host): 32-bit index arithmetic
+            const int r32 = (int)r;
+            h = r32 % a.H;
+            const int bi = r32 / a.H;
+            i = bi % a.NqPad;
+            b = bi / a.NqPad;
         }
         float D = 0.f;
         const int c0 = sub * 8;
@@ -207,7 +208,10 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct BwdTraits {
-    static constexpr int QS = (CP == 64) ? 2 : 3;               // Q/dOa/row-stat stages
+    // dQ partials (CP = 32): written into a 128-byte-swizzled fp32 staging tile and added to
+    // the accumulator by one TMA tensor reduction per step; otherwise vector reductions
+    static constexpr bool DQ_TMA = CP == 32;
+    static constexpr int QS = (CP == 16) ? 3 : 2;               // Q/dOa/row-stat stages
     static constexpr int BS = (CP == 64) ? 1 : 2;               // bias stages
     static constexpr int KVB = (CP == 64) ? 1 : 2;              // K/V stages (items)
     static constexpr int DKB = (CP == 64) ? 1 : 2;              // dK/dV TMEM buffers (items)
@@ -222,7 +226,8 @@ struct BwdTraits {
     static constexpr int OFF_BIAS = OFF_DS + PS_BYTES;          // + bs * BIAS_BYTES
     static constexpr int OFF_RS = OFF_BIAS + BS * BIAS_BYTES;   // float2 [QS][128]
     static constexpr int OFF_MASK = OFF_RS + QS * 1024;         // u32 [KVB][8]
-    static constexpr int SMEM_BYTES = OFF_MASK + KVB * 32 + 1024;
+    static constexpr int OFF_DQS = OFF_MASK + 1024;             // fp32 [128][CP] staging (DQ_TMA)
+    static constexpr int SMEM_BYTES = OFF_DQS + (DQ_TMA ? 128 * CP * 4 : 0) + 1024;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
     static constexpr uint32_t ROWB = CP * 2;
     // TMEM columns: S, dP, then per dK/dV buffer x: dK at T_DK + 2 CP x, dV after it, then
@@ -241,11 +246,12 @@ template <int CP>
 __global__ void __launch_bounds__(352, 1)
 pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tmBias, const __grid_constant__ CUtensorMap tmDQ,
+                    const BwdArgs a) {
     using T = BwdTraits<CP>;
     constexpr int QS = T::QS, BS = T::BS, KVB = T::KVB, DKB = T::DKB;
     extern __shared__ uint8_t dsmem[];
-    __shared__ __align__(8) uint64_t bars[16 + 2 * QS + 2 * BS + 2 * KVB + 2 * DKB];
+    __shared__ __align__(8) uint64_t bars[16 + 2 * QS + 2 * BS + 2 * KVB + 2 * DKB + 2];
     __shared__ uint32_t s_tmem_base;
     __shared__ int s_abort;
 
@@ -265,6 +271,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     auto b_kv_empty = [&](int x) { return smem_u32(&bars[OK_ + KVB + x]); };   // item's MMAs done
     auto b_dkv_full = [&](int x) { return smem_u32(&bars[OK_ + 2 * KVB + x]); };        // dK/dV final
     auto b_dkv_free = [&](int x) { return smem_u32(&bars[OK_ + 2 * KVB + DKB + x]); };  // read out
+    const uint32_t b_stg_full = smem_u32(&bars[OK_ + 2 * KVB + 2 * DKB]);       // dQ staging written
+    const uint32_t b_stg_free = smem_u32(&bars[OK_ + 2 * KVB + 2 * DKB + 1]);   // staging read by TMA
 
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -313,6 +321,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_init(b_dkv_full(x), 1);
             mbar_init(b_dkv_free(x), 256);
         }
+        mbar_init(b_stg_full, 256);
+        mbar_init(b_stg_free, 1);
         s_abort = 0;
         fence_mbar_init();
     }
@@ -502,7 +512,35 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             mbar_arrive(b_dq_free(t & 1));
             const int i = (t % nI) * 128 + row;
-            if (i < a.Nq) {
+            if constexpr (T::DQ_TMA) {
+                // the staging tile of the previous flush has been read by its TMA reduction:
+                // thread 0, which issued it, checks that here (a step later, so it no longer
+                // waits) and releases the tile
+                if (t > 0) {
+                    if (threadIdx.x == 0) {
+                        bulk_wait_read_all();
+                        mbar_arrive(b_stg_free);
+                    }
+                    okf = mbar_wait(b_stg_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x70 | (t << 12));
+                    okf = __all_sync(0xffffffffu, okf);
+                    if (!okf) return false;
+                }
+                // this thread's 16 channels = 16-byte chunks 4 e .. 4 e + 3 of row `row`
+                const uint32_t srow = sbase + T::OFF_DQS + row * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    sts128(srow + (((e * 4 + q4) ^ (row & 7)) << 4),
+                           make_uint4(r[q4 * 4], r[q4 * 4 + 1], r[q4 * 4 + 2], r[q4 * 4 + 3]));
+                fence_proxy_async();
+                mbar_arrive(b_stg_full);
+                if (threadIdx.x == 0) {
+                    // rows >= Nq and channels >= C fall outside the map and are skipped
+                    okf = mbar_wait(b_stg_full, t & 1, abort_flag, SITE_BWD_EW | 0x80 | (t << 12));
+                    if (!okf) return false;
+                    tma_reduce_add_4d(&tmDQ, sbase + T::OFF_DQS, 0, it.h, (t % nI) * 128, it.b);
+                    bulk_commit();
+                }
+            } else if (i < a.Nq) {
                 float *dst = a.dqacc + (((long long)it.b * a.Nq + i) * a.H + it.h) * a.C;
 #pragma unroll
                 for (int c4 = 0; c4 < CP / 8; ++c4) {
@@ -600,6 +638,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         if (ok && Tn > 0) ok = flush_dq(Tn - 1, cur);
         if (ok && M > 0) ok = epilogue(M - 1, cur);
+        if (T::DQ_TMA && threadIdx.x == 0) bulk_wait_all();   // its TMA reductions are done
     }
 
     tc_fence_before();
@@ -865,19 +904,22 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 // dq = bf16(scale * dqacc), eight channels per thread.
 __global__ void __launch_bounds__(256) pba_dq_convert_kernel(const BwdArgs a) {
+    // element groups e = (row r, c8) with r = (b, i, h) < 2^31 rows (checked on the host):
+    // 32-bit index arithmetic
     const int c8n = a.C / 8;
-    const long long n = (long long)a.B * a.Nq * a.H * c8n;
+    const int nrows = a.B * a.Nq * a.H;
+    const long long n = (long long)nrows * c8n;
+    const float s = a.scale;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
          e += (long long)gridDim.x * blockDim.x) {
-        const int c8 = (int)(e % c8n);
-        const long long r = e / c8n;
-        const int h = (int)(r % a.H);
-        const long long bi = r / a.H;
-        const int i = (int)(bi % a.Nq);
-        const int b = (int)(bi / a.Nq);
-        const float4 *src = reinterpret_cast<const float4 *>(a.dqacc + r * a.C + c8 * 8);
-        const float4 x0 = src[0], x1 = src[1];
-        const float s = a.scale;
+        const int r = (int)(e / c8n);
+        const int c8 = (int)(e - (long long)r * c8n);
+        const int h = r % a.H;
+        const int bi = r / a.H;
+        const int i = bi % a.Nq;
+        const int b = bi / a.Nq;
+        const float4 *src = reinterpret_cast<const float4 *>(a.dqacc + (long long)r * a.C + c8 * 8);
+        const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
         __nv_bfloat16 *dst = a.dq + b * a.sq0 + (long long)i * a.sq1 + h * a.sq2 + c8 * 8;
         *reinterpret_cast<uint4 *>(dst) =
             make_uint4(pack_bf16x2(x0.x * s, x0.y * s), pack_bf16x2(x0.z * s, x0.w * s),

@@ -80,6 +80,12 @@ CASES = {
     "single_row_head": (1, 1, 256, 256, 32, ((250, 256),), True, True),
     "three_key_tiles": (10, 2, 384, 384, 32, ((100, 140), (300, 384)), True, True),
     "many_rows_split": (70, 1, 128, 128, 32, ((120, 128),), True, True),
+    # more (b, h, key tile) items than SMs: CTAs of the dq/dk/dv kernel run several items,
+    # crossing K/V stages and dK/dV buffers (one of each at c = 64)
+    "multi_item_c32": (40, 4, 136, 136, 32, ((130, 136),), True, True),
+    "multi_item_c24": (30, 4, 200, 200, 24, ((190, 200),), True, True),
+    "multi_item_c16": (40, 4, 72, 72, 16, (), True, True),
+    "multi_item_c64": (24, 4, 136, 136, 64, ((0, 3),), True, True),
 }
 
 
