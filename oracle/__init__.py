@@ -51,6 +51,8 @@ def _load():
                                        d, d]
         lib.pba_oracle_dbias_row.argtypes = [i, i, i, i, i, f, i, i, d, d, d, d, u8, ll, d, d,
                                              d]
+        lib.pba_oracle_pwa_fwd.argtypes = [i, i, i, i, d, d, u8, d, d, d]
+        lib.pba_oracle_pwa_bwd.argtypes = [i, i, i, i, d, d, u8, d, d, d, d, d]
         lib.pba_oracle_threads.argtypes = []
         lib.pba_oracle_threads.restype = ctypes.c_int
         _lib = lib
@@ -175,3 +177,31 @@ def dbias_row(q, k, v, bias, keep, g, dout, h, i, scale=None):
     lib.pba_oracle_dbias_row(B, H, Nq, Nk, C, scale, int(h), int(i), _d(q), _d(k), _d(v),
                              _d(bias), _u8(keep), ksb, _d(g), _d(dout), _d(row))
     return row
+
+
+def pwa_fwd(v, bias=None, keep=None, g=None):
+    """MSA pair-weighted averaging: out [B,N,H,C] and lse_w [H,N] (weights softmax_j(bias
+    + mask), shared by every row b; keep is one [N] row or None)."""
+    lib = _load()
+    v, bias, g = map(_f64, (v, bias, g))
+    B, N, H, C = v.shape
+    keep = None if keep is None else np.ascontiguousarray(keep, dtype=np.uint8).reshape(N)
+    out = np.empty((B, N, H, C))
+    lse = np.empty((H, N))
+    lib.pba_oracle_pwa_fwd(B, H, N, C, _d(v), _d(bias), _u8(keep), _d(g), _d(out), _d(lse))
+    return out, lse
+
+
+def pwa_bwd(v, bias, keep, g, dout):
+    """dv [B,N,H,C], dg (None without gate), dbias [H,N,N] of MSA pair-weighted averaging."""
+    lib = _load()
+    v, bias, g, dout = map(_f64, (v, bias, g, dout))
+    B, N, H, C = v.shape
+    keep = None if keep is None else np.ascontiguousarray(keep, dtype=np.uint8).reshape(N)
+    dv = np.empty_like(v)
+    dg = np.empty_like(v) if g is not None else None
+    dbias = np.empty((H, N, N))
+    lib.pba_oracle_pwa_bwd(B, H, N, C, _d(v), _d(bias), _u8(keep), _d(g), _d(dout), _d(dv), _d(dg),
+                           _d(dbias))
+    return dv, dg, dbias
+

@@ -292,3 +292,114 @@ void pba_oracle_dbias_row(int B, int H, int Nq, int Nk, int C, double scale, int
     }
     free(qi); free(dOa); free(ks); free(vs); free(s); free(p); free(dP);
 }
+
+/*
+ * MSA pair-weighted averaging ("AlphaFold3 open-source implementation" page, sections
+ * "MSA Pair Averaging" and "Model Efficiency"): the MSA module averages the value rows of
+ * every MSA sequence with weights taken from the pair representation alone.  The pages
+ * print no formula; the plainest reading, the gated operator above without its key-query
+ * term, shared by all B rows (Nq = Nk = N, key mask one row shared by all b):
+ *
+ *   w[h,i,j]    = exp(bias[h,i,j] - m_i) / sum_j' exp(bias[h,i,j'] - m_i)  (masked j: w = 0)
+ *   lse_w[h,i]  = m_i + ln sum_j exp(bias[h,i,j] - m_i)                    (-inf: all masked)
+ *   o[b,i,h,c]  = sum_j w[h,i,j] v[b,j,h,c] ;   out = sigmoid(g) * o
+ *
+ *   Backward:  dOa = dout * sigmoid(g) ;  dg = dout * o * sigmoid(g) (1 - sigmoid(g))
+ *              dv[b,j,h,c] = sum_i w[h,i,j] dOa[b,i,h,c]
+ *              dW[h,i,j]   = sum_b sum_c dOa[b,i,h,c] v[b,j,h,c]
+ *              dbias[h,i,j] = w[h,i,j] (dW[h,i,j] - sum_j' w[h,i,j'] dW[h,i,j'])
+ *
+ * Layouts: v, g, out, dout, dv, dg are [B, N, H, C]; bias, dbias are [H, N, N]; keep is
+ * [N] (1 = attended) or NULL; lse_w is [H, N].
+ */
+static void pwa_weights(int N, const double *brow, const uint8_t *keep, double *w, double *lse)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < N; ++j)
+        if (!keep || keep[j]) m = fmax(m, brow ? brow[j] : 0.0);
+    if (m == -INFINITY) {   /* every key masked */
+        for (int j = 0; j < N; ++j) w[j] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    for (int j = 0; j < N; ++j) {
+        w[j] = (!keep || keep[j]) ? exp((brow ? brow[j] : 0.0) - m) : 0.0;
+        l += w[j];
+    }
+    for (int j = 0; j < N; ++j) w[j] /= l;
+    *lse = m + log(l);
+}
+
+void pba_oracle_pwa_fwd(int B, int H, int N, int C, const double *v, const double *bias,
+                        const uint8_t *keep, const double *g, double *out, double *lse)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int h = 0; h < H; ++h) {
+        double *w = malloc(sizeof(double) * (size_t)N + 8);
+        for (int i = 0; i < N; ++i) {
+            pwa_weights(N, bias ? bias + ((size_t)h * N + i) * N : NULL, keep, w,
+                        lse + (size_t)h * N + i);
+            for (int b = 0; b < B; ++b)
+                for (int c = 0; c < C; ++c) {
+                    double o = 0.0;
+                    for (int j = 0; j < N; ++j) o += w[j] * v[(((size_t)b * N + j) * H + h) * C + c];
+                    const size_t e = (((size_t)b * N + i) * H + h) * C + c;
+                    out[e] = g ? sigmoid(g[e]) * o : o;
+                }
+        }
+        free(w);
+    }
+}
+
+void pba_oracle_pwa_bwd(int B, int H, int N, int C, const double *v, const double *bias,
+                        const uint8_t *keep, const double *g, const double *dout, double *dv,
+                        double *dg, double *dbias)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int h = 0; h < H; ++h) {
+        double *w = malloc(sizeof(double) * (size_t)N * N + 8);
+        double *lse = malloc(sizeof(double) * (size_t)N + 8);
+        double *doa = malloc(sizeof(double) * (size_t)B * N * C + 8);   /* [b][i][c] */
+        for (int i = 0; i < N; ++i)
+            pwa_weights(N, bias ? bias + ((size_t)h * N + i) * N : NULL, keep, w + (size_t)i * N, lse + i);
+        /* dOa and dg need the ungated o */
+        for (int b = 0; b < B; ++b)
+            for (int i = 0; i < N; ++i)
+                for (int c = 0; c < C; ++c) {
+                    const size_t e = (((size_t)b * N + i) * H + h) * C + c;
+                    double o = 0.0;
+                    for (int j = 0; j < N; ++j) o += w[(size_t)i * N + j] * v[(((size_t)b * N + j) * H + h) * C + c];
+                    const double s = g ? sigmoid(g[e]) : 1.0;
+                    doa[((size_t)b * N + i) * C + c] = dout[e] * s;
+                    if (g && dg) dg[e] = dout[e] * o * s * (1.0 - s);
+                }
+        /* dv[b,j] = sum_i w[i,j] dOa[b,i] */
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < N; ++j)
+                for (int c = 0; c < C; ++c) {
+                    double a = 0.0;
+                    for (int i = 0; i < N; ++i) a += w[(size_t)i * N + j] * doa[((size_t)b * N + i) * C + c];
+                    dv[(((size_t)b * N + j) * H + h) * C + c] = a;
+                }
+        /* dW[i,j] = sum_b sum_c dOa[b,i,c] v[b,j,c]; dbias = w (dW - sum_j w dW), row by row */
+        if (dbias) {
+            double *dw = malloc(sizeof(double) * (size_t)N + 8);
+            for (int i = 0; i < N; ++i) {
+                for (int j = 0; j < N; ++j) {
+                    double a = 0.0;
+                    for (int b = 0; b < B; ++b)
+                        for (int c = 0; c < C; ++c)
+                            a += doa[((size_t)b * N + i) * C + c] * v[(((size_t)b * N + j) * H + h) * C + c];
+                    dw[j] = a;
+                }
+                double r = 0.0;
+                for (int j = 0; j < N; ++j) r += w[(size_t)i * N + j] * dw[j];
+                for (int j = 0; j < N; ++j)
+                    dbias[((size_t)h * N + i) * N + j] = w[(size_t)i * N + j] * (dw[j] - r);
+            }
+            free(dw);
+        }
+        free(w); free(lse); free(doa);
+    }
+}
