@@ -136,6 +136,43 @@ pba_status pba_bwd_noalloc(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 
                            pba_bf16 *dgate, const pba_dims *dims, void *stream);
 
 /*
+ * MSA pair-weighted averaging ("AlphaFold3 open-source implementation" page, sections "MSA
+ * Pair Averaging" and "Model Efficiency"): the value rows of every broadcast row b (MSA
+ * sequence) are averaged with weights taken from the pair representation alone, shared by
+ * all rows -- the operator above without its key-query term:
+ *   w[h,i,j] = softmax_j(bias[h,i,j] + mask_j),  lse_w[h,i] = ln sum_j exp(bias + mask)
+ *   out[b,i,h,:] = sigmoid(gate[b,i,h,:]) * sum_j w[h,i,j] v[b,j,h,:]      (no gate: no factor)
+ * The weights are computed once per (h, i), not per b.  Arguments follow pba_fwd with
+ * Nq = Nk = N (else PBA_ERR_UNSUPPORTED): v, gate, out use dims->sv, sg, so; bias (nullable,
+ * = 0) dims->sbias; key_mask (nullable) is one [N] row shared by every b (dims->smask_b must
+ * be 0 when B > 1, else PBA_ERR_UNSUPPORTED).  dims->scale and q/k strides are ignored.
+ * lse_w: fp32 [H, N], written; -inf for a row whose keys are all masked (its out is 0).
+ * workspace: caller-owned device memory of pba_pwa_fwd_workspace_size(dims) bytes,
+ * 256-byte aligned (PBA_ERR_WORKSPACE if smaller); it holds the bf16 weights.
+ */
+size_t pba_pwa_fwd_workspace_size(const pba_dims *dims);
+pba_status pba_pwa_fwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *key_mask,
+                       const pba_bf16 *gate, pba_bf16 *out, float *lse_w, void *workspace,
+                       size_t workspace_bytes, const pba_dims *dims, void *stream);
+
+/*
+ * Backward of pba_pwa_fwd, given v, bias, key_mask, gate, the forward output `out` (only
+ * needed with a gate) and dout:
+ *   dOa = dout * sigmoid(gate);  dgate = dout * out * (1 - sigmoid(gate))
+ *   dv[b,j,h,:] = sum_i w[h,i,j] dOa[b,i,h,:]
+ *   dW[h,i,j] = sum_b sum_c dOa[b,i,h,c] v[b,j,h,c];  dbias = w * (dW - sum_j w dW)
+ * dv (required, strides of v), dgate (required iff gate), dbias (fp32 [H,N,N], may be NULL
+ * to skip it; bit-identical from run to run: fixed reduction orders).  The weights are
+ * recomputed from bias and key_mask.  workspace: pba_pwa_bwd_workspace_size(dims) bytes,
+ * 256-byte aligned.
+ */
+size_t pba_pwa_bwd_workspace_size(const pba_dims *dims);
+pba_status pba_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *key_mask,
+                       const pba_bf16 *gate, const pba_bf16 *out, const pba_bf16 *dout,
+                       pba_bf16 *dv, float *dbias, pba_bf16 *dgate, void *workspace,
+                       size_t workspace_bytes, const pba_dims *dims, void *stream);
+
+/*
  * Synchronizes `stream`, then reports and clears the device watchdog word of the
  * current device: PBA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, PBA_ERR_CUDA if the synchronization itself failed, else PBA_OK.

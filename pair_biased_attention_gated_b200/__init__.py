@@ -49,6 +49,14 @@ lib.pba_bwd.argtypes = [_vp] * 14 + [_vp, ctypes.c_size_t, ctypes.POINTER(PbaDim
 lib.pba_bwd.restype = ctypes.c_int
 lib.pba_bwd_noalloc.argtypes = [_vp] * 14 + [ctypes.POINTER(PbaDims), _vp]
 lib.pba_bwd_noalloc.restype = ctypes.c_int
+lib.pba_pwa_fwd_workspace_size.argtypes = [ctypes.POINTER(PbaDims)]
+lib.pba_pwa_fwd_workspace_size.restype = ctypes.c_size_t
+lib.pba_pwa_bwd_workspace_size.argtypes = [ctypes.POINTER(PbaDims)]
+lib.pba_pwa_bwd_workspace_size.restype = ctypes.c_size_t
+lib.pba_pwa_fwd.argtypes = [_vp] * 7 + [ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
+lib.pba_pwa_fwd.restype = ctypes.c_int
+lib.pba_pwa_bwd.argtypes = [_vp] * 10 + [ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
+lib.pba_pwa_bwd.restype = ctypes.c_int
 lib.pba_device_status.argtypes = [_vp]
 lib.pba_device_status.restype = ctypes.c_int
 lib.pba_status_string.argtypes = [ctypes.c_int]
@@ -169,6 +177,40 @@ def pba_bwd_noalloc(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, d
                                ctypes.byref(d), _stream(stream)))
 
 
+def pwa_dims(v, gate=None, out=None, bias=None, key_mask=None, dout=None) -> PbaDims:
+    """pba_dims for MSA pair-weighted averaging: v/gate/out [B,N,H,C], bias [H,N,N],
+    key_mask one [N] row shared by every b."""
+    d = make_dims(v, v, v, gate, out, bias, key_mask, 0.0, dout=dout)
+    d.smask_b = 0
+    return d
+
+
+def pba_pwa_fwd(v, bias, key_mask, gate, out, lse_w, workspace, stream=None) -> None:
+    """Pair-weighted averaging forward into preallocated `out` (like v) and `lse_w` (fp32
+    [H,N]); `workspace`: uint8 CUDA tensor of pba_pwa_fwd_workspace_size bytes."""
+    if key_mask is not None and key_mask.dim() != 1:
+        raise ValueError("pair-weighted averaging takes one [N] key mask shared by every row")
+    d = pwa_dims(v, gate, out, bias, key_mask)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pba_pwa_fwd(_ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate), _ptr(out), _ptr(lse_w),
+                           _ptr(workspace), ws_bytes, ctypes.byref(d), _stream(stream)))
+
+
+def pba_pwa_bwd(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, workspace, stream=None) -> None:
+    """Pair-weighted averaging backward into preallocated dv (like v), dbias (fp32 [H,N,N] or
+    None) and dgate (like gate, or None)."""
+    if key_mask is not None and key_mask.dim() != 1:
+        raise ValueError("pair-weighted averaging takes one [N] key mask shared by every row")
+    d = pwa_dims(v, gate, out, bias, key_mask, dout=dout)
+    for name, a, b in (("dv", dv, v), ("dgate", dgate, gate), ("dout", dout, out)):
+        if a is not None and b is not None and a.stride() != b.stride():
+            raise ValueError("%s must have the same strides as its forward tensor" % name)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pba_pwa_bwd(_ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate), _ptr(out), _ptr(dout),
+                           _ptr(dv), _ptr(dbias), _ptr(dgate), _ptr(workspace), ws_bytes,
+                           ctypes.byref(d), _stream(stream)))
+
+
 def pba_device_status(stream=None) -> None:
     """Synchronize the stream and raise if a kernel's bounded wait ran out."""
     _check(lib.pba_device_status(_stream(stream)))
@@ -219,3 +261,30 @@ def profile_read() -> dict:
     if n < 0:
         raise PbaError(3, "reading kernel timing events failed")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}
+
+
+def pwa_fwd(v, bias=None, key_mask=None, gate=None, stream=None):
+    """MSA pair-weighted averaging: out = sigmoid(gate) * sum_j softmax_j(bias + mask) v."""
+    import torch
+    B, N, H, C = v.shape
+    out = torch.empty_like(v)
+    lse_w = torch.empty((H, N), dtype=torch.float32, device=v.device)
+    d = pwa_dims(v, gate, out, bias, key_mask)
+    ws = torch.empty(max(int(lib.pba_pwa_fwd_workspace_size(ctypes.byref(d))), 1), dtype=torch.uint8,
+                     device=v.device)
+    pba_pwa_fwd(v, bias, key_mask, gate, out, lse_w, ws, stream)
+    return out, lse_w
+
+
+def pwa_bwd(v, bias, key_mask, gate, out, dout, want_dbias: bool = True, stream=None):
+    import torch
+    B, N, H, C = v.shape
+    dv = torch.empty_like(v)
+    dgate = torch.empty_like(gate) if gate is not None else None
+    dbias = torch.empty((H, N, N), dtype=torch.float32, device=v.device) if want_dbias else None
+    d = pwa_dims(v, gate, out, bias, key_mask, dout=dout)
+    ws = torch.empty(max(int(lib.pba_pwa_bwd_workspace_size(ctypes.byref(d))), 1), dtype=torch.uint8,
+                     device=v.device)
+    pba_pwa_bwd(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, stream)
+    return dv, dgate, dbias
+

@@ -18,6 +18,7 @@
 #include "../../include/pba.h"
 #include "pba_bwd.cuh"
 #include "pba_fwd.cuh"
+#include "pba_pwa.cuh"
 
 namespace {
 
@@ -39,10 +40,14 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 // ---------------------------------------------------------------------------- profiling
-enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS, K_COUNT };
+enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS,
+                K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS, K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
                                            "pba_dbias_kernel",
-                                           "pba_dq_convert_kernel", "zero_rows_kernel"};
+                                           "pba_dq_convert_kernel", "zero_rows_kernel",
+                                           "pba_pwa_weights_kernel", "pba_pwa_gemm_kernel (out)",
+                                           "pba_pwa_pre_kernel", "pba_pwa_gemm_kernel (dv)",
+                                           "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel"};
 struct ProfRec {
     int kid;
     cudaEvent_t a, b;
@@ -487,6 +492,212 @@ pba_status noalloc_scratch(void **out) {
     return PBA_OK;
 }
 
+
+// ---------------------------------------------------------------------------- pair-weighted
+// The [H, N, Wld] bf16 weights as a 3-D map (N, N, H), box (64, 128, 1), 128-byte swizzle:
+// the same tiles as the bias.
+pba_status map_w(CUtensorMap *m, void *base, int H, int N, int Wld) {
+    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H};
+    cuuint64_t strides[2] = {(cuuint64_t)Wld * 2, (cuuint64_t)N * Wld * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "tensor map for the weights failed (CUresult %d)", (int)r);
+    return PBA_OK;
+}
+
+struct PwaPlan {
+    int N, Wld, NPad, nT, splits, rows_per_split;
+    size_t off_w, off_lse, off_doa, off_part, fwd_total, bwd_total;
+};
+
+PwaPlan plan_pwa(const pba_dims *d) {
+    PwaPlan p;
+    p.N = d->Nq;
+    p.Wld = (p.N + 7) / 8 * 8;
+    p.nT = (p.N + 127) / 128;
+    p.NPad = p.nT * 128;
+    // splits of the rows b for the dW partials: a function of the sizes only (bit-stable
+    // dbias), chosen like the attention's dbias splits
+    const long long tiles = (long long)d->H * p.nT * p.nT;
+    const long long maxs = d->B < 64 ? (d->B > 0 ? d->B : 1) : 64;
+    long long best = -1;
+    p.splits = 1;
+    p.rows_per_split = d->B > 0 ? d->B : 1;
+    for (long long sp = 1; sp <= maxs; ++sp) {
+        const long long rows = d->B > 0 ? (d->B + sp - 1) / sp : 1;
+        const long long actual = d->B > 0 ? (d->B + rows - 1) / rows : 1;
+        const long long waves = (tiles * actual + 2 * kSmCount - 1) / (2 * kSmCount);   // 2 CTAs per SM
+        const long long cost = waves * (rows + 3);
+        if (best < 0 || cost < best) {
+            best = cost;
+            p.splits = (int)actual;
+            p.rows_per_split = (int)rows;
+        }
+    }
+    p.off_w = 0;
+    p.fwd_total = align256((size_t)d->H * p.N * p.Wld * 2);
+    p.off_lse = p.fwd_total;
+    p.off_doa = align256(p.off_lse + (size_t)d->H * p.N * 4);
+    p.off_part = align256(p.off_doa + (size_t)d->B * p.N * d->H * d->C * 2);
+    p.bwd_total = align256(p.off_part + (size_t)p.splits * d->H * p.NPad * p.NPad * 4);
+    return p;
+}
+
+pba_status check_pwa_dims(const pba_dims *d) {
+    pba_status st = check_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->Nq != d->Nk) return fail(PBA_ERR_UNSUPPORTED, "pair-weighted averaging needs Nq == Nk");
+    if (d->smask_b != 0 && d->B > 1)
+        return fail(PBA_ERR_UNSUPPORTED, "pair-weighted averaging needs a key mask shared by every row (smask_b = 0)");
+    return PBA_OK;
+}
+
+void fill_pwa_args(pba::PwaArgs &a, const PwaPlan &pl, const pba_dims *d, const pba_bf16 *bias,
+                   const uint8_t *mask, const pba_bf16 *gate, uint8_t *ws) {
+    std::memset(&a, 0, sizeof(a));
+    a.B = d->B; a.H = d->H; a.N = pl.N; a.C = d->C;
+    a.nT = pl.nT; a.NPad = pl.NPad; a.Wld = pl.Wld;
+    a.splits = pl.splits; a.rows_per_split = pl.rows_per_split;
+    a.has_bias = bias != nullptr;
+    a.has_gate = gate != nullptr;
+    a.bias = reinterpret_cast<const __nv_bfloat16 *>(bias);
+    a.sb0 = d->sbias[0]; a.sb1 = d->sbias[1];
+    a.mask = mask;
+    a.gate = reinterpret_cast<const __nv_bfloat16 *>(gate);
+    a.sg0 = d->sg[0]; a.sg1 = d->sg[1]; a.sg2 = d->sg[2];
+    a.w = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_w);
+}
+
+template <int CP>
+pba_status launch_pwa_gemm(const CUtensorMap &tw, const CUtensorMap &tx, const pba::PwaArgs &a0, bool dv,
+                           cudaStream_t s) {
+    using T = pba::PwaTraits<CP>;
+    pba::PwaArgs a = a0;
+    a.nChunks = (a.B + T::BC - 1) / T::BC;
+    const long long grid = (long long)a.H * a.nT * a.nChunks;
+    if (dv) {
+        pba_status st = set_smem(pba::pba_pwa_gemm_kernel<CP, true>, T::SMEM_BYTES);
+        if (st != PBA_OK) return st;
+        cudaFuncSetAttribute(pba::pba_pwa_gemm_kernel<CP, true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+        ProfScope ps(K_PWA_DV, s);
+        pba::pba_pwa_gemm_kernel<CP, true><<<(unsigned)grid, 192, T::SMEM_BYTES, s>>>(tw, tx, a);
+    } else {
+        pba_status st = set_smem(pba::pba_pwa_gemm_kernel<CP, false>, T::SMEM_BYTES);
+        if (st != PBA_OK) return st;
+        cudaFuncSetAttribute(pba::pba_pwa_gemm_kernel<CP, false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+        ProfScope ps(K_PWA_FWD, s);
+        pba::pba_pwa_gemm_kernel<CP, false><<<(unsigned)grid, 192, T::SMEM_BYTES, s>>>(tw, tx, a);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PBA_OK : cuda_fail(e, "pba_pwa_gemm_kernel launch");
+}
+
+pba_status launch_pwa_weights(const pba::PwaArgs &a, cudaStream_t s) {
+    {
+        ProfScope ps(K_PWA_WEIGHTS, s);
+        pba::pba_pwa_weights_kernel<<<grid_for((long long)a.H * a.N * 32, 256), 256, 0, s>>>(a);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PBA_OK : cuda_fail(e, "pba_pwa_weights_kernel launch");
+}
+
+template <int CP>
+pba_status launch_pwa_fwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
+                          pba_bf16 *out, float *lse, uint8_t *ws, const PwaPlan &pl, const pba_dims *d,
+                          cudaStream_t s) {
+    pba::PwaArgs a;
+    fill_pwa_args(a, pl, d, bias, mask, gate, ws);
+    a.lse = lse;
+    a.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
+    pba_status st;
+    CUtensorMap tw, tv;
+    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld)) != PBA_OK) return st;
+    if ((st = map_bnhc(&tv, v, d->B, pl.N, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
+    if ((st = launch_pwa_weights(a, s)) != PBA_OK) return st;
+    return launch_pwa_gemm<CP>(tw, tv, a, false, s);
+}
+
+template <int CP>
+pba_status launch_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
+                          const pba_bf16 *out, const pba_bf16 *dout, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                          uint8_t *ws, const PwaPlan &pl, const pba_dims *d, cudaStream_t s) {
+    using DT = pba::PwaDwTraits<CP>;
+    pba::PwaArgs a;
+    fill_pwa_args(a, pl, d, bias, mask, gate, ws);
+    a.lse = reinterpret_cast<float *>(ws + pl.off_lse);
+    a.doa = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_doa);
+    a.dw_part = reinterpret_cast<float *>(ws + pl.off_part);
+    a.dbias = dbias;
+    a.dgate = reinterpret_cast<__nv_bfloat16 *>(dgate);
+    a.oin = reinterpret_cast<const __nv_bfloat16 *>(out);
+    a.dout = reinterpret_cast<const __nv_bfloat16 *>(dout);
+    a.si0 = d->so[0]; a.si1 = d->so[1]; a.si2 = d->so[2];
+    pba_status st;
+    CUtensorMap tw, tv, tdo;
+    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld)) != PBA_OK) return st;
+    if ((st = map_bnhc(&tv, v, d->B, pl.N, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
+    if (gate) {
+        const int64_t sd[3] = {(int64_t)pl.N * d->H * d->C, (int64_t)d->H * d->C, d->C};
+        if ((st = map_bnhc(&tdo, a.doa, d->B, pl.N, d->H, d->C, sd, CP, "dOa")) != PBA_OK) return st;
+    } else {
+        if ((st = map_bnhc(&tdo, dout, d->B, pl.N, d->H, d->C, d->so, CP, "dout")) != PBA_OK) return st;
+    }
+    if ((st = launch_pwa_weights(a, s)) != PBA_OK) return st;
+    cudaError_t e;
+    if (gate) {
+        {
+            ProfScope ps(K_PWA_PRE, s);
+            pba::pba_pwa_pre_kernel<<<grid_for((long long)d->B * pl.N * d->H * (d->C / 8), 256), 256, 0, s>>>(a);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pwa_pre_kernel launch");
+    }
+    // dv = W^T dOa (rows j)
+    pba::PwaArgs av = a;
+    av.out = reinterpret_cast<__nv_bfloat16 *>(dv);
+    av.so0 = d->sv[0]; av.so1 = d->sv[1]; av.so2 = d->sv[2];
+    if ((st = launch_pwa_gemm<CP>(tw, tdo, av, true, s)) != PBA_OK) return st;
+    if (dbias) {
+        if ((st = set_smem(pba::pba_pwa_dw_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
+        cudaFuncSetAttribute(pba::pba_pwa_dw_kernel<CP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+        const long long g2 = (long long)pl.splits * d->H * pl.nT * pl.nT;
+        {
+            ProfScope ps(K_PWA_DW, s);
+            pba::pba_pwa_dw_kernel<CP><<<(unsigned)g2, 192, DT::SMEM_BYTES, s>>>(tdo, tv, a);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pwa_dw_kernel launch");
+        {
+            ProfScope ps(K_PWA_DBIAS, s);
+            pba::pba_pwa_dbias_kernel<<<grid_for((long long)d->H * pl.N * 32, 256), 256, 0, s>>>(a);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pwa_dbias_kernel launch");
+    }
+    return PBA_OK;
+}
+
+pba_status check_pwa_common(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
+                            const pba_dims *d) {
+    pba_status st;
+    if ((st = check_strides(d->sv, d->B, d->Nk, d->H, "v")) != PBA_OK) return st;
+    if ((st = check_strides(d->so, d->B, d->Nq, d->H, "out")) != PBA_OK) return st;
+    if (!v) return fail(PBA_ERR_INVALID_ARG, "v is required");
+    if (!aligned16(v)) return fail(PBA_ERR_INVALID_ARG, "v must be 16-byte aligned");
+    if (gate) {
+        if (!aligned16(gate)) return fail(PBA_ERR_INVALID_ARG, "gate must be 16-byte aligned");
+        if ((st = check_strides(d->sg, d->B, d->Nq, d->H, "gate")) != PBA_OK) return st;
+    }
+    if (bias && d->H > 1 && d->sbias[0] <= 0) return fail(PBA_ERR_INVALID_ARG, "bias: H stride must be positive");
+    if (bias && d->Nq > 1 && d->sbias[1] <= 0) return fail(PBA_ERR_INVALID_ARG, "bias: row stride must be positive");
+    (void)mask;
+    return get_encoder();
+}
+
 }  // namespace
 
 extern "C" {
@@ -622,7 +833,7 @@ pba_status pba_device_status(void *stream) {
         cudaMemcpyFromSymbol(&site, pba::g_pba_watchdog_site, sizeof(site));
         cudaMemcpyToSymbol(pba::g_pba_watchdog, &zero, sizeof(zero));
         cudaMemcpyToSymbol(pba::g_pba_watchdog_site, &zero, sizeof(zero));
-        if ((site & 0xFFFu) == pba::SITE_FWD_ALIGN)
+        if ((site & 0xFFFu) == pba::SITE_FWD_ALIGN || (site & 0xFFFu) == pba::SITE_PWA_ALIGN)
             return fail(PBA_ERR_UNSUPPORTED, "forward kernel refused: dynamic shared memory "
                                              "is not 1024-byte aligned");
         return fail(PBA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (site 0x%x)", site);
@@ -672,6 +883,67 @@ int pba_profile_read(pba_kernel_stat *out, int max) {
         ++n;
     }
     return n < max ? n : max;
+}
+
+size_t pba_pwa_fwd_workspace_size(const pba_dims *d) {
+    if (!d || check_pwa_dims(d) != PBA_OK) return 0;
+    return plan_pwa(d).fwd_total;
+}
+
+size_t pba_pwa_bwd_workspace_size(const pba_dims *d) {
+    if (!d || check_pwa_dims(d) != PBA_OK) return 0;
+    return plan_pwa(d).bwd_total;
+}
+
+pba_status pba_pwa_fwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                       pba_bf16 *out, float *lse_w, void *workspace, size_t workspace_bytes,
+                       const pba_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_pwa_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->B == 0 || d->Nq == 0 || d->H == 0) return PBA_OK;
+    if (!out || !lse_w) return fail(PBA_ERR_INVALID_ARG, "out and lse_w are required");
+    if (!aligned16(out)) return fail(PBA_ERR_INVALID_ARG, "out must be 16-byte aligned");
+    if ((st = check_pwa_common(v, bias, key_mask, gate, d)) != PBA_OK) return st;
+    const PwaPlan pl = plan_pwa(d);
+    if (!workspace || workspace_bytes < pl.fwd_total)
+        return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.fwd_total, workspace_bytes);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(PBA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    switch (padded_c(d->C)) {
+        case 16: return launch_pwa_fwd<16>(v, bias, key_mask, gate, out, lse_w, ws, pl, d, s);
+        case 32: return launch_pwa_fwd<32>(v, bias, key_mask, gate, out, lse_w, ws, pl, d, s);
+        default: return launch_pwa_fwd<64>(v, bias, key_mask, gate, out, lse_w, ws, pl, d, s);
+    }
+}
+
+pba_status pba_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                       const pba_bf16 *out, const pba_bf16 *dout, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                       void *workspace, size_t workspace_bytes, const pba_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_pwa_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->B == 0 || d->Nq == 0 || d->H == 0) return PBA_OK;
+    if (!dout || !dv) return fail(PBA_ERR_INVALID_ARG, "dout and dv are required");
+    if (gate && (!out || !dgate)) return fail(PBA_ERR_INVALID_ARG, "out and dgate are required with a gate");
+    const void *al[] = {dout, dv, out, dgate};
+    for (const void *p : al)
+        if (p && !aligned16(p)) return fail(PBA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    if ((st = check_pwa_common(v, bias, key_mask, gate, d)) != PBA_OK) return st;
+    const PwaPlan pl = plan_pwa(d);
+    if (!workspace || workspace_bytes < pl.bwd_total)
+        return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.bwd_total, workspace_bytes);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(PBA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    switch (padded_c(d->C)) {
+        case 16: return launch_pwa_bwd<16>(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, pl, d, s);
+        case 32: return launch_pwa_bwd<32>(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, pl, d, s);
+        default: return launch_pwa_bwd<64>(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, pl, d, s);
+    }
 }
 
 const char *pba_status_string(pba_status s) {
