@@ -17,6 +17,7 @@ on the host cores instead.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -79,7 +80,13 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = {"pba_fwd_kernel": "pba_fwd.cuh"}   # every other kernel lives in pba_bwd.cuh
+KERNEL_SOURCES = {"pba_fwd_kernel": "pba_fwd.cuh"}   # every other attention kernel: pba_bwd.cuh
+
+
+def kernel_source_file(kernel: str) -> str:
+    if kernel.startswith("pba_pwa_"):
+        return "pba_pwa.cuh"
+    return KERNEL_SOURCES.get(kernel, "pba_bwd.cuh")
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -87,7 +94,7 @@ def kernel_source_hash(kernel: str) -> str:
     header (launch configuration in the API file is not covered)."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc")
-    for name in (KERNEL_SOURCES.get(kernel, "pba_bwd.cuh"), "pba_device.cuh"):
+    for name in (kernel_source_file(kernel), "pba_device.cuh"):
         with open(os.path.join(cdir, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -453,6 +460,185 @@ def run_reference(args, cfg):
                 "d2h_bytes_per_step": 0},
     }
 
+# ---------------------------------------------------------------------------------------
+# MSA pair-weighted averaging (--op pwa): the same contract on the second operator
+# ---------------------------------------------------------------------------------------
+PWA_METRIC = "MSA pair-weighted averaging fwd+bwd TFLOP/s and %roofline on 1 B200"
+
+
+def pwa_work(cfg, B=None):
+    """Algorithmic work of pair-weighted averaging (Nv = attended keys): fwd 2 B H N Nv c
+    (W V), bwd 4 B H N Nv c (W^T dOa and dOa V^T); bytes as each pass must move."""
+    B = cfg.B if B is None else B
+    H, N, c, Nv = cfg.H, cfg.N, cfg.c, cfg.n_valid_keys
+    e = B * N * H * c
+    unit = B * H * N * Nv * c
+    bias_b, nn4 = H * N * N * 2, H * N * N * 4
+    f = {"fwd_flops": 2 * unit, "bwd_flops": 4 * unit,
+         "fwd_bytes": 3 * e * 2 + bias_b + H * N * 4 + N,
+         "bwd_bytes": 6 * e * 2 + bias_b + nn4 + N}
+    f["kernels"] = {
+        "pba_pwa_weights_kernel": (0, 2 * bias_b + H * N * 4),
+        "pba_pwa_gemm_kernel (out)": (2 * unit, 3 * e * 2 + bias_b),
+        "pba_pwa_pre_kernel": (0, 5 * e * 2),
+        "pba_pwa_gemm_kernel (dv)": (2 * unit, 2 * e * 2 + bias_b),
+        "pba_pwa_dw_kernel": (2 * unit, 2 * e * 2),
+        "pba_pwa_dbias_kernel": (0, bias_b + nn4),
+    }
+    return f
+
+
+def time_pwa_oracle(cfg, target_s, seed):
+    import oracle
+    B1 = max(1, min(cfg.B, 2))
+    d = pi.make_inputs(cfg, seed=seed, B=B1)
+    f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+    t0 = time.perf_counter()
+    oracle.pwa_fwd(f["v"], f["bias"], f["keep"], f.get("g"))
+    oracle.pwa_bwd(f["v"], f["bias"], f["keep"], f.get("g"), f["dout"])
+    per_row = (time.perf_counter() - t0) / B1
+    rows = int(max(1, min(cfg.B, target_s / max(per_row, 1e-6))))
+    d = pi.make_inputs(cfg, seed=seed, B=rows)
+    f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+    t0 = time.perf_counter()
+    oracle.pwa_fwd(f["v"], f["bias"], f["keep"], f.get("g"))
+    oracle.pwa_bwd(f["v"], f["bias"], f["keep"], f.get("g"), f["dout"])
+    el = time.perf_counter() - t0
+    w = pwa_work(cfg, B=rows)
+    threads = oracle.threads()
+    return {"value": (w["fwd_flops"] + w["bwd_flops"]) / el / 1e12, "unit": "TFLOP/s",
+            "cores": min(threads, cfg.H), "kind": "oracle",
+            "sample": "%s pair-weighted averaging fwd+bwd on %d of %d broadcast rows, %.1f s; fp64 C "
+                      "loops, OpenMP over the %d heads (%d threads available)"
+                      % (cfg.name, rows, cfg.B, el, cfg.H, threads),
+            "seconds": el, "rows": rows}
+
+
+def run_pwa(args, cfg):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    import numpy as np
+    import pair_biased_attention_gated_b200 as pba
+    d = pi.make_inputs(cfg, seed=args.seed)
+    host = {}
+    for k in ("v", "bias", "keep", "g", "dout"):
+        if k not in d:
+            continue
+        a = d[k]
+        t = torch.from_numpy(np.ascontiguousarray(a)) if k == "keep" else \
+            torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        host[k] = t.pin_memory()
+    dev = {k: v.cuda() for k, v in host.items()}
+    v, bias, keep, g, dout = dev["v"], dev["bias"], dev["keep"], dev.get("g"), dev["dout"]
+    B, N, H, C = v.shape
+    out = torch.empty_like(v)
+    lse = torch.empty(H, N, dtype=torch.float32, device="cuda")
+    dv = torch.empty_like(v)
+    dg = torch.empty_like(g) if g is not None else None
+    db = torch.empty(H, N, N, dtype=torch.float32, device="cuda")
+    dims = pba.pwa_dims(v, g, out, bias, keep)
+    wsf = torch.empty(int(pba.lib.pba_pwa_fwd_workspace_size(ctypes.byref(dims))), dtype=torch.uint8, device="cuda")
+    wsb = torch.empty(int(pba.lib.pba_pwa_bwd_workspace_size(ctypes.byref(dims))), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pba.pba_pwa_fwd(v, bias, keep, g, out, lse, wsf)
+        pba.pba_pwa_bwd(v, bias, keep, g, out, dout, dv, db, dg, wsb)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    pba.pba_device_status()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    torch.cuda.synchronize()
+    pba.profile_read()
+    pba.profile_enable(True)
+    sampler.start()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    pba.profile_enable(False)
+    kstats = pba.profile_read()
+    pba.pba_device_status()
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in ev)
+    # end to end: host buffers, copies inside the events
+    houts = {"out": out, "lse": lse, "dv": dv, "db": db}
+    if dg is not None:
+        houts["dg"] = dg
+    hbufs = {k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in houts.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in hbufs.values())
+    K2 = max(1, min(K, 20))
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
+    torch.cuda.synchronize()
+    for i in range(K2):
+        flush.fill_(i & 0xFF)
+        ev2[i][0].record(stream)
+        for k2, t in host.items():
+            dev[k2].copy_(t, non_blocking=True)
+        step()
+        for k2, t in hbufs.items():
+            t.copy_(houts[k2], non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    pba.pba_device_status()
+
+    w = pwa_work(cfg)
+    step_flops = w["fwd_flops"] + w["bwd_flops"]
+    value = step_flops * K / (elapsed_ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tens = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    total_k = sum(ms for _, ms in kstats.values()) or 1.0
+    dom = max(kstats.items(), key=lambda kv: kv[1][1])[0] if kstats else None
+    roof = None
+    if dom:
+        launches, ms = kstats[dom]
+        avg_s = ms / launches / 1e3
+        kf, kb = w["kernels"].get(dom, (0, 0))
+        if kf / (tens * 1e12) > kb / (hbm * 1e9):
+            achieved, peak, unit, bound = kf / avg_s / 1e12, tens, "TFLOP/s", "tensor"
+        else:
+            achieved, peak, unit, bound = kb / avg_s / 1e9, hbm, "GB/s", "hbm"
+        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                "frac": round(achieved / peak, 4),
+                "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
+                "algorithmic_per_launch": {"flops": kf, "bytes": kb}, "avg_launch_us": round(avg_s * 1e6, 2),
+                "traffic": ncu_traffic(dom, "pwa-" + cfg.name)}
+    ms_per_step = elapsed_ms / K
+    t_step_roof = max(step_flops / (tens * 1e12), (w["fwd_bytes"] + w["bwd_bytes"]) / (hbm * 1e9))
+    kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
+               for n, (l, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1])}
+    res = {
+        "metric": PWA_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 v/gate/dout, N(0,%g^2) bias, shapes of the named workload"
+                % cfg.bias_std,
+        "config": {"workload": "%s: %s (pair-weighted averaging of its value rows)" % (cfg.name, cfg.desc),
+                   "B": cfg.B, "H": cfg.H, "N": cfg.N, "c": cfg.c, "masked_keys": cfg.N - cfg.n_valid_keys,
+                   "gate": cfg.gate, "passes": "fwd+bwd (dv, dgate, dbias)",
+                   "l2": "flushed before every timed step (256 MiB write outside the events)",
+                   "parallelism": "single GPU"},
+        "roofline": roof,
+        "step_roofline": {"time_us": round(t_step_roof * 1e6, 2), "frac": round(t_step_roof * 1e3 / ms_per_step, 4)},
+        "kernels": kernels, "gpu_launches": sum(l for l, _ in kstats.values()), "clocks": clocks,
+        "e2e": {"value": round(step_flops * K2 / (e2e_ms / 1e3) / 1e12, 4), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = time_pwa_oracle(cfg, target_s=args.cpu_seconds, seed=args.seed)
+    return res if rank == 0 else None
+
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -465,11 +651,18 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="attention", choices=["attention", "pwa"],
+                    help="pwa: MSA pair-weighted averaging of the workload's value rows (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = pi.CONFIGS[args.config]
-    res = run_reference(args, cfg) if args.impl == "reference" else run_ours(args, cfg)
+    if args.op == "pwa":
+        if args.impl == "reference" or args.gpus != 1:
+            ap.error("--op pwa times our kernels on one GPU; its oracle baseline is the cpu_baseline key")
+        res = run_pwa(args, cfg)
+    else:
+        res = run_reference(args, cfg) if args.impl == "reference" else run_ours(args, cfg)
     if res is not None:
         print(json.dumps(res), flush=True)
 
