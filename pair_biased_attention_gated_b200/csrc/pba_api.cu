@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -221,6 +223,8 @@ pba_status set_smem(K kernel, int bytes) {
     return PBA_OK;
 }
 
+long long num_sms();
+
 template <int CP>
 pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                       const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
@@ -259,7 +263,11 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                                           cudaFuncAttributePreferredSharedMemoryCarveout,
                                           cudaSharedmemCarveoutMaxShared);
     if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute (carveout)");
-    const long long grid = tiles * a.nChunks;
+    const long long items = tiles * a.nChunks;
+    if (items > INT_MAX) return fail(PBA_ERR_UNSUPPORTED, "too many forward work items");
+    a.items = (int)items;
+    // persistent: at most two CTAs per SM (their shared memory allows no more)
+    const long long grid = std::min<long long>(items, 2LL * num_sms());
     {
         ProfScope ps(K_FWD, stream);
         pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);

@@ -5,12 +5,16 @@
 // Model Efficiency section: the pair bias is added after the key-query dot product and
 // is shared by every broadcast row b (triangle rows, MSA sequences, diffusion copies).
 //
-// One CTA owns one (head h, 128-query tile, chunk of BC broadcast rows); two CTAs share an
-// SM, so one CTA's prologue and epilogue overlap the other's main loop.  The loop runs over
+// Work item = (head h, 128-query tile, chunk of BC broadcast rows).  The kernel is
+// persistent: two CTAs per SM, each walking the items blockIdx.x, blockIdx.x + gridDim.x,
+// ... with one pipeline that runs across item boundaries (every ring and barrier counts
+// steps and tiles of the CTA, not of the item), so the next item's loads and Q K^T
+// overlap the current item's last steps and epilogue.  Within an item the loop runs over
 // key tiles j (outer) and the chunk's rows b (inner): each 128x128 bias tile is moved into
-// shared memory once and reused by all rows of the chunk.  The chunk's Q tiles stay
-// resident; K and V tiles stream through two rings: a K stage is refilled as soon as its
-// Q K^T is done, a V stage only after its P V.
+// shared memory once and reused by all rows of the chunk.  The chunk's Q tiles are
+// reloaded per item once the previous item's last Q K^T is done; K and V tiles stream
+// through two rings: a K stage is refilled as soon as its Q K^T is done, a V stage only
+// after its P V.
 //
 // Warp roles (256 threads, two warpgroups):
 //   warps 0-3  softmax and epilogue: thread = query row = TMEM lane
@@ -26,7 +30,9 @@
 // Tensor memory (256 columns): S [0,128), P as packed bf16 [128,192), then one
 // CP-column fp32 O accumulator per row of the chunk [192,256).  S and P are separate, so
 // the next Q K^T runs while the softmax turns the current S into P: step k's softmax
-// frees S right after reading it, and P only has to wait for the previous P V.
+// frees S right after reading it, and P only has to wait for the previous P V.  The O
+// slots start over with the first P V of the next item, which waits for the P of that
+// step, written only after the softmax warps have read this item's O out.
 #pragma once
 
 #include "pba_device.cuh"
@@ -36,6 +42,7 @@ namespace pba {
 struct FwdArgs {
     int B, H, Nq, Nk, C;
     int nI, nJ, nChunks;
+    int items;       // H * nI * nChunks work items, walked by a grid of at most 2 CTAs per SM
     float scale;
     int has_bias;
     int mask_shared;  // the key mask (if any) is one row shared by every b
@@ -61,7 +68,7 @@ struct FwdTraits {
     static constexpr int OFF_K = OFF_Q + BC * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KVS * TILE_BYTES;
     static constexpr int OFF_MASK = OFF_V + KVS * TILE_BYTES;  // u32 [KVS][8] per-row words (V ring)
-    static constexpr int NBAR = 1 + 4 * KVS + 3 * BS + 6;
+    static constexpr int NBAR = 2 + 4 * KVS + 3 * BS + 6;
     static constexpr int OFF_BAR = OFF_MASK + KVS * 32;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // TMEM base, abort flag
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -116,12 +123,13 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
-    const uint32_t b_q = smem_u32(&bars[0]);
-    auto b_k_full = [&](int st) { return smem_u32(&bars[1 + st]); };
-    auto b_k_empty = [&](int st) { return smem_u32(&bars[1 + KVS + st]); };
-    auto b_v_full = [&](int st) { return smem_u32(&bars[1 + 2 * KVS + st]); };
-    auto b_v_empty = [&](int st) { return smem_u32(&bars[1 + 3 * KVS + st]); };
-    constexpr int OBB = 1 + 4 * KVS;
+    const uint32_t b_q_full = smem_u32(&bars[0]);    // the item's Q tiles landed
+    const uint32_t b_q_empty = smem_u32(&bars[1]);   // the item's last Q K^T done
+    auto b_k_full = [&](int st) { return smem_u32(&bars[2 + st]); };
+    auto b_k_empty = [&](int st) { return smem_u32(&bars[2 + KVS + st]); };
+    auto b_v_full = [&](int st) { return smem_u32(&bars[2 + 2 * KVS + st]); };
+    auto b_v_empty = [&](int st) { return smem_u32(&bars[2 + 3 * KVS + st]); };
+    constexpr int OBB = 2 + 4 * KVS;
     auto b_bias_full = [&](int x) { return smem_u32(&bars[OBB + x]); };            // landed
     auto b_bias_ready = [&](int x) { return smem_u32(&bars[OBB + BS + x]); };      // folded
     auto b_bias_empty = [&](int x) { return smem_u32(&bars[OBB + 2 * BS + x]); };
@@ -130,25 +138,37 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t b_s_free = smem_u32(&bars[OB + 1]);   // S read out
     const uint32_t b_p_full = smem_u32(&bars[OB + 2]);   // P in TMEM, O rescaled
     const uint32_t b_p_free = smem_u32(&bars[OB + 3]);   // P V done
-    const uint32_t b_ofinal = smem_u32(&bars[OB + 4]);   // every P V done
+    const uint32_t b_ofinal = smem_u32(&bars[OB + 4]);   // every P V of the item done
     const uint32_t b_drain = smem_u32(&bars[OB + 5]);    // abort path
     uint32_t *s_tmem_base = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC + 4);
 
     const int warp = warp_id(), lane = lane_id();
-    int idx = blockIdx.x;
-    const int itile = idx % a.nI;
-    idx /= a.nI;
-    const int chunk = idx % a.nChunks;
-    const int h = idx / a.nChunks;
-    const int i0 = itile * 128, b0 = chunk * BC;
-    const int nb = min(BC, a.B - b0);
     const int nJ = a.nJ;
-    const int K = nJ * nb;   // steps (j, s), k = j * nb + s
     const bool row_mask = a.mask != nullptr && !a.mask_shared;
+    // item n of this CTA is blockIdx.x + n gridDim.x: query tile fastest, then the chunk of
+    // rows, then the head (CTAs running at the same time share K/V and bias tiles in L2)
+    struct FItem {
+        int h, i0, b0, nb;
+    };
+    auto item = [&](int n) {
+        int idx = blockIdx.x + n * gridDim.x;
+        const int itile = idx % a.nI;
+        idx /= a.nI;
+        const int chunk = idx % a.nChunks;
+        FItem it;
+        it.h = idx / a.nChunks;
+        it.i0 = itile * 128;
+        it.b0 = chunk * BC;
+        it.nb = min(BC, a.B - it.b0);
+        return it;
+    };
+    const int n_items = (int)blockIdx.x < a.items ? (a.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // steps of an item: (j, s), local index j * nb + s; k below is the CTA's step count
 
     if (threadIdx.x == 0) {
-        mbar_init(b_q, 1);
+        mbar_init(b_q_full, 1);
+        mbar_init(b_q_empty, 1);
         for (int st = 0; st < KVS; ++st) {
             mbar_init(b_k_full(st), 1);
             mbar_init(b_k_empty(st), 1);
@@ -179,8 +199,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tbase = *s_tmem_base;
 
     // K loads issued for steps [0, k_done), V loads for [0, v_done), bias tiles
-    // [0, n_bias): what has to land before the CTA may exit after an abort
-    int k_done = 0, v_done = 0, n_bias = 0;
+    // [0, n_bias), Q for items [0, q_done): what has to land before the CTA may exit after
+    // an abort
+    int k_done = 0, v_done = 0, n_bias = 0, q_done = 0;
 
     if (warp >= 4) reg_dealloc<T::REGS_OTHER>();   // the whole second warpgroup, same point
     if (warp == 4) {
@@ -190,36 +211,47 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             if (a.has_bias) tma_prefetch_desc(&tmBias);
-            mbar_arrive_tx(b_q, nb * T::TILE_BYTES);
-            for (int s = 0; s < nb; ++s)
-                tma_load_4d(sbase + T::OFF_Q + s * T::TILE_BYTES, &tmQ, b_q, 0, h, i0, b0 + s);
         }
-        // Load order: B(0), K(0), then for every step k: K(k + 1), V(k), and the bias tile
-        // of the next key tile once step k + 1 starts one.  K runs a step ahead of V; a bias
-        // tile (which waits for the softmax to leave the buffer's previous tile) comes after
-        // the V loads whose mask words that softmax may be waiting for.
-        auto load_bias = [&](int j) -> bool {
-            const int bs = j % BS;
+        // Load order of an item: B(0), K(0), the item's Q tiles (once the previous item's
+        // last Q K^T is done), then for every step k: K(k + 1), V(k), and the bias tile of
+        // the next key tile once step k + 1 starts one.  K runs a step ahead of V; a bias
+        // tile (which waits for the softmax to leave the buffer's previous tile) comes
+        // after the V loads whose mask words that softmax may be waiting for.
+        auto load_bias = [&](int jg, int j, const FItem &it) -> bool {
+            const int bs = jg % BS;
             bool ok = true;
-            if (j >= BS)
-                ok = mbar_wait(b_bias_empty(bs), ((j / BS) - 1) & 1, abort_flag,
-                               SITE_FWD_PROD | 0x20 | (j << 12));
+            if (jg >= BS)
+                ok = mbar_wait(b_bias_empty(bs), ((jg / BS) - 1) & 1, abort_flag,
+                               SITE_FWD_PROD | 0x20 | (jg << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return false;
             if (lane == 0) {
                 if (a.has_bias) {
                     const uint32_t dst = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
                     mbar_arrive_tx(b_bias_full(bs), T::BIAS_BYTES);
-                    tma_load_3d(dst, &tmBias, b_bias_full(bs), j * 128, i0, h);
-                    tma_load_3d(dst + 16384, &tmBias, b_bias_full(bs), j * 128 + 64, i0, h);
+                    tma_load_3d(dst, &tmBias, b_bias_full(bs), j * 128, it.i0, it.h);
+                    tma_load_3d(dst + 16384, &tmBias, b_bias_full(bs), j * 128 + 64, it.i0, it.h);
                 } else {
                     mbar_arrive(b_bias_full(bs));   // buffer free: the fold warps build it
                 }
             }
-            n_bias = j + 1;
+            n_bias = jg + 1;
             return true;
         };
-        auto load_k = [&](int k) -> bool {
+        auto load_q = [&](int n, const FItem &it) -> bool {
+            bool ok = true;
+            if (n >= 1) ok = mbar_wait(b_q_empty, (n - 1) & 1, abort_flag, SITE_FWD_PROD | 0x30 | (n << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return false;
+            if (lane == 0) {
+                mbar_arrive_tx(b_q_full, it.nb * T::TILE_BYTES);
+                for (int s = 0; s < it.nb; ++s)
+                    tma_load_4d(sbase + T::OFF_Q + s * T::TILE_BYTES, &tmQ, b_q_full, 0, it.h, it.i0, it.b0 + s);
+            }
+            q_done = n + 1;
+            return true;
+        };
+        auto load_k = [&](int k, int kl, const FItem &it) -> bool {
             const int st = k % KVS, use = k / KVS;
             bool ok = true;
             if (use >= 1)
@@ -228,20 +260,20 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (!ok) return false;
             if (lane == 0 && k != a.skip_step) {
                 mbar_arrive_tx(b_k_full(st), T::TILE_BYTES);
-                tma_load_4d(sbase + T::OFF_K + st * T::TILE_BYTES, &tmK, b_k_full(st), 0, h,
-                            (k / nb) * 128, b0 + k % nb);
+                tma_load_4d(sbase + T::OFF_K + st * T::TILE_BYTES, &tmK, b_k_full(st), 0, it.h,
+                            (kl / it.nb) * 128, it.b0 + kl % it.nb);
             }
             k_done = k + 1;
             return true;
         };
-        auto load_v = [&](int k) -> bool {
+        auto load_v = [&](int k, int kl, const FItem &it) -> bool {
             const int st = k % KVS, use = k / KVS;
             bool ok = true;
             if (use >= 1)
                 ok = mbar_wait(b_v_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | 0x10 | (k << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return false;
-            const int j = k / nb, b = b0 + k % nb;
+            const int j = kl / it.nb, b = it.b0 + kl % it.nb;
             if (row_mask) {
                 // words of row b: word q bit t <-> key 128 j + 32 q + t attended
                 uint32_t w[4];
@@ -262,38 +294,54 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             }
             if (lane == 0) {
                 mbar_arrive_tx(b_v_full(st), T::TILE_BYTES);
-                tma_load_4d(sbase + T::OFF_V + st * T::TILE_BYTES, &tmV, b_v_full(st), 0, h, j * 128, b);
+                tma_load_4d(sbase + T::OFF_V + st * T::TILE_BYTES, &tmV, b_v_full(st), 0, it.h, j * 128, b);
             }
             v_done = k + 1;
             return true;
         };
-        bool ok = K > 0 ? (load_bias(0) && load_k(0)) : true;
-        for (int k = 0; k < K && ok; ++k) {
-            if (k + 1 < K) ok = load_k(k + 1);
-            if (ok) ok = load_v(k);
-            if (ok && k + 1 < K && (k + 1) % nb == 0) ok = load_bias((k + 1) / nb);
+        bool ok = true;
+        int kg = 0, jg = 0;   // the CTA's steps and bias tiles before this item
+        for (int n = 0; n < n_items && ok; ++n) {
+            const FItem it = item(n);
+            const int Kn = nJ * it.nb;
+            ok = load_bias(jg, 0, it) && load_k(kg, 0, it) && load_q(n, it);
+            for (int kl = 0; kl < Kn && ok; ++kl) {
+                if (kl + 1 < Kn) ok = load_k(kg + kl + 1, kl + 1, it);
+                if (ok) ok = load_v(kg + kl, kl, it);
+                if (ok && kl + 1 < Kn && (kl + 1) % it.nb == 0)
+                    ok = load_bias(jg + (kl + 1) / it.nb, (kl + 1) / it.nb, it);
+            }
+            kg += Kn;
+            jg += nJ;
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------------ Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             constexpr uint32_t SBO = 8 * T::ROWB;
-            bool ok = mbar_wait(b_q, 0, abort_flag, SITE_FWD_MMA);
-            // step k: S must have been read out by the softmax of step k - 1
-            for (int k = 0; k < K && ok; ++k) {
-                const int s = k % nb, st = k % KVS;
-                if (k > 0) ok = mbar_wait(b_s_free, (k - 1) & 1, abort_flag, SITE_FWD_MMA | 0x20 | (k << 12));
-                if (ok) ok = mbar_wait(b_k_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x10 | (k << 12));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t qa = sbase + T::OFF_Q + s * T::TILE_BYTES;
-                const uint32_t ka = sbase + T::OFF_K + st * T::TILE_BYTES;
+            bool ok = true;
+            int kg = 0;
+            for (int n = 0; n < n_items && ok; ++n) {
+                const int nb = item(n).nb, Kn = nJ * nb;
+                ok = mbar_wait(b_q_full, n & 1, abort_flag, SITE_FWD_MMA | 0x50 | (n << 12));
+                // step k: S must have been read out by the softmax of step k - 1
+                for (int kl = 0; kl < Kn && ok; ++kl) {
+                    const int k = kg + kl, s = kl % nb, st = k % KVS;
+                    if (k > 0) ok = mbar_wait(b_s_free, (k - 1) & 1, abort_flag, SITE_FWD_MMA | 0x20 | (k << 12));
+                    if (ok) ok = mbar_wait(b_k_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x10 | (k << 12));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t qa = sbase + T::OFF_Q + s * T::TILE_BYTES;
+                    const uint32_t ka = sbase + T::OFF_K + st * T::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < CP / 16; ++kk)
-                    umma_ss(tbase + T::T_S, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
-                umma_commit(b_s_full);
-                umma_commit(b_k_empty(st));
+                    for (int kk = 0; kk < CP / 16; ++kk)
+                        umma_ss(tbase + T::T_S, sdesc(qa + kk * 32, 16, SBO, T::SWZ),
+                                sdesc(ka + kk * 32, 16, SBO, T::SWZ), idesc_qk, kk > 0 ? 1u : 0u);
+                    umma_commit(b_s_full);
+                    umma_commit(b_k_empty(st));
+                    if (kl == Kn - 1) umma_commit(b_q_empty);   // the next item's Q may load
+                }
+                kg += Kn;
             }
         }
     } else if (warp == 6) {
@@ -302,31 +350,37 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             constexpr uint32_t idesc_pv = idesc_bf16(128, CP, false, true);
             constexpr uint32_t SBO = 8 * T::ROWB;
             bool ok = true;
-            // step k: P of step k written (and O[s] rescaled) by the softmax, V landed
-            for (int k = 0; k < K && ok; ++k) {
-                const int j = k / nb, s = k % nb, st = k % KVS;
-                ok = mbar_wait(b_p_full, k & 1, abort_flag, SITE_FWD_MMA | 0x30 | (k << 12));
-                if (ok) ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x40 | (k << 12));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t va = sbase + T::OFF_V + st * T::TILE_BYTES;
-                const uint32_t d = tbase + T::T_O + s * CP;
+            int kg = 0;
+            for (int n = 0; n < n_items && ok; ++n) {
+                const int nb = item(n).nb, Kn = nJ * nb;
+                // step k: P of step k written (and O[s] rescaled) by the softmax, V landed
+                for (int kl = 0; kl < Kn && ok; ++kl) {
+                    const int k = kg + kl, j = kl / nb, s = kl % nb, st = k % KVS;
+                    ok = mbar_wait(b_p_full, k & 1, abort_flag, SITE_FWD_MMA | 0x30 | (k << 12));
+                    if (ok) ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x40 | (k << 12));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t va = sbase + T::OFF_V + st * T::TILE_BYTES;
+                    const uint32_t d = tbase + T::T_O + s * CP;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(d, tbase + T::T_P + kk * 8,
-                            sdesc(va + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), idesc_pv,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(b_p_free);
-                umma_commit(b_v_empty(st));
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(d, tbase + T::T_P + kk * 8,
+                                sdesc(va + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), idesc_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(b_p_free);
+                    umma_commit(b_v_empty(st));
+                }
+                if (ok) umma_commit(b_ofinal);
+                kg += Kn;
             }
-            if (ok) umma_commit(b_ofinal);
         }
     } else if (warp == 7) {
         // ------------------------------------------------------------------ mask fold
         const int t = lane;   // rows t, t + 32, t + 64, t + 96 of every bias tile
         bool ok = true;
-        for (int j = 0; j < nJ && ok; ++j) {
-            const int bs = j % BS;
+        const int n_tiles = n_items * nJ;   // the CTA's bias tiles; tile jg has key tile jg % nJ
+        for (int jg = 0; jg < n_tiles && ok; ++jg) {
+            const int bs = jg % BS, j = jg % nJ;
             // word q bit l <-> key 128 j + 32 q + l attended by every row of the chunk
             uint32_t w[4];
 #pragma unroll
@@ -336,7 +390,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (valid && a.mask && !row_mask) valid = a.mask[key] != 0;
                 w[q] = __ballot_sync(0xffffffffu, valid);
             }
-            ok = mbar_wait(b_bias_full(bs), (j / BS) & 1, abort_flag, SITE_FWD_FOLD | (j << 12));
+            ok = mbar_wait(b_bias_full(bs), (jg / BS) & 1, abort_flag, SITE_FWD_FOLD | (jg << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             uint8_t *tile = dsmem + T::OFF_BIAS + bs * T::BIAS_BYTES;
@@ -387,192 +441,196 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t tP = tbase + T::T_P + lane_off;
         const float2 sc2 = make_float2(a.scale, a.scale);
         const float2 l2e2 = make_float2(kLog2e, kLog2e);
-        float m_run[BC], l_run[BC];   // running (max, sum) of this row in every slot
-#pragma unroll
-        for (int t = 0; t < BC; ++t) {
-            m_run[t] = -INFINITY;
-            l_run[t] = 0.f;
-        }
         bool ok = true;
-        int k = 0;
-        for (int j = 0; j < nJ && ok; ++j) {
-            const int bs = j % BS;
-            for (int s = 0; s < nb; ++s, ++k) {
-                const int st = k % KVS;
-                ok = mbar_wait(b_s_full, k & 1, abort_flag, SITE_FWD_SOFTMAX | (k << 12));
-                if (ok && s == 0)
-                    ok = mbar_wait(b_bias_ready(bs), (j / BS) & 1, abort_flag,
-                                   SITE_FWD_SOFTMAX | 0x10 | (k << 12));
-                if (ok && row_mask)   // this step's mask words come with its V tile
-                    ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag,
-                                   SITE_FWD_SOFTMAX | 0x20 | (k << 12));
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                tc_fence_after();
-
-                // S of this row, then hand the S columns back for the next Q K^T
-                uint32_t xr[128];
-                tmem_ld128(tS, xr);
-                tc_fence_before();
-                mbar_arrive(b_s_free);
-
-                // logits in place: x = scale * S + bias (natural-log units; -inf if masked)
-                {
-                    const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + row * 128;
+        int k = 0, jg = 0;   // the CTA's steps and bias tiles before this one
+        for (int n = 0; n < n_items && ok; ++n) {
+            const FItem it = item(n);
+            const int nb = it.nb;
+            float m_run[BC], l_run[BC];   // running (max, sum) of this row in every slot
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {  // 16-byte chunk q holds keys 8q .. 8q+7
-                        const uint4 bw = lds128(bias_row + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4));
-                        const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = q * 8 + 2 * e;
-                            const float2 v = ffma2(make_float2(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])),
-                                                   sc2, make_float2(bf16lo(bb[e]), bf16hi(bb[e])));
-                            xr[c] = __float_as_uint(v.x);
-                            xr[c + 1] = __float_as_uint(v.y);
-                        }
-                    }
-                }
-                if (s == nb - 1) mbar_arrive(b_bias_empty(bs));   // last reader of the tile
-                float *x = reinterpret_cast<float *>(xr);
-                if (row_mask) {
-                    const uint32_t *mw = reinterpret_cast<const uint32_t *>(dsmem + T::OFF_MASK) + st * 8;
-                    if (mw[4] == 0u) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t wd = mw[q];
-#pragma unroll
-                            for (int t = 0; t < 32; ++t)
-                                if (!((wd >> t) & 1u)) x[q * 32 + t] = -INFINITY;
-                        }
-                    }
-                }
-                // row maximum: four independent chains of three-input max
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < 128; c += 8) {
-                    m4[0] = max3(m4[0], x[c], x[c + 1]);
-                    m4[1] = max3(m4[1], x[c + 2], x[c + 3]);
-                    m4[2] = max3(m4[2], x[c + 4], x[c + 5]);
-                    m4[3] = max3(m4[3], x[c + 6], x[c + 7]);
-                }
-                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-
-                float m_use = m_run[0], l_prev = l_run[0];
-#pragma unroll
-                for (int t = 1; t < BC; ++t)
-                    if (s == t) {
-                        m_use = m_run[t];
-                        l_prev = l_run[t];
-                    }
-                float alpha = 1.f;
-                bool resc = false;
-                if (j == 0) {
-                    m_use = mx;
-                    l_prev = 0.f;
-                } else if (mx > m_use + kRescaleThresh) {
-                    alpha = (m_use == -INFINITY) ? 0.f : ex2((m_use - mx) * kLog2e);
-                    m_use = mx;
-                    resc = true;
-                }
-                const float nm = (m_use == -INFINITY) ? 0.f : -m_use * kLog2e;
-                const float2 nm2 = make_float2(nm, nm);
-
-                // P and O[s] may only be written once the previous P V is done
-                if (k > 0) {
-                    ok = mbar_wait(b_p_free, (k - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x30 | (k << 12));
+            for (int t = 0; t < BC; ++t) {
+                m_run[t] = -INFINITY;
+                l_run[t] = 0.f;
+            }
+            for (int j = 0; j < nJ && ok; ++j, ++jg) {
+                const int bs = jg % BS;
+                for (int s = 0; s < nb; ++s, ++k) {
+                    const int st = k % KVS;
+                    ok = mbar_wait(b_s_full, k & 1, abort_flag, SITE_FWD_SOFTMAX | (k << 12));
+                    if (ok && s == 0)
+                        ok = mbar_wait(b_bias_ready(bs), (jg / BS) & 1, abort_flag,
+                                       SITE_FWD_SOFTMAX | 0x10 | (k << 12));
+                    if (ok && row_mask)   // this step's mask words come with its V tile
+                        ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag,
+                                       SITE_FWD_SOFTMAX | 0x20 | (k << 12));
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
-                }
-                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+
+                    // S of this row, then hand the S columns back for the next Q K^T
+                    uint32_t xr[128];
+                    tmem_ld128(tS, xr);
+                    tc_fence_before();
+                    mbar_arrive(b_s_free);
+
+                    // logits in place: x = scale * S + bias (natural-log units; -inf if masked)
+                    {
+                        const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + row * 128;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t p[32];
+                        for (int q = 0; q < 16; ++q) {  // 16-byte chunk q holds keys 8q .. 8q+7
+                            const uint4 bw = lds128(bias_row + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4));
+                            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int i2 = hf * 64 + 2 * c;
-                        const float2 tt = ffma2(make_float2(x[i2], x[i2 + 1]), l2e2, nm2);
-                        const float2 pv = make_float2(ex2(tt.x), ex2(tt.y));
-                        if (c & 1) acc1 = fadd2(acc1, pv);
-                        else acc0 = fadd2(acc0, pv);
-                        p[c] = pack_bf16x2(pv.x, pv.y);
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = q * 8 + 2 * e;
+                                const float2 v = ffma2(make_float2(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])),
+                                                       sc2, make_float2(bf16lo(bb[e]), bf16hi(bb[e])));
+                                xr[c] = __float_as_uint(v.x);
+                                xr[c + 1] = __float_as_uint(v.y);
+                            }
+                        }
                     }
-                    tmem_st32(tP + hf * 32, p);
-                }
-                const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-                if (__any_sync(0xffffffffu, resc)) {
-                    const uint32_t tO = tbase + T::T_O + s * CP + lane_off;
-                    uint32_t o[CP];
-                    tmem_ld_cols<CP>(tO, o);
+                    if (s == nb - 1) mbar_arrive(b_bias_empty(bs));   // last reader of the tile
+                    float *x = reinterpret_cast<float *>(xr);
+                    if (row_mask) {
+                        const uint32_t *mw = reinterpret_cast<const uint32_t *>(dsmem + T::OFF_MASK) + st * 8;
+                        if (mw[4] == 0u) {
 #pragma unroll
-                    for (int c = 0; c < CP; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st_cols<CP>(tO, o);
-                }
-                tmem_wait_st();
-                const float l_new = l_prev * alpha + sum;
+                            for (int q = 0; q < 4; ++q) {
+                                const uint32_t wd = mw[q];
 #pragma unroll
-                for (int t = 0; t < BC; ++t)
-                    if (s == t) {
-                        m_run[t] = m_use;
-                        l_run[t] = l_new;
+                                for (int t = 0; t < 32; ++t)
+                                    if (!((wd >> t) & 1u)) x[q * 32 + t] = -INFINITY;
+                            }
+                        }
                     }
-                tc_fence_before();
-                mbar_arrive(b_p_full);
-            }
-        }
-        // ------------------------------------------------------------------ epilogue
-        // The gate does not depend on O: fetch it for all slots before waiting for the
-        // last P V products, so its latency overlaps theirs.
-        uint4 gw[BC][CP / 8];
-        const int i = i0 + row;
-        const bool row_ok = i < a.Nq;
+                    // row maximum: four independent chains of three-input max
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int t = 0; t < BC; ++t) {
+                    for (int c = 0; c < 128; c += 8) {
+                        m4[0] = max3(m4[0], x[c], x[c + 1]);
+                        m4[1] = max3(m4[1], x[c + 2], x[c + 3]);
+                        m4[2] = max3(m4[2], x[c + 4], x[c + 5]);
+                        m4[3] = max3(m4[3], x[c + 6], x[c + 7]);
+                    }
+                    const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+
+                    float m_use = m_run[0], l_prev = l_run[0];
 #pragma unroll
-            for (int c8 = 0; c8 < CP / 8; ++c8) {
-                gw[t][c8] = make_uint4(0, 0, 0, 0);
-                if (ok && a.gate && row_ok && t < nb && c8 * 8 < a.C)
-                    gw[t][c8] = *reinterpret_cast<const uint4 *>(
-                        a.gate + (b0 + t) * a.sg0 + (long long)i * a.sg1 + h * a.sg2 + c8 * 8);
+                    for (int t = 1; t < BC; ++t)
+                        if (s == t) {
+                            m_use = m_run[t];
+                            l_prev = l_run[t];
+                        }
+                    float alpha = 1.f;
+                    bool resc = false;
+                    if (j == 0) {
+                        m_use = mx;
+                        l_prev = 0.f;
+                    } else if (mx > m_use + kRescaleThresh) {
+                        alpha = (m_use == -INFINITY) ? 0.f : ex2((m_use - mx) * kLog2e);
+                        m_use = mx;
+                        resc = true;
+                    }
+                    const float nm = (m_use == -INFINITY) ? 0.f : -m_use * kLog2e;
+                    const float2 nm2 = make_float2(nm, nm);
+
+                    // P and O[s] may only be written once the previous P V is done
+                    if (k > 0) {
+                        ok = mbar_wait(b_p_free, (k - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x30 | (k << 12));
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t p[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int i2 = hf * 64 + 2 * c;
+                            const float2 tt = ffma2(make_float2(x[i2], x[i2 + 1]), l2e2, nm2);
+                            const float2 pv = make_float2(ex2(tt.x), ex2(tt.y));
+                            if (c & 1) acc1 = fadd2(acc1, pv);
+                            else acc0 = fadd2(acc0, pv);
+                            p[c] = pack_bf16x2(pv.x, pv.y);
+                        }
+                        tmem_st32(tP + hf * 32, p);
+                    }
+                    const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+                    if (__any_sync(0xffffffffu, resc)) {
+                        const uint32_t tO = tbase + T::T_O + s * CP + lane_off;
+                        uint32_t o[CP];
+                        tmem_ld_cols<CP>(tO, o);
+#pragma unroll
+                        for (int c = 0; c < CP; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st_cols<CP>(tO, o);
+                    }
+                    tmem_wait_st();
+                    const float l_new = l_prev * alpha + sum;
+#pragma unroll
+                    for (int t = 0; t < BC; ++t)
+                        if (s == t) {
+                            m_run[t] = m_use;
+                            l_run[t] = l_new;
+                        }
+                    tc_fence_before();
+                    mbar_arrive(b_p_full);
+                }
             }
-        }
-        if (ok) {
-            ok = mbar_wait(b_ofinal, 0, abort_flag, SITE_FWD_EPI);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        if (ok) {
-            tc_fence_after();
+            // ------------------------------------------------------------------ epilogue
+            // The gate does not depend on O: fetch it for all slots before waiting for the
+            // last P V products, so its latency overlaps theirs.
+            uint4 gw[BC][CP / 8];
+            const int i = it.i0 + row;
+            const bool row_ok = i < a.Nq;
 #pragma unroll
             for (int t = 0; t < BC; ++t) {
-                if (t >= nb) break;
-                uint32_t o[CP];
-                tmem_ld_cols<CP>(tbase + T::T_O + t * CP + lane_off, o);
-                if (!row_ok) continue;
-                const int b = b0 + t;
-                const bool live = l_run[t] > 0.f;
-                const float inv = live ? rcp_approx(l_run[t]) : 0.f;
-                __nv_bfloat16 *op = a.out + b * a.so0 + (long long)i * a.so1 + h * a.so2;
 #pragma unroll
                 for (int c8 = 0; c8 < CP / 8; ++c8) {
-                    if (c8 * 8 < a.C) {
-                        const uint32_t g4[4] = {gw[t][c8].x, gw[t][c8].y, gw[t][c8].z, gw[t][c8].w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float lo = __uint_as_float(o[c8 * 8 + 2 * e]) * inv;
-                            float hi = __uint_as_float(o[c8 * 8 + 2 * e + 1]) * inv;
-                            if (a.gate) {
-                                lo *= sigmoid_fast(bf16lo(g4[e]));
-                                hi *= sigmoid_fast(bf16hi(g4[e]));
-                            }
-                            ow[e] = pack_bf16x2(lo, hi);
-                        }
-                        *reinterpret_cast<uint4 *>(op + c8 * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
+                    gw[t][c8] = make_uint4(0, 0, 0, 0);
+                    if (ok && a.gate && row_ok && t < nb && c8 * 8 < a.C)
+                        gw[t][c8] = *reinterpret_cast<const uint4 *>(
+                            a.gate + (it.b0 + t) * a.sg0 + (long long)i * a.sg1 + it.h * a.sg2 + c8 * 8);
                 }
-                a.lse[((long long)b * a.H + h) * a.Nq + i] =
-                    live ? m_run[t] + lg2_approx(l_run[t]) * 0.6931471805599453f : -INFINITY;
+            }
+            if (ok) {
+                ok = mbar_wait(b_ofinal, n & 1, abort_flag, SITE_FWD_EPI | (n << 12));
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < BC; ++t) {
+                    if (t >= nb) break;
+                    uint32_t o[CP];
+                    tmem_ld_cols<CP>(tbase + T::T_O + t * CP + lane_off, o);
+                    if (!row_ok) continue;
+                    const int b = it.b0 + t;
+                    const bool live = l_run[t] > 0.f;
+                    const float inv = live ? rcp_approx(l_run[t]) : 0.f;
+                    __nv_bfloat16 *op = a.out + b * a.so0 + (long long)i * a.so1 + it.h * a.so2;
+#pragma unroll
+                    for (int c8 = 0; c8 < CP / 8; ++c8) {
+                        if (c8 * 8 < a.C) {
+                            const uint32_t g4[4] = {gw[t][c8].x, gw[t][c8].y, gw[t][c8].z, gw[t][c8].w};
+                            uint32_t ow[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float lo = __uint_as_float(o[c8 * 8 + 2 * e]) * inv;
+                                float hi = __uint_as_float(o[c8 * 8 + 2 * e + 1]) * inv;
+                                if (a.gate) {
+                                    lo *= sigmoid_fast(bf16lo(g4[e]));
+                                    hi *= sigmoid_fast(bf16hi(g4[e]));
+                                }
+                                ow[e] = pack_bf16x2(lo, hi);
+                            }
+                            *reinterpret_cast<uint4 *>(op + c8 * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        }
+                    }
+                    a.lse[((long long)b * a.H + it.h) * a.Nq + i] =
+                        live ? m_run[t] + lg2_approx(l_run[t]) * 0.6931471805599453f : -INFINITY;
+                }
             }
         }
     }
@@ -584,7 +642,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // Some wait ran out.  Every role has stopped; before shared memory and TMEM are
         // released, let the copies and MMAs already issued finish (bounded waits).
         if (warp == 4 && lane == 0) {
-            mbar_wait_drain(b_q, 0);
+            if (q_done > 0) mbar_wait_drain(b_q_full, (q_done - 1) & 1);
             for (int kk = max(0, k_done - KVS); kk < k_done; ++kk)
                 if (kk != a.skip_step) mbar_wait_drain(b_k_full(kk % KVS), (kk / KVS) & 1);
             for (int kk = max(0, v_done - KVS); kk < v_done; ++kk)

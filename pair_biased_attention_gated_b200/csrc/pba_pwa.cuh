@@ -233,31 +233,50 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
         const int row = warp * 32 + lane;
         const uint32_t lane_off = ((uint32_t)(warp * 32)) << 16;
         const int n = t0 + row;   // output row: i (forward) or j (dv)
+        const bool row_ok = n < a.N;
+        // The forward's gate rows do not depend on the products: the first GA slots are
+        // fetched before the MMAs are waited for, and every later one GA slots ahead of
+        // its use, so the loads' latency overlaps the MMAs and the stores.
+        constexpr int GA = CP == 64 ? 1 : BC / 2;
+        uint4 gq[GA][CP / 8];
+        auto fetch_gate = [&](int s, uint4 (&g)[CP / 8]) {
+#pragma unroll
+            for (int c8 = 0; c8 < CP / 8; ++c8) {
+                g[c8] = make_uint4(0, 0, 0, 0);
+                if (!DV && a.has_gate && row_ok && s < nb && c8 * 8 < a.C)
+                    g[c8] = *reinterpret_cast<const uint4 *>(a.gate + (b0 + s) * a.sg0 + (long long)n * a.sg1 +
+                                                             h * a.sg2 + c8 * 8);
+            }
+        };
+#pragma unroll
+        for (int s = 0; s < GA; ++s) fetch_gate(s, gq[s]);
         bool ok = mbar_wait(b_done, 0, abort_flag, SITE_PWA_EPI);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc_fence_after();
-            for (int s = 0; s < nb; ++s) {
+#pragma unroll
+            for (int s = 0; s < BC; ++s) {
+                if (s >= nb) break;   // uniform: the TMEM loads below are warp-collective
                 uint32_t o[CP];
                 tmem_ld_cols<CP>(tbase + s * CP + lane_off, o);
-                if (n >= a.N) continue;
+                uint4 g[CP / 8];
+#pragma unroll
+                for (int c8 = 0; c8 < CP / 8; ++c8) g[c8] = gq[s % GA][c8];
+                if (s + GA < BC) fetch_gate(s + GA, gq[s % GA]);
+                if (!row_ok) continue;
                 const int b = b0 + s;
                 __nv_bfloat16 *op = a.out + b * a.so0 + (long long)n * a.so1 + h * a.so2;
-                const __nv_bfloat16 *gp = (!DV && a.has_gate) ? a.gate + b * a.sg0 + (long long)n * a.sg1 + h * a.sg2 : nullptr;
+                const bool gated = !DV && a.has_gate;
 #pragma unroll
                 for (int c8 = 0; c8 < CP / 8; ++c8) {
                     if (c8 * 8 < a.C) {
-                        uint32_t gw[4] = {0, 0, 0, 0};
-                        if (gp) {
-                            const uint4 g4 = *reinterpret_cast<const uint4 *>(gp + c8 * 8);
-                            gw[0] = g4.x; gw[1] = g4.y; gw[2] = g4.z; gw[3] = g4.w;
-                        }
+                        const uint32_t gw[4] = {g[c8].x, g[c8].y, g[c8].z, g[c8].w};
                         uint32_t ow[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             float lo = __uint_as_float(o[c8 * 8 + 2 * e]);
                             float hi = __uint_as_float(o[c8 * 8 + 2 * e + 1]);
-                            if (gp) {
+                            if (gated) {
                                 lo *= sigmoid_fast(bf16lo(gw[e]));
                                 hi *= sigmoid_fast(bf16hi(gw[e]));
                             }
