@@ -53,6 +53,8 @@ def _load():
                                              d]
         lib.pba_oracle_pwa_fwd.argtypes = [i, i, i, i, d, d, u8, d, d, d]
         lib.pba_oracle_pwa_bwd.argtypes = [i, i, i, i, d, d, u8, d, d, d, d, d]
+        lib.pba_oracle_pair_bias_fwd.argtypes = [i, i, i, i, f, d, d, d, d, d]
+        lib.pba_oracle_pair_bias_bwd.argtypes = [i, i, i, i, f, d, d, d, d, d, d, d, d, d]
         lib.pba_oracle_threads.argtypes = []
         lib.pba_oracle_threads.restype = ctypes.c_int
         _lib = lib
@@ -205,3 +207,29 @@ def pwa_bwd(v, bias, keep, g, dout):
                            _d(dbias))
     return dv, dg, dbias
 
+
+def pair_bias_fwd(z, gamma, beta, w, eps=1e-5):
+    """Pair-bias projection: bias [H,Ni,Nj] = LayerNorm(z[i,j,:]; gamma, beta, eps) . w[:,h],
+    z [Ni,Nj,Cz], w [Cz,H]."""
+    lib = _load()
+    z, gamma, beta, w = map(_f64, (z, gamma, beta, w))
+    Ni, Nj, Cz = z.shape
+    H = w.shape[1]
+    bias = np.zeros((H, Ni, Nj))
+    lib.pba_oracle_pair_bias_fwd(Ni, Nj, Cz, H, float(eps), _d(z), _d(gamma), _d(beta), _d(w), _d(bias))
+    return bias
+
+
+def pair_bias_bwd(z, gamma, beta, w, dbias, eps=1e-5):
+    """dz [Ni,Nj,Cz], dw [Cz,H], dgamma [Cz], dbeta [Cz] of the pair-bias projection."""
+    lib = _load()
+    z, gamma, beta, w, dbias = map(_f64, (z, gamma, beta, w, dbias))
+    Ni, Nj, Cz = z.shape
+    H = w.shape[1]
+    dz = np.zeros_like(z)
+    dw = np.zeros((Cz, H))
+    dgamma = np.zeros(Cz)
+    dbeta = np.zeros(Cz)
+    lib.pba_oracle_pair_bias_bwd(Ni, Nj, Cz, H, float(eps), _d(z), _d(gamma), _d(beta), _d(w), _d(dbias),
+                                 _d(dz), _d(dw), _d(dgamma), _d(dbeta))
+    return dz, dw, dgamma, dbeta

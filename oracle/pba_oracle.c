@@ -403,3 +403,99 @@ void pba_oracle_pwa_bwd(int B, int H, int N, int C, const double *v, const doubl
         free(w); free(lse); free(doa);
     }
 }
+
+/*
+ * Pair-bias projection, the prologue of every pair-biased attention: the bias is
+ * projected from the pair representation ("AlphaFold3 open-source implementation" page,
+ * section "Model Efficiency"), after a LayerNorm of that representation (the Protenix
+ * page "Protenix: AlphaFold3的再现", section on scalability, which names LayerNorm as the
+ * op its custom CUDA kernel speeds up).  The pages print no formula; the plainest reading
+ * is a LayerNorm over the channels of z[i,j,:] followed by a linear map without bias:
+ *
+ *   mu = mean_c z[i,j,c],  var = mean_c (z - mu)^2,  xh_c = (z_c - mu) / sqrt(var + eps)
+ *   y_c = gamma_c xh_c + beta_c
+ *   bias[h,i,j] = sum_c y_c w[c,h]
+ *
+ * Backward for a given dbias[h,i,j] = g_h (the chain rule through the three steps):
+ *   dw[c,h]   = sum_{i,j} y_c g_h
+ *   dy_c      = sum_h w[c,h] g_h
+ *   dgamma_c  = sum_{i,j} dy_c xh_c ;  dbeta_c = sum_{i,j} dy_c
+ *   dxh_c     = gamma_c dy_c
+ *   dz_c      = (dxh_c - mean_c dxh - xh_c mean_c(dxh xh)) / sqrt(var + eps)
+ *
+ * Layouts: z, dz [Ni][Nj][Cz]; w [Cz][H]; gamma, beta [Cz]; bias, dbias [H][Ni][Nj].
+ */
+static void pb_normalize(int Cz, double eps, const double *zr, double *xh, double *sigma)
+{
+    double mu = 0.0;
+    for (int c = 0; c < Cz; ++c) mu += zr[c];
+    mu /= Cz;
+    double var = 0.0;
+    for (int c = 0; c < Cz; ++c) var += (zr[c] - mu) * (zr[c] - mu);
+    var /= Cz;
+    *sigma = sqrt(var + eps);
+    for (int c = 0; c < Cz; ++c) xh[c] = (zr[c] - mu) / *sigma;
+}
+
+void pba_oracle_pair_bias_fwd(int Ni, int Nj, int Cz, int H, double eps, const double *z,
+                              const double *gamma, const double *beta, const double *w,
+                              double *bias)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int i = 0; i < Ni; ++i) {
+        double *xh = malloc(sizeof(double) * (size_t)Cz + 8);
+        for (int j = 0; j < Nj; ++j) {
+            double sigma;
+            pb_normalize(Cz, eps, z + ((size_t)i * Nj + j) * Cz, xh, &sigma);
+            for (int h = 0; h < H; ++h) {
+                double s = 0.0;
+                for (int c = 0; c < Cz; ++c) s += (gamma[c] * xh[c] + beta[c]) * w[(size_t)c * H + h];
+                bias[((size_t)h * Ni + i) * Nj + j] = s;
+            }
+        }
+        free(xh);
+    }
+}
+
+void pba_oracle_pair_bias_bwd(int Ni, int Nj, int Cz, int H, double eps, const double *z,
+                              const double *gamma, const double *beta, const double *w,
+                              const double *dbias, double *dz, double *dw, double *dgamma,
+                              double *dbeta)
+{
+    memset(dw, 0, sizeof(double) * (size_t)Cz * H);
+    memset(dgamma, 0, sizeof(double) * (size_t)Cz);
+    memset(dbeta, 0, sizeof(double) * (size_t)Cz);
+    double *xh = malloc(sizeof(double) * (size_t)Cz + 8);
+    double *dy = malloc(sizeof(double) * (size_t)Cz + 8);
+    double *g = malloc(sizeof(double) * (size_t)H + 8);
+    /* sums over (i, j) in the order i = 0, 1, ...; j = 0, 1, ... */
+    for (int i = 0; i < Ni; ++i)
+        for (int j = 0; j < Nj; ++j) {
+            double sigma;
+            pb_normalize(Cz, eps, z + ((size_t)i * Nj + j) * Cz, xh, &sigma);
+            for (int h = 0; h < H; ++h) g[h] = dbias[((size_t)h * Ni + i) * Nj + j];
+            for (int c = 0; c < Cz; ++c) {
+                const double y = gamma[c] * xh[c] + beta[c];
+                double s = 0.0;
+                for (int h = 0; h < H; ++h) {
+                    dw[(size_t)c * H + h] += y * g[h];
+                    s += w[(size_t)c * H + h] * g[h];
+                }
+                dy[c] = s;
+                dgamma[c] += s * xh[c];
+                dbeta[c] += s;
+            }
+            double m1 = 0.0, m2 = 0.0;
+            for (int c = 0; c < Cz; ++c) {
+                m1 += gamma[c] * dy[c];
+                m2 += gamma[c] * dy[c] * xh[c];
+            }
+            m1 /= Cz;
+            m2 /= Cz;
+            double *dzr = dz + ((size_t)i * Nj + j) * Cz;
+            for (int c = 0; c < Cz; ++c) dzr[c] = (gamma[c] * dy[c] - m1 - xh[c] * m2) / sigma;
+        }
+    free(xh);
+    free(dy);
+    free(g);
+}
