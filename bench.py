@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import pba_inputs as pi  # noqa: E402
 
 METRIC = "pair-bias attention fwd / fwd+bwd TFLOP/s and %roofline on 1 B200"
@@ -86,6 +87,8 @@ KERNEL_SOURCES = {"pba_fwd_kernel": "pba_fwd.cuh"}   # every other attention ker
 def kernel_source_file(kernel: str) -> str:
     if kernel.startswith("pba_pwa_"):
         return "pba_pwa.cuh"
+    if kernel.startswith("pba_pair_bias_"):
+        return "pba_pairbias.cuh"
     return KERNEL_SOURCES.get(kernel, "pba_bwd.cuh")
 
 
@@ -639,6 +642,156 @@ def run_pwa(args, cfg):
         res["cpu_baseline"] = time_pwa_oracle(cfg, target_s=args.cpu_seconds, seed=args.seed)
     return res if rank == 0 else None
 
+# ---------------------------------------------------------------------------------------
+# pair-bias projection (--op pairbias): LayerNorm(z) -> linear -> bias, and its backward
+# ---------------------------------------------------------------------------------------
+PB_METRIC = "pair-bias projection (LayerNorm + linear) fwd+bwd GB/s and %roofline on 1 B200"
+
+
+def pb_work(N, Cz, H, Ni=None):
+    """Algorithmic bytes: forward reads z and writes the bf16 bias; backward reads z and the
+    fp32 dbias and writes dz (parameters and their gradients are a few KB)."""
+    Ni = N if Ni is None else Ni
+    P = Ni * N
+    fwd = P * Cz * 2 + H * P * 2
+    bwd = P * Cz * 2 + H * P * 4 + P * Cz * 2
+    return {"fwd_bytes": fwd, "bwd_bytes": bwd,
+            "kernels": {"pba_pair_bias_fwd_kernel": (0, fwd), "pba_pair_bias_bwd_kernel": (0, bwd),
+                        "pba_pair_bias_reduce_kernel": (0, 0), "pba_pair_bias_param_kernel": (0, 0)}}
+
+
+def time_pb_oracle(N, Cz, H, target_s, seed):
+    import oracle
+    rows = 1
+    for _ in range(2):
+        d = pi.make_pair_bias_inputs(rows, N, Cz, H, seed)
+        z = pi.bf16_bits_to_f64(d["z"])
+        args = [d[k].astype(np.float64) for k in ("gamma", "beta", "w")]
+        t0 = time.perf_counter()
+        oracle.pair_bias_fwd(z, *args)
+        oracle.pair_bias_bwd(z, *args, d["dbias"].astype(np.float64))
+        el = time.perf_counter() - t0
+        if el >= target_s or rows >= N:
+            break
+        rows = int(max(1, min(N, rows * target_s / max(el, 1e-6))))
+    w = pb_work(N, Cz, H, Ni=rows)
+    return {"value": (w["fwd_bytes"] + w["bwd_bytes"]) / el / 1e9, "unit": "GB/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": "pair-bias projection fwd+bwd on %d of %d rows i (x %d positions j, Cz=%d, H=%d), %.1f s; "
+                      "fp64 C loops, the forward over OpenMP threads, the backward on one (its sums run in one fixed order)"
+                      % (rows, N, N, Cz, H, el),
+            "seconds": el, "rows": rows}
+
+
+def run_pairbias(args, cfg):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    import pair_biased_attention_gated_b200 as pba
+    N, H, Cz = cfg.N, cfg.H, pi.CZ_PAIR
+    d = pi.make_pair_bias_inputs(N, N, Cz, H, seed=args.seed)
+    host = {"z": torch.from_numpy(d["z"].view(np.int16)).view(torch.bfloat16).pin_memory()}
+    for k in ("gamma", "beta", "w", "dbias"):
+        host[k] = torch.from_numpy(d[k]).pin_memory()
+    dev = {k: v.cuda() for k, v in host.items()}
+    bias = torch.empty((H, N, N), dtype=torch.bfloat16, device="cuda")
+    dz = torch.empty_like(dev["z"])
+    dw = torch.empty((Cz, H), dtype=torch.float32, device="cuda")
+    dg = torch.empty(Cz, dtype=torch.float32, device="cuda")
+    db = torch.empty(Cz, dtype=torch.float32, device="cuda")
+    dims = pba.pair_bias_dims(dev["z"], dbias=dev["dbias"])
+    ws = torch.empty(max(int(pba.lib.pba_pair_bias_bwd_workspace_size(ctypes.byref(dims))), 256),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pba.pba_pair_bias_fwd(dev["z"], dev["gamma"], dev["beta"], dev["w"], bias)
+        pba.pba_pair_bias_bwd(dev["z"], dev["gamma"], dev["beta"], dev["w"], dev["dbias"], dz, dw, dg, db, ws)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    pba.pba_device_status()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    torch.cuda.synchronize()
+    pba.profile_read()
+    pba.profile_enable(True)
+    sampler.start()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    pba.profile_enable(False)
+    kstats = pba.profile_read()
+    pba.pba_device_status()
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in ev)
+    houts = {"bias": bias, "dz": dz, "dw": dw, "dg": dg, "db": db}
+    hbufs = {k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in houts.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in hbufs.values())
+    K2 = max(1, min(K, 20))
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
+    torch.cuda.synchronize()
+    for i in range(K2):
+        flush.fill_(i & 0xFF)
+        ev2[i][0].record(stream)
+        for k2, t in host.items():
+            dev[k2].copy_(t, non_blocking=True)
+        step()
+        for k2, t in hbufs.items():
+            t.copy_(houts[k2], non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    pba.pba_device_status()
+
+    w = pb_work(N, Cz, H)
+    step_bytes = w["fwd_bytes"] + w["bwd_bytes"]
+    value = step_bytes * K / (elapsed_ms / 1e3) / 1e9
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    total_k = sum(ms for _, ms in kstats.values()) or 1.0
+    dom = max(kstats.items(), key=lambda kv: kv[1][1])[0] if kstats else None
+    roof = None
+    if dom:
+        launches, ms = kstats[dom]
+        avg_s = ms / launches / 1e3
+        kb = w["kernels"].get(dom, (0, 0))[1]
+        achieved = kb / avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": "%s (copy)" % peak_src,
+                "algorithmic_per_launch": {"flops": 0, "bytes": kb}, "avg_launch_us": round(avg_s * 1e6, 2),
+                "traffic": ncu_traffic(dom, "pairbias-" + cfg.name)}
+    ms_per_step = elapsed_ms / K
+    kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
+               for n, (l, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1])}
+    res = {
+        "metric": PB_METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded bf16 z (N(0,1) channels, per-position offset and scale), fp32 "
+                "LayerNorm and projection parameters and dbias",
+        "config": {"workload": "%s pair representation: z [%d, %d, %d] -> bias [%d, %d, %d]" % (cfg.name, N, N, Cz, H, N, N),
+                   "N": N, "Cz": Cz, "H": H, "passes": "fwd (bias) + bwd (dz, dw, dgamma, dbeta)",
+                   "l2": "flushed before every timed step (256 MiB write outside the events)",
+                   "parallelism": "single GPU"},
+        "roofline": roof,
+        "step_roofline": {"time_us": round(step_bytes / (hbm * 1e9) * 1e6, 2),
+                          "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms_per_step, 4)},
+        "kernels": kernels, "gpu_launches": sum(l for l, _ in kstats.values()), "clocks": clocks,
+        "e2e": {"value": round(step_bytes * K2 / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = time_pb_oracle(N, Cz, H, args.cpu_seconds, args.seed)
+    return res if rank == 0 else None
+
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -651,16 +804,17 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="attention", choices=["attention", "pwa"],
-                    help="pwa: MSA pair-weighted averaging of the workload's value rows (one GPU)")
+    ap.add_argument("--op", default="attention", choices=["attention", "pwa", "pairbias"],
+                    help="pwa: MSA pair-weighted averaging of the workload's value rows; pairbias: "
+                         "the LayerNorm + projection that makes the workload's bias (one GPU each)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = pi.CONFIGS[args.config]
-    if args.op == "pwa":
+    if args.op != "attention":
         if args.impl == "reference" or args.gpus != 1:
-            ap.error("--op pwa times our kernels on one GPU; its oracle baseline is the cpu_baseline key")
-        res = run_pwa(args, cfg)
+            ap.error("--op %s times our kernels on one GPU; its oracle baseline is the cpu_baseline key" % args.op)
+        res = run_pwa(args, cfg) if args.op == "pwa" else run_pairbias(args, cfg)
     else:
         res = run_reference(args, cfg) if args.impl == "reference" else run_ours(args, cfg)
     if res is not None:

@@ -173,6 +173,50 @@ pba_status pba_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *k
                        size_t workspace_bytes, const pba_dims *dims, void *stream);
 
 /*
+ * Pair-bias projection, the prologue that makes an attention's bias from the pair
+ * representation ("AlphaFold3 open-source implementation" page, Model Efficiency section:
+ * every attention projects its pair bias from the pair representation; the Protenix page,
+ * scalability section: the LayerNorm of the pair representation is worth a custom
+ * kernel).  A LayerNorm over the Cz channels of z[i,j,:], then a linear map without bias:
+ *   bias[h,i,j] = sum_c (gamma_c (z[i,j,c] - mean) / sqrt(var + eps) + beta_c) w[c,h]
+ * (mean and biased variance over the channels of one position).  The output feeds
+ * pba_fwd / pba_bwd as their bias (Ni = Nq, Nj = Nk); a transposed bias (the ending-node
+ * triangle attention) is the same call with the two z strides exchanged.
+ *
+ * Sizes: Cz in {64, 128, 192, 256}; 1 <= H <= 16; eps finite and > 0; Ni, Nj >= 0.
+ * z: bf16, element (i, j, c) at z[i * sz[0] + j * sz[1] + c]; base 16-byte aligned,
+ * sz[0] and sz[1] positive multiples of 8 (the Tensor Memory Accelerator's rule).
+ * gamma, beta: fp32 [Cz]; w: fp32 [Cz][H] (row c, column h), all device pointers.
+ * bias: bf16, element (h, i, j) at bias[h * sbias[0] + i * sbias[1] + j].
+ */
+typedef struct {
+    int Ni, Nj, Cz, H;
+    float eps;
+    int64_t sz[2];      /* z (and dz) strides of i and j, in elements; channel stride 1 */
+    int64_t sbias[2];   /* bias strides of h and i, in elements; j stride 1 */
+    int64_t sdbias[2];  /* dbias strides of h and i, in elements; j stride 1 */
+} pba_pair_bias_dims;
+
+pba_status pba_pair_bias_fwd(const pba_bf16 *z, const float *gamma, const float *beta,
+                             const float *w, pba_bf16 *bias, const pba_pair_bias_dims *dims,
+                             void *stream);
+
+/*
+ * Backward of pba_pair_bias_fwd for a given dbias (fp32, e.g. the dbias of pba_bwd):
+ *   dz (bf16, the layout of z), dw (fp32 [Cz][H]), dgamma, dbeta (fp32 [Cz]), all written
+ *   in full.  dw, dgamma and dbeta are sums over all Ni * Nj positions, added in an order
+ *   that depends only on the sizes: bit-identical from run to run.
+ * workspace: caller-owned device memory of pba_pair_bias_bwd_workspace_size(dims) bytes,
+ * 256-byte aligned (PBA_ERR_WORKSPACE if smaller).
+ */
+size_t pba_pair_bias_bwd_workspace_size(const pba_pair_bias_dims *dims);
+pba_status pba_pair_bias_bwd(const pba_bf16 *z, const float *gamma, const float *beta,
+                             const float *w, const float *dbias, pba_bf16 *dz, float *dw,
+                             float *dgamma, float *dbeta, void *workspace,
+                             size_t workspace_bytes, const pba_pair_bias_dims *dims,
+                             void *stream);
+
+/*
  * Synchronizes `stream`, then reports and clears the device watchdog word of the
  * current device: PBA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, PBA_ERR_CUDA if the synchronization itself failed, else PBA_OK.

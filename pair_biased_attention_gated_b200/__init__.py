@@ -57,6 +57,20 @@ lib.pba_pwa_fwd.argtypes = [_vp] * 7 + [ctypes.c_size_t, ctypes.POINTER(PbaDims)
 lib.pba_pwa_fwd.restype = ctypes.c_int
 lib.pba_pwa_bwd.argtypes = [_vp] * 10 + [ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
 lib.pba_pwa_bwd.restype = ctypes.c_int
+
+
+class PbaPairBiasDims(ctypes.Structure):
+    _fields_ = [("Ni", ctypes.c_int32), ("Nj", ctypes.c_int32), ("Cz", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("eps", ctypes.c_float), ("sz", ctypes.c_int64 * 2),
+                ("sbias", ctypes.c_int64 * 2), ("sdbias", ctypes.c_int64 * 2)]
+
+
+lib.pba_pair_bias_fwd.argtypes = [_vp] * 5 + [ctypes.POINTER(PbaPairBiasDims), _vp]
+lib.pba_pair_bias_fwd.restype = ctypes.c_int
+lib.pba_pair_bias_bwd_workspace_size.argtypes = [ctypes.POINTER(PbaPairBiasDims)]
+lib.pba_pair_bias_bwd_workspace_size.restype = ctypes.c_size_t
+lib.pba_pair_bias_bwd.argtypes = [_vp] * 10 + [ctypes.c_size_t, ctypes.POINTER(PbaPairBiasDims), _vp]
+lib.pba_pair_bias_bwd.restype = ctypes.c_int
 lib.pba_device_status.argtypes = [_vp]
 lib.pba_device_status.restype = ctypes.c_int
 lib.pba_status_string.argtypes = [ctypes.c_int]
@@ -256,8 +270,8 @@ def profile_enable(on: bool = True) -> None:
 
 def profile_read() -> dict:
     """{kernel name: (launches, total device ms)} since the last read."""
-    arr = (PbaKernelStat * 16)()
-    n = lib.pba_profile_read(arr, 16)
+    arr = (PbaKernelStat * 32)()
+    n = lib.pba_profile_read(arr, 32)
     if n < 0:
         raise PbaError(3, "reading kernel timing events failed")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}
@@ -288,3 +302,64 @@ def pwa_bwd(v, bias, key_mask, gate, out, dout, want_dbias: bool = True, stream=
     pba_pwa_bwd(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, stream)
     return dv, dgate, dbias
 
+
+def pair_bias_dims(z, bias=None, dbias=None, eps: float = 1e-5) -> PbaPairBiasDims:
+    """pba_pair_bias_dims for z [Ni, Nj, Cz] (channel stride 1), bias [H, Ni, Nj] and dbias
+    [H, Ni, Nj] (j stride 1); H is taken from bias or dbias."""
+    Ni, Nj, Cz = z.shape
+    assert z.stride(2) == 1, "z: channel stride must be 1"
+    ref = bias if bias is not None else dbias
+    d = PbaPairBiasDims()
+    d.Ni, d.Nj, d.Cz, d.H = Ni, Nj, Cz, ref.shape[0]
+    d.eps = eps
+    d.sz[0], d.sz[1] = z.stride(0), z.stride(1)
+    if bias is not None:
+        assert bias.stride(2) == 1, "bias: j stride must be 1"
+        d.sbias[0], d.sbias[1] = bias.stride(0), bias.stride(1)
+    if dbias is not None:
+        assert dbias.stride(2) == 1, "dbias: j stride must be 1"
+        d.sdbias[0], d.sdbias[1] = dbias.stride(0), dbias.stride(1)
+    return d
+
+
+def pba_pair_bias_fwd(z, gamma, beta, w, bias, eps: float = 1e-5, stream=None) -> None:
+    """Pair-bias projection into a preallocated bf16 `bias` [H, Ni, Nj]: LayerNorm over the
+    channels of z [Ni, Nj, Cz] (bf16; gamma, beta fp32 [Cz]) then w (fp32 [Cz, H])."""
+    d = pair_bias_dims(z, bias=bias, eps=eps)
+    _check(lib.pba_pair_bias_fwd(_ptr(z), _ptr(gamma), _ptr(beta), _ptr(w), _ptr(bias),
+                                 ctypes.byref(d), _stream(stream)))
+
+
+def pba_pair_bias_bwd(z, gamma, beta, w, dbias, dz, dw, dgamma, dbeta, workspace, eps: float = 1e-5,
+                      stream=None) -> None:
+    """Backward of pba_pair_bias_fwd for a given fp32 dbias [H, Ni, Nj], into preallocated dz
+    (like z), dw (fp32 [Cz, H]), dgamma and dbeta (fp32 [Cz])."""
+    d = pair_bias_dims(z, dbias=dbias, eps=eps)
+    _check(lib.pba_pair_bias_bwd(_ptr(z), _ptr(gamma), _ptr(beta), _ptr(w), _ptr(dbias), _ptr(dz),
+                                 _ptr(dw), _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                 workspace.numel() if workspace is not None else 0, ctypes.byref(d),
+                                 _stream(stream)))
+
+
+def pair_bias_fwd(z, gamma, beta, w, eps: float = 1e-5, stream=None):
+    """bias [H, Ni, Nj] (bf16) = LayerNorm(z[i, j, :]; gamma, beta, eps) . w[:, h]."""
+    import torch
+    Ni, Nj, Cz = z.shape
+    bias = torch.empty((w.shape[1], Ni, Nj), dtype=torch.bfloat16, device=z.device)
+    pba_pair_bias_fwd(z, gamma, beta, w, bias, eps, stream)
+    return bias
+
+
+def pair_bias_bwd(z, gamma, beta, w, dbias, eps: float = 1e-5, stream=None):
+    """(dz, dw, dgamma, dbeta) of the pair-bias projection for a given fp32 dbias."""
+    import torch
+    Cz = z.shape[2]
+    dz = torch.empty_like(z)
+    dw = torch.empty((Cz, w.shape[1]), dtype=torch.float32, device=z.device)
+    dgamma = torch.empty(Cz, dtype=torch.float32, device=z.device)
+    dbeta = torch.empty(Cz, dtype=torch.float32, device=z.device)
+    d = pair_bias_dims(z, dbias=dbias, eps=eps)
+    ws = torch.empty(max(int(lib.pba_pair_bias_bwd_workspace_size(ctypes.byref(d))), 256),
+                     dtype=torch.uint8, device=z.device)
+    pba_pair_bias_bwd(z, gamma, beta, w, dbias, dz, dw, dgamma, dbeta, ws, eps, stream)
+    return dz, dw, dgamma, dbeta

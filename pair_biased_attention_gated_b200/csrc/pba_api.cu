@@ -20,6 +20,7 @@
 #include "../../include/pba.h"
 #include "pba_bwd.cuh"
 #include "pba_fwd.cuh"
+#include "pba_pairbias.cuh"
 #include "pba_pwa.cuh"
 
 namespace {
@@ -43,13 +44,16 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 
 // ---------------------------------------------------------------------------- profiling
 enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS,
-                K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS, K_COUNT };
+                K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS,
+                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
                                            "pba_dbias_kernel",
                                            "pba_dq_convert_kernel", "zero_rows_kernel",
                                            "pba_pwa_weights_kernel", "pba_pwa_gemm_kernel (out)",
                                            "pba_pwa_pre_kernel", "pba_pwa_gemm_kernel (dv)",
-                                           "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel"};
+                                           "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel",
+                                           "pba_pair_bias_fwd_kernel", "pba_pair_bias_bwd_kernel",
+                                           "pba_pair_bias_reduce_kernel", "pba_pair_bias_param_kernel"};
 struct ProfRec {
     int kid;
     cudaEvent_t a, b;
@@ -117,14 +121,14 @@ CUtensorMapSwizzle swizzle_for_row_bytes(int rowb) {
 
 // A [B, N, H, C] bf16 tensor (C stride 1) as a 4-D map (C, H, N, B), box (CP, 1, 128, 1).
 pba_status map_bnhc(CUtensorMap *m, const void *base, int B, int N, int H, int C,
-                    const int64_t s[3], int CP, const char *name) {
+                    const int64_t s[3], int CP, const char *name, int rows = 128) {
     cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)(N > 0 ? N : 1),
                           (cuuint64_t)(B > 0 ? B : 1)};
     // a dimension of extent 1 is never stepped along: give it a harmless legal stride
     cuuint64_t strides[3] = {(cuuint64_t)(H > 1 ? s[2] * 2 : 16),
                              (cuuint64_t)(N > 1 ? s[1] * 2 : 16),
                              (cuuint64_t)(B > 1 ? s[0] * 2 : 16)};
-    cuuint32_t box[4] = {(cuuint32_t)CP, 1, 128, 1};
+    cuuint32_t box[4] = {(cuuint32_t)CP, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -504,10 +508,10 @@ pba_status noalloc_scratch(void **out) {
 // ---------------------------------------------------------------------------- pair-weighted
 // The [H, N, Wld] bf16 weights as a 3-D map (N, N, H), box (64, 128, 1), 128-byte swizzle:
 // the same tiles as the bias.
-pba_status map_w(CUtensorMap *m, void *base, int H, int N, int Wld) {
+pba_status map_w(CUtensorMap *m, void *base, int H, int N, int Wld, int rows = 128) {
     cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H};
     cuuint64_t strides[2] = {(cuuint64_t)Wld * 2, (cuuint64_t)N * Wld * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -625,8 +629,9 @@ pba_status launch_pwa_fwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t
     a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
     pba_status st;
     CUtensorMap tw, tv;
-    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld)) != PBA_OK) return st;
-    if ((st = map_bnhc(&tv, v, d->B, pl.N, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
+    // the GEMM's stages: 128 output rows x 64 reduction columns of w, 64 rows of each V tile
+    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld, 128)) != PBA_OK) return st;
+    if ((st = map_bnhc(&tv, v, d->B, pl.N, d->H, d->C, d->sv, CP, "v", 64)) != PBA_OK) return st;
     if ((st = launch_pwa_weights(a, s)) != PBA_OK) return st;
     return launch_pwa_gemm<CP>(tw, tv, a, false, s);
 }
@@ -647,14 +652,18 @@ pba_status launch_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t
     a.dout = reinterpret_cast<const __nv_bfloat16 *>(dout);
     a.si0 = d->so[0]; a.si1 = d->so[1]; a.si2 = d->so[2];
     pba_status st;
-    CUtensorMap tw, tv, tdo;
-    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld)) != PBA_OK) return st;
+    // dW partials: 128-row tiles of dOa and V; dv GEMM: 64 x 128 blocks of w (rows i =
+    // reduction, columns j = output) and 64-row tiles of dOa
+    CUtensorMap tw, tv, tdo, tdo64;
+    if ((st = map_w(&tw, a.w, d->H, pl.N, pl.Wld, 64)) != PBA_OK) return st;
     if ((st = map_bnhc(&tv, v, d->B, pl.N, d->H, d->C, d->sv, CP, "v")) != PBA_OK) return st;
     if (gate) {
         const int64_t sd[3] = {(int64_t)pl.N * d->H * d->C, (int64_t)d->H * d->C, d->C};
         if ((st = map_bnhc(&tdo, a.doa, d->B, pl.N, d->H, d->C, sd, CP, "dOa")) != PBA_OK) return st;
+        if ((st = map_bnhc(&tdo64, a.doa, d->B, pl.N, d->H, d->C, sd, CP, "dOa", 64)) != PBA_OK) return st;
     } else {
         if ((st = map_bnhc(&tdo, dout, d->B, pl.N, d->H, d->C, d->so, CP, "dout")) != PBA_OK) return st;
+        if ((st = map_bnhc(&tdo64, dout, d->B, pl.N, d->H, d->C, d->so, CP, "dout", 64)) != PBA_OK) return st;
     }
     if ((st = launch_pwa_weights(a, s)) != PBA_OK) return st;
     cudaError_t e;
@@ -669,7 +678,7 @@ pba_status launch_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t
     pba::PwaArgs av = a;
     av.out = reinterpret_cast<__nv_bfloat16 *>(dv);
     av.so0 = d->sv[0]; av.so1 = d->sv[1]; av.so2 = d->sv[2];
-    if ((st = launch_pwa_gemm<CP>(tw, tdo, av, true, s)) != PBA_OK) return st;
+    if ((st = launch_pwa_gemm<CP>(tw, tdo64, av, true, s)) != PBA_OK) return st;
     if (dbias) {
         if ((st = set_smem(pba::pba_pwa_dw_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
         cudaFuncSetAttribute(pba::pba_pwa_dw_kernel<CP>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -704,6 +713,127 @@ pba_status check_pwa_common(const pba_bf16 *v, const pba_bf16 *bias, const uint8
     if (bias && d->Nq > 1 && d->sbias[1] <= 0) return fail(PBA_ERR_INVALID_ARG, "bias: row stride must be positive");
     (void)mask;
     return get_encoder();
+}
+
+// ------------------------------------------------------------------ pair-bias projection
+int pb_hp(int H) { return H <= 4 ? 4 : (H <= 8 ? 8 : 16); }
+
+pba_status check_pb_dims(const pba_pair_bias_dims *d) {
+    if (!d) return fail(PBA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->Ni < 0 || d->Nj < 0 || d->Cz < 0 || d->H < 0) return fail(PBA_ERR_INVALID_ARG, "negative size");
+    if (d->Cz != 64 && d->Cz != 128 && d->Cz != 192 && d->Cz != 256)
+        return fail(PBA_ERR_UNSUPPORTED, "Cz=%d: must be 64, 128, 192 or 256", d->Cz);
+    if (d->H < 1 || d->H > 16) return fail(PBA_ERR_UNSUPPORTED, "H=%d: must be in [1, 16]", d->H);
+    if (!(d->eps > 0.f) || !std::isfinite(d->eps)) return fail(PBA_ERR_INVALID_ARG, "eps must be finite and > 0");
+    if (d->Ni > (1 << 24) || d->Nj > (1 << 24)) return fail(PBA_ERR_UNSUPPORTED, "sizes too large");
+    if ((long long)d->Ni * ((d->Nj + 127) / 128) > INT_MAX) return fail(PBA_ERR_UNSUPPORTED, "too many tiles");
+    const int ext[2] = {d->Ni, d->Nj};
+    for (int k = 0; k < 2; ++k) {
+        if (ext[k] > 1 && (d->sz[k] <= 0 || d->sz[k] % 8 != 0))
+            return fail(PBA_ERR_INVALID_ARG, "z: stride %d must be a positive multiple of 8 elements", k);
+        if (d->sz[k] * 2 >= (int64_t(1) << 40)) return fail(PBA_ERR_UNSUPPORTED, "z: stride too large");
+    }
+    return PBA_OK;
+}
+
+long long pb_grid(const pba_pair_bias_dims *d, int smem_bytes) {
+    const long long tiles = (long long)d->Ni * ((d->Nj + 127) / 128);
+    long long per_sm = 233472 / (smem_bytes + 1024);
+    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    // a fixed function of the sizes (not of the device): the order of the backward's sums
+    // depends on it
+    const long long g = per_sm * kSmCount;
+    return tiles < g ? tiles : g;
+}
+
+template <int CZ, int HP>
+int pb_smem() { return pba::PbTraits<CZ, HP>::SMEM_BYTES; }
+
+int pb_smem_for(int Cz, int HP) {
+#define PB_CASE(cz, hp) if (Cz == cz && HP == hp) return pb_smem<cz, hp>();
+    PB_CASE(64, 4) PB_CASE(64, 8) PB_CASE(64, 16) PB_CASE(128, 4) PB_CASE(128, 8) PB_CASE(128, 16)
+    PB_CASE(192, 4) PB_CASE(192, 8) PB_CASE(192, 16) PB_CASE(256, 4) PB_CASE(256, 8) PB_CASE(256, 16)
+#undef PB_CASE
+    return 0;
+}
+
+// workspace: the per-block partials [grid][Cz * HP + HP], then their sums [Cz * HP + HP]
+size_t pb_ws_bytes(const pba_pair_bias_dims *d) {
+    const int HP = pb_hp(d->H);
+    const long long g = pb_grid(d, pb_smem_for(d->Cz, HP));
+    return (size_t)((g > 0 ? g : 1) + 1) * ((size_t)d->Cz * HP + HP) * 4;
+}
+
+// z as a 3-D map (Cz, Nj, Ni), box (64, 128, 1), 128-byte swizzle
+pba_status map_z(CUtensorMap *m, const void *z, const pba_pair_bias_dims *d) {
+    cuuint64_t dims[3] = {(cuuint64_t)d->Cz, (cuuint64_t)(d->Nj > 0 ? d->Nj : 1), (cuuint64_t)(d->Ni > 0 ? d->Ni : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)(d->Nj > 1 ? d->sz[1] * 2 : 16), (cuuint64_t)(d->Ni > 1 ? d->sz[0] * 2 : 16)};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(z), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "tensor map for z failed (CUresult %d)", (int)r);
+    return PBA_OK;
+}
+
+pba::PbArgs pb_args(const pba_pair_bias_dims *d, const float *gamma, const float *beta, const float *w) {
+    pba::PbArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.Ni = d->Ni; a.Nj = d->Nj; a.Cz = d->Cz; a.H = d->H;
+    a.nJt = (d->Nj + 127) / 128;
+    a.tiles = (int)((long long)d->Ni * a.nJt);
+    a.eps = d->eps;
+    a.gamma = gamma; a.beta = beta; a.w = w;
+    a.sz0 = d->sz[0]; a.sz1 = d->sz[1];
+    a.sb0 = d->sbias[0]; a.sb1 = d->sbias[1];
+    a.sd0 = d->sdbias[0]; a.sd1 = d->sdbias[1];
+    a.hp = pb_hp(d->H);
+    return a;
+}
+
+template <int CZ, int HP>
+pba_status launch_pb(bool bwd, const CUtensorMap &tm, pba::PbArgs a, const pba_pair_bias_dims *d, cudaStream_t s) {
+    using T = pba::PbTraits<CZ, HP>;
+    const long long grid = pb_grid(d, T::SMEM_BYTES);
+    a.nparts = (int)grid;
+    pba_status st;
+    cudaError_t e;
+    if (!bwd) {
+        if ((st = set_smem(pba::pba_pair_bias_fwd_kernel<CZ, HP>, T::SMEM_BYTES)) != PBA_OK) return st;
+        ProfScope ps(K_PB_FWD, s);
+        pba::pba_pair_bias_fwd_kernel<CZ, HP><<<(unsigned)grid, 128, T::SMEM_BYTES, s>>>(tm, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_fwd_kernel launch");
+        return PBA_OK;
+    }
+    if ((st = set_smem(pba::pba_pair_bias_bwd_kernel<CZ, HP>, T::SMEM_BYTES)) != PBA_OK) return st;
+    {
+        ProfScope ps(K_PB_BWD, s);
+        pba::pba_pair_bias_bwd_kernel<CZ, HP><<<(unsigned)grid, 128, T::SMEM_BYTES, s>>>(tm, a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_bwd_kernel launch");
+    a.sums = a.part + grid * ((long long)CZ * HP + HP);
+    {
+        ProfScope ps(K_PB_REDUCE, s);
+        pba::pba_pair_bias_reduce_kernel<<<(unsigned)((CZ * HP + HP + 31) / 32), 512, 0, s>>>(a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_reduce_kernel launch");
+    {
+        ProfScope ps(K_PB_PARAM, s);
+        pba::pba_pair_bias_param_kernel<<<(unsigned)((CZ + 127) / 128), 128, 0, s>>>(a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_param_kernel launch");
+    return PBA_OK;
+}
+
+pba_status dispatch_pb(bool bwd, const CUtensorMap &tm, const pba::PbArgs &a, const pba_pair_bias_dims *d,
+                       cudaStream_t s) {
+    const int HP = pb_hp(d->H);
+#define PB_CASE(cz, hp) if (d->Cz == cz && HP == hp) return launch_pb<cz, hp>(bwd, tm, a, d, s);
+    PB_CASE(64, 4) PB_CASE(64, 8) PB_CASE(64, 16) PB_CASE(128, 4) PB_CASE(128, 8) PB_CASE(128, 16)
+    PB_CASE(192, 4) PB_CASE(192, 8) PB_CASE(192, 16) PB_CASE(256, 4) PB_CASE(256, 8) PB_CASE(256, 16)
+#undef PB_CASE
+    return fail(PBA_ERR_UNSUPPORTED, "unsupported Cz / H");
 }
 
 }  // namespace
@@ -841,7 +971,8 @@ pba_status pba_device_status(void *stream) {
         cudaMemcpyFromSymbol(&site, pba::g_pba_watchdog_site, sizeof(site));
         cudaMemcpyToSymbol(pba::g_pba_watchdog, &zero, sizeof(zero));
         cudaMemcpyToSymbol(pba::g_pba_watchdog_site, &zero, sizeof(zero));
-        if ((site & 0xFFFu) == pba::SITE_FWD_ALIGN || (site & 0xFFFu) == pba::SITE_PWA_ALIGN)
+        if ((site & 0xFFFu) == pba::SITE_FWD_ALIGN || (site & 0xFFFu) == pba::SITE_PWA_ALIGN ||
+            (site & 0xFFFu) == pba::SITE_PB_ALIGN)
             return fail(PBA_ERR_UNSUPPORTED, "forward kernel refused: dynamic shared memory "
                                              "is not 1024-byte aligned");
         return fail(PBA_ERR_TIMEOUT, "a bounded in-kernel wait ran out (site 0x%x)", site);
@@ -952,6 +1083,67 @@ pba_status pba_pwa_bwd(const pba_bf16 *v, const pba_bf16 *bias, const uint8_t *k
         case 32: return launch_pwa_bwd<32>(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, pl, d, s);
         default: return launch_pwa_bwd<64>(v, bias, key_mask, gate, out, dout, dv, dbias, dgate, ws, pl, d, s);
     }
+}
+
+pba_status pba_pair_bias_fwd(const pba_bf16 *z, const float *gamma, const float *beta, const float *w,
+                             pba_bf16 *bias, const pba_pair_bias_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_pb_dims(d);
+    if (st != PBA_OK) return st;
+    if (d->Ni == 0 || d->Nj == 0) return PBA_OK;
+    if (!z || !gamma || !beta || !w || !bias) return fail(PBA_ERR_INVALID_ARG, "z, gamma, beta, w and bias are required");
+    if (!aligned16(z)) return fail(PBA_ERR_INVALID_ARG, "z must be 16-byte aligned");
+    if ((d->H > 1 && d->sbias[0] <= 0) || (d->Ni > 1 && d->sbias[1] <= 0))
+        return fail(PBA_ERR_INVALID_ARG, "bias strides must be positive");
+    if ((st = get_encoder()) != PBA_OK) return st;
+    CUtensorMap tm;
+    if ((st = map_z(&tm, z, d)) != PBA_OK) return st;
+    pba::PbArgs a = pb_args(d, gamma, beta, w);
+    a.bias = reinterpret_cast<__nv_bfloat16 *>(bias);
+    return dispatch_pb(false, tm, a, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t pba_pair_bias_bwd_workspace_size(const pba_pair_bias_dims *d) {
+    if (check_pb_dims(d) != PBA_OK) return 0;
+    return pb_ws_bytes(d);
+}
+
+pba_status pba_pair_bias_bwd(const pba_bf16 *z, const float *gamma, const float *beta, const float *w,
+                             const float *dbias, pba_bf16 *dz, float *dw, float *dgamma, float *dbeta,
+                             void *workspace, size_t workspace_bytes, const pba_pair_bias_dims *d, void *stream) {
+    g_last_error.clear();
+    pba_status st = check_pb_dims(d);
+    if (st != PBA_OK) return st;
+    if (!gamma || !beta || !w || !dw || !dgamma || !dbeta)
+        return fail(PBA_ERR_INVALID_ARG, "gamma, beta, w, dw, dgamma and dbeta are required");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d->Ni == 0 || d->Nj == 0) {
+        // no position: every parameter gradient is an empty sum
+        cudaError_t e;
+        if ((e = cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)d->Cz * d->H, s)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dgamma, 0, sizeof(float) * (size_t)d->Cz, s)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dbeta, 0, sizeof(float) * (size_t)d->Cz, s)) != cudaSuccess)
+            return cuda_fail(e, "cudaMemsetAsync");
+        return PBA_OK;
+    }
+    if (!z || !dbias || !dz) return fail(PBA_ERR_INVALID_ARG, "z, dbias and dz are required");
+    if (!aligned16(z) || !aligned16(dz)) return fail(PBA_ERR_INVALID_ARG, "z and dz must be 16-byte aligned");
+    if ((d->H > 1 && d->sdbias[0] <= 0) || (d->Ni > 1 && d->sdbias[1] <= 0))
+        return fail(PBA_ERR_INVALID_ARG, "dbias strides must be positive");
+    const size_t need = pb_ws_bytes(d);
+    if (!workspace || workspace_bytes < need)
+        return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(PBA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if ((st = get_encoder()) != PBA_OK) return st;
+    CUtensorMap tm;
+    if ((st = map_z(&tm, z, d)) != PBA_OK) return st;
+    pba::PbArgs a = pb_args(d, gamma, beta, w);
+    a.dbias = dbias;
+    a.dz = reinterpret_cast<__nv_bfloat16 *>(dz);
+    a.part = static_cast<float *>(workspace);
+    a.dw = dw; a.dgamma = dgamma; a.dbeta = dbeta;
+    return dispatch_pb(true, tm, a, d, s);
 }
 
 const char *pba_status_string(pba_status s) {

@@ -1,0 +1,420 @@
+// Pair-bias projection: the prologue that makes every pair-biased attention's bias from the
+// pair representation z ("AlphaFold3 open-source implementation" page, Model Efficiency
+// section: each attention projects its pair bias from the pair representation; the
+// Protenix page, scalability section: LayerNorm over the pair representation is the op
+// worth a custom kernel).  Read as a LayerNorm over the channels of z[i,j,:] followed by a
+// linear map without bias:
+//
+//   xh = (z - mean) / sqrt(var + eps),  y = gamma xh + beta,  bias[h,i,j] = sum_c y_c w[c,h]
+//
+// and its backward for a given dbias:
+//   dz_c = rstd (dxh_c - mean_c dxh - xh_c mean_c(dxh xh)),  dxh_c = gamma_c sum_h w[c,h] g_h
+//   dw[c,h] = sum_pos y_c g_h,  dgamma_c = sum_pos dy_c xh_c,  dbeta_c = sum_pos dy_c
+//
+// The kernels rewrite the sums so that one pass over a row suffices.  With w' = gamma w
+// (columns padded with zeros to HP), S_h = sum_c w'[c,h] and acc_h = sum_c w'[c,h](z_c - mean):
+//   bias_h = rstd acc_h + sum_c beta_c w[c,h]
+//   mean_c dxh = sum_h g_h S_h / Cz,  mean_c(dxh xh) = rstd sum_h g_h acc_h / Cz
+// and the parameter gradients need only A[c,h] = sum_pos xh_c g_h and G_h = sum_pos g_h:
+//   dw[c,h] = gamma_c A[c,h] + beta_c G_h,  dgamma_c = sum_h w[c,h] A[c,h],
+//   dbeta_c = sum_h w[c,h] G_h.
+//
+// Work unit: a tile of 128 consecutive positions j of one row i.  Every block (128 threads,
+// thread = position in phase 1) is persistent over tiles blockIdx.x, blockIdx.x + gridDim.x,
+// ...; tiles arrive by TMA (the Cz channels as 64-channel boxes with the 128-byte swizzle,
+// so that each thread reads its own row without bank conflicts) into two buffers, the next
+// but one tile loading while the current one is processed.  HBM-bound: z is read once and
+// the bias (or dz) written once.  The backward's parameter sums are added per block in tile
+// order, then over the blocks in block order by two small kernels (bit-stable).
+#pragma once
+
+#include "pba_device.cuh"
+
+namespace pba {
+
+struct PbArgs {
+    int Ni, Nj, Cz, H;
+    int nJt, tiles;                 // tiles of 128 positions along j per row, all tiles
+    float eps;
+    const float *gamma, *beta, *w;  // [Cz], [Cz], [Cz][H]
+    __nv_bfloat16 *bias;            // forward output [H][Ni][Nj], strides (sb0, sb1), j stride 1
+    long long sb0, sb1;
+    const float *dbias;             // backward input, strides (sd0, sd1), j stride 1
+    long long sd0, sd1;
+    __nv_bfloat16 *dz;              // backward output, the layout of z: strides (sz0, sz1)
+    long long sz0, sz1;
+    float *part;                    // [gridDim.x][Cz * HP + HP] per-block sums A, G
+    float *sums;                    // [Cz * HP + HP] their sums over the blocks
+    float *dw, *dgamma, *dbeta;
+    int nparts, hp;
+};
+
+enum : unsigned { SITE_PB_FWD = 0x501, SITE_PB_BWD = 0x502, SITE_PB_ALIGN = 0x5FF };
+
+template <int CZ, int HP>
+struct PbTraits {
+    static constexpr int TILE_BYTES = 128 * CZ * 2;            // CZ / 64 boxes of 16 KB
+    static constexpr int OFF_Z = 0;                            // 1024-byte aligned (SW128)
+    static constexpr int OFF_W = OFF_Z + 2 * TILE_BYTES;       // w' fp32, channel pairs interleaved
+    static constexpr int OFF_S = OFF_W + CZ * HP * 4;          // S [HP]
+    static constexpr int OFF_BB = OFF_S + HP * 4;              // sum_c beta_c w[c,h] [HP]
+    static constexpr int OFF_MU = OFF_BB + HP * 4;             // bwd: mean per position [128]
+    static constexpr int OFF_G1 = OFF_MU + 128 * 4;            // bwd: rstd g [128][HP]
+    static constexpr int OFF_G0 = OFF_G1 + 128 * HP * 4;       // bwd: g [128][HP]
+    static constexpr int OFF_BAR = OFF_G0 + 128 * HP * 4;      // full[2]
+    static constexpr int OFF_MISC = OFF_BAR + 16;              // abort flag
+    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+};
+
+// 16-byte chunk q (channels 8q .. 8q+7) of row r in a swizzled tile buffer
+__device__ __forceinline__ uint32_t pb_chunk(uint32_t buf, int r, int q) {
+    return buf + (uint32_t)((q >> 3) * 16384 + r * 128 + (((q & 7) ^ (r & 7)) << 4));
+}
+
+// w'[c,h] sits at ((c / 2) HP + h) 2 + c % 2: one 16-byte load gives columns h, h + 1 of
+// the channel pair (c, c + 1) as two float2, the operands of the packed fp32 FMA.
+__device__ __forceinline__ int pb_widx(int c, int h, int HP) { return ((c >> 1) * HP + h) * 2 + (c & 1); }
+
+// Block setup: w' = gamma w (zero-padded to HP columns), its column sums S and the beta
+// projection; initialises the two tile barriers.
+template <int CZ, int HP>
+__device__ __forceinline__ void pb_setup(const PbArgs &a, uint8_t *dsmem, bool with_bb) {
+    using T = PbTraits<CZ, HP>;
+    float *sW = reinterpret_cast<float *>(dsmem + T::OFF_W);
+    float *sS = reinterpret_cast<float *>(dsmem + T::OFF_S);
+    float *sB = reinterpret_cast<float *>(dsmem + T::OFF_BB);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        *reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC) = 0;
+        fence_mbar_init();
+    }
+    for (int e = tid; e < CZ * HP; e += blockDim.x) {
+        const int c = e / HP, h = e % HP;
+        sW[pb_widx(c, h, HP)] = h < a.H ? a.gamma[c] * a.w[c * a.H + h] : 0.f;
+    }
+    __syncthreads();
+    // column sums: warp w takes columns h = w, w + 4, ...; lanes stride over the channels,
+    // then a fixed butterfly
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int h = warp; h < HP; h += 4) {
+        float s = 0.f, bb = 0.f;
+        for (int c = lane; c < CZ; c += 32) {
+            s += sW[pb_widx(c, h, HP)];
+            if (with_bb && h < a.H) bb = fmaf(a.beta[c], a.w[c * a.H + h], bb);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+            bb += __shfl_xor_sync(0xffffffffu, bb, o);
+        }
+        if (lane == 0) {
+            sS[h] = s;
+            sB[h] = bb;
+        }
+    }
+    __syncthreads();
+}
+
+template <int CZ>
+__device__ __forceinline__ void pb_issue(const CUtensorMap *tm, uint32_t dst, uint32_t bar, int tile,
+                                         int nJt) {
+    const int i = tile / nJt, j0 = (tile % nJt) * 128;
+    mbar_arrive_tx(bar, CZ * 128 * 2);
+#pragma unroll
+    for (int hf = 0; hf < CZ / 64; ++hf) tma_load_3d(dst + hf * 16384, tm, bar, hf * 64, j0, i);
+}
+
+// Row r of a tile buffer: its mean (first pass), then in one second pass over the row
+// 1 / sqrt(var + eps) and acc_h = sum_c w'[c,h] (x_c - mean).  The row is read from shared
+// memory, not held in registers, which keeps Cz = 256 spill-free.
+template <int CZ, int HP>
+__device__ __forceinline__ void pb_row_stats(const float *sW, uint32_t buf, int r, float eps, float &mu,
+                                             float &rstd, float (&acc)[HP]) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < CZ / 8; ++q) {
+        const uint4 v = lds128(pb_chunk(buf, r, q));
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s0 += bf16lo(x[e]);
+            s1 += bf16hi(x[e]);
+        }
+    }
+    mu = (s0 + s1) * (1.f / CZ);
+#pragma unroll
+    float2 acc2[HP];   // (even channel, odd channel) partial sums of acc_h
+#pragma unroll
+    for (int h = 0; h < HP; ++h) acc2[h] = make_float2(0.f, 0.f);
+    float2 var2 = make_float2(0.f, 0.f);
+    const float2 nmu = make_float2(-mu, -mu);
+#pragma unroll 1
+    for (int q = 0; q < CZ / 8; ++q) {
+        const uint4 v = lds128(pb_chunk(buf, r, q));
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float4 *wp = reinterpret_cast<const float4 *>(sW + pb_widx(q * 8 + 2 * e, 0, HP));
+            const float2 d = fadd2(make_float2(bf16lo(x[e]), bf16hi(x[e])), nmu);
+            var2 = ffma2(d, d, var2);
+#pragma unroll
+            for (int h2 = 0; h2 < HP / 2; ++h2) {
+                const float4 w4 = wp[h2];   // columns 2 h2, 2 h2 + 1 of channels (c, c + 1)
+                acc2[2 * h2] = ffma2(make_float2(w4.x, w4.y), d, acc2[2 * h2]);
+                acc2[2 * h2 + 1] = ffma2(make_float2(w4.z, w4.w), d, acc2[2 * h2 + 1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < HP; ++h) acc[h] = acc2[h].x + acc2[h].y;
+    rstd = rsqrtf((var2.x + var2.y) * (1.f / CZ) + eps);
+}
+
+template <int CZ, int HP>
+__global__ void __launch_bounds__(128) pba_pair_bias_fwd_kernel(const __grid_constant__ CUtensorMap tmZ,
+                                                                 const PbArgs a) {
+    using T = PbTraits<CZ, HP>;
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    const uint32_t sbase = smem_u32(dsmem);
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) watchdog_fire(SITE_PB_ALIGN);
+        return;
+    }
+    const int tid = threadIdx.x;
+    const float *sW = reinterpret_cast<const float *>(dsmem + T::OFF_W);
+    const float *sB = reinterpret_cast<const float *>(dsmem + T::OFF_BB);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC);
+    const int n_items = (int)blockIdx.x < a.tiles ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
+
+    pb_setup<CZ, HP>(a, dsmem, true);
+    int issued = 0;
+    if (tid == 0) {
+        tma_prefetch_desc(&tmZ);
+        for (; issued < 2 && issued < n_items; ++issued)
+            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, smem_u32(&bars[issued]),
+                         tile_of(issued), a.nJt);
+    }
+    int n = 0;
+    for (; n < n_items; ++n) {
+        const int buf = n & 1;
+        bool ok = mbar_wait(smem_u32(&bars[buf]), (n >> 1) & 1, abort_flag, SITE_PB_FWD | (n << 12));
+        if (!__syncthreads_and(ok)) break;
+        const uint32_t zb = sbase + T::OFF_Z + buf * T::TILE_BYTES;
+        float mu, rstd, acc[HP];
+        pb_row_stats<CZ, HP>(sW, zb, tid, a.eps, mu, rstd, acc);
+        __syncthreads();   // every row has been read: the buffer may be refilled
+        if (tid == 0 && issued < n_items) {
+            pb_issue<CZ>(&tmZ, zb, smem_u32(&bars[buf]), tile_of(issued), a.nJt);
+            ++issued;
+        }
+        const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
+        if (j < a.Nj) {
+            __nv_bfloat16 *dst = a.bias + (long long)i * a.sb1 + j;
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+                if (h < a.H) dst[h * a.sb0] = __float2bfloat16_rn(fmaf(rstd, acc[h], sB[h]));
+        }
+    }
+    if (*abort_flag && tid == 0) {
+        // loads issued for tiles [n, issued) may still be in flight: let them land
+        for (int m = n; m < issued; ++m) mbar_wait_drain(smem_u32(&bars[m & 1]), (m >> 1) & 1);
+    }
+    __syncthreads();
+}
+
+template <int CZ, int HP>
+__global__ void __launch_bounds__(128) pba_pair_bias_bwd_kernel(const __grid_constant__ CUtensorMap tmZ,
+                                                                 const PbArgs a) {
+    using T = PbTraits<CZ, HP>;
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    const uint32_t sbase = smem_u32(dsmem);
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) watchdog_fire(SITE_PB_ALIGN);
+        return;
+    }
+    const int tid = threadIdx.x;
+    const float *sW = reinterpret_cast<const float *>(dsmem + T::OFF_W);
+    const float *sS = reinterpret_cast<const float *>(dsmem + T::OFF_S);
+    float *sMu = reinterpret_cast<float *>(dsmem + T::OFF_MU);
+    float *sG1 = reinterpret_cast<float *>(dsmem + T::OFF_G1);
+    float *sG0 = reinterpret_cast<float *>(dsmem + T::OFF_G0);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC);
+    const int n_items = (int)blockIdx.x < a.tiles ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
+    constexpr int CPT = (CZ + 127) / 128;   // channels per thread in phase 2
+
+    pb_setup<CZ, HP>(a, dsmem, false);
+    float A[CPT][HP];   // this block's sum over positions of xh_c g_h, channels c = tid + 128 k
+    float G = 0.f;      // threads h < HP: sum over positions of g_h
+#pragma unroll
+    for (int k = 0; k < CPT; ++k)
+#pragma unroll
+        for (int h = 0; h < HP; ++h) A[k][h] = 0.f;
+    int issued = 0;
+    if (tid == 0) {
+        tma_prefetch_desc(&tmZ);
+        for (; issued < 2 && issued < n_items; ++issued)
+            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, smem_u32(&bars[issued]),
+                         tile_of(issued), a.nJt);
+    }
+    int n = 0;
+    for (; n < n_items; ++n) {
+        const int buf = n & 1;
+        const uint32_t zb = sbase + T::OFF_Z + buf * T::TILE_BYTES;
+        bool ok = mbar_wait(smem_u32(&bars[buf]), (n >> 1) & 1, abort_flag, SITE_PB_BWD | (n << 12));
+        if (!__syncthreads_and(ok)) break;
+        const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
+        const bool valid = j < a.Nj;
+        // ---- phase 1: thread = position j; dz of its row
+        {
+            float mu, rstd, acc[HP];
+            pb_row_stats<CZ, HP>(sW, zb, tid, a.eps, mu, rstd, acc);
+            float g[HP];
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+                g[h] = (valid && h < a.H) ? a.dbias[h * a.sd0 + (long long)i * a.sd1 + j] : 0.f;
+            float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+                s1 = fmaf(g[h], sS[h], s1);
+                s2 = fmaf(g[h], acc[h], s2);
+            }
+            const float m1 = s1 * (1.f / CZ);             // mean_c dxh
+            const float m2r = s2 * rstd * rstd * (1.f / CZ);   // mean_c(dxh xh) * rstd
+            if (valid) {
+                __nv_bfloat16 *dst = a.dz + (long long)i * a.sz0 + (long long)j * a.sz1;
+#pragma unroll 1
+                for (int q = 0; q < CZ / 8; ++q) {
+                    const uint4 v = lds128(pb_chunk(zb, tid, q));
+                    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 *wp = reinterpret_cast<const float4 *>(sW + pb_widx(q * 8 + 2 * e, 0, HP));
+                        float2 dx = make_float2(0.f, 0.f);   // dxh of the channel pair
+#pragma unroll
+                        for (int h2 = 0; h2 < HP / 2; ++h2) {
+                            const float4 w4 = wp[h2];
+                            dx = ffma2(make_float2(w4.x, w4.y), make_float2(g[2 * h2], g[2 * h2]), dx);
+                            dx = ffma2(make_float2(w4.z, w4.w), make_float2(g[2 * h2 + 1], g[2 * h2 + 1]), dx);
+                        }
+                        const float d0 = bf16lo(x[e]) - mu, d1 = bf16hi(x[e]) - mu;
+                        ow[e] = pack_bf16x2(rstd * (dx.x - m1 - d0 * m2r), rstd * (dx.y - m1 - d1 * m2r));
+                    }
+                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+            }
+            sMu[tid] = mu;
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+                sG1[tid * HP + h] = valid ? rstd * g[h] : 0.f;
+                sG0[tid * HP + h] = g[h];
+            }
+        }
+        __syncthreads();
+        // ---- phase 2: thread = channel; A[c,h] += (z - mean) rstd g over the tile's positions
+#pragma unroll 2
+        for (int p = 0; p < 128; ++p) {
+            const float mu = sMu[p];
+            const float4 *g1 = reinterpret_cast<const float4 *>(sG1 + p * HP);
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int c = tid + 128 * k;
+                if (c < CZ) {
+                    const uint32_t addr = pb_chunk(zb, p, c >> 3) + (c & 7) * 2;
+                    uint16_t raw;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(raw) : "r"(addr));
+                    const float d = __uint_as_float((uint32_t)raw << 16) - mu;
+#pragma unroll
+                    for (int h4 = 0; h4 < HP / 4; ++h4) {
+                        const float4 gg = g1[h4];
+                        A[k][4 * h4] = fmaf(d, gg.x, A[k][4 * h4]);
+                        A[k][4 * h4 + 1] = fmaf(d, gg.y, A[k][4 * h4 + 1]);
+                        A[k][4 * h4 + 2] = fmaf(d, gg.z, A[k][4 * h4 + 2]);
+                        A[k][4 * h4 + 3] = fmaf(d, gg.w, A[k][4 * h4 + 3]);
+                    }
+                }
+            }
+            if (tid < HP) G += sG0[p * HP + tid];
+        }
+        __syncthreads();   // the tile buffer and the per-position arrays are free again
+        if (tid == 0 && issued < n_items) {
+            pb_issue<CZ>(&tmZ, zb, smem_u32(&bars[buf]), tile_of(issued), a.nJt);
+            ++issued;
+        }
+    }
+    const bool aborted = *abort_flag != 0;
+    if (aborted && tid == 0) {
+        for (int m = n; m < issued; ++m) mbar_wait_drain(smem_u32(&bars[m & 1]), (m >> 1) & 1);
+    }
+    if (!aborted) {
+        float *dst = a.part + (long long)blockIdx.x * (CZ * HP + HP);
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            const int c = tid + 128 * k;
+            if (c < CZ) {
+#pragma unroll
+                for (int h = 0; h < HP; ++h) dst[c * HP + h] = A[k][h];
+            }
+        }
+        if (tid < HP) dst[CZ * HP + tid] = G;
+    }
+    __syncthreads();
+}
+
+// Sums of the per-block partials, column by column: block = 32 columns x 16 warps; warp w
+// adds the partials of blocks [w R, (w + 1) R) in order, then warp 0 adds the 16 warp sums
+// in order (bit-stable).  sums[e] for e < Cz * HP + HP: A[c,h] at c * HP + h, then G_h.
+__global__ void __launch_bounds__(512) pba_pair_bias_reduce_kernel(const PbArgs a) {
+    __shared__ float red[16][33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cols = a.Cz * a.hp + a.hp;
+    const int e = blockIdx.x * 32 + lane;
+    const int R = (a.nparts + 15) / 16;
+    const int b_lo = warp * R, b_hi = min(a.nparts, b_lo + R);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    if (e < cols) {
+        const float *src = a.part + e;
+        int b = b_lo;
+        for (; b + 4 <= b_hi; b += 4) {
+            s0 += src[(long long)b * cols];
+            s1 += src[(long long)(b + 1) * cols];
+            s2 += src[(long long)(b + 2) * cols];
+            s3 += src[(long long)(b + 3) * cols];
+        }
+        for (; b < b_hi; ++b) s0 += src[(long long)b * cols];
+    }
+    red[warp][lane] = (s0 + s1) + (s2 + s3);
+    __syncthreads();
+    if (warp == 0 && e < cols) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) t += red[w][lane];
+        a.sums[e] = t;
+    }
+}
+
+// dw[c,h] = gamma_c A[c,h] + beta_c G_h, dgamma_c = sum_h w[c,h] A[c,h], dbeta_c = sum_h w[c,h] G_h
+__global__ void __launch_bounds__(128) pba_pair_bias_param_kernel(const PbArgs a) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= a.Cz) return;
+    const int HP = a.hp;
+    float dg = 0.f, db = 0.f;
+    for (int h = 0; h < a.H; ++h) {
+        const float A = a.sums[c * HP + h], G = a.sums[a.Cz * HP + h];
+        const float wch = a.w[c * a.H + h];
+        a.dw[c * a.H + h] = a.gamma[c] * A + a.beta[c] * G;
+        dg = fmaf(wch, A, dg);
+        db = fmaf(wch, G, db);
+    }
+    a.dgamma[c] = dg;
+    a.dbeta[c] = db;
+}
+
+}  // namespace pba

@@ -91,13 +91,14 @@ __global__ void __launch_bounds__(256) pba_pwa_weights_kernel(const PwaArgs a) {
 template <int CP>
 struct PwaTraits {
     static constexpr int BC = 256 / CP;                        // rows b per CTA (TMEM slots)
-    static constexpr int XS = CP == 64 ? 2 : 4;                // V / dOa tile stages
-    static constexpr int TILE_BYTES = 128 * CP * 2;
-    static constexpr int W_BYTES = 128 * 128 * 2;              // two 64-column halves
-    static constexpr int OFF_W = 0;                            // 1024-byte aligned (SW128)
-    static constexpr int OFF_X = 2 * W_BYTES;
-    static constexpr int NBAR = 2 * 2 + 2 * XS + 2;
-    static constexpr int OFF_BAR = OFF_X + XS * TILE_BYTES;
+    static constexpr int KH = 64;                              // reduction rows per stage
+    static constexpr int XT_BYTES = KH * CP * 2;               // one row b's V / dOa tile
+    static constexpr int W_BYTES = 128 * 64 * 2;               // the stage's 128 x 64 block of w
+    static constexpr int STAGE_BYTES = W_BYTES + BC * XT_BYTES;   // 48 KB at every CP
+    static constexpr int NS = 2;                               // stages
+    static constexpr int OFF_ST = 0;                           // 1024-byte aligned (SW128)
+    static constexpr int NBAR = 2 * NS + 2;
+    static constexpr int OFF_BAR = OFF_ST + NS * STAGE_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
@@ -109,12 +110,18 @@ static_assert(2 * (PwaTraits<64>::SMEM_BYTES + 1024) <= 233472, "smem");
 
 // Warp roles (192 threads): warps 0-3 epilogue (thread = output row = TMEM lane), warp 4
 // TMA producer, warp 5 TMEM allocator and (lane 0) MMA issuer.
+//
+// One MMA covers every row b of the chunk: the chunk's BC tiles of V (or dOa) sit side by
+// side in a stage and form one B operand of N = BC * CP = 256 columns (MN-major, one
+// swizzle atom per row b, LBO = one tile), so each 64-row reduction stage takes four
+// M = 128, N = 256, K = 16 instructions instead of four per row b; the accumulator of row
+// b is TMEM columns [b CP, (b + 1) CP).
 template <int CP, bool DV>
 __global__ void __launch_bounds__(192, 2)
 pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                     const PwaArgs a) {
     using T = PwaTraits<CP>;
-    constexpr int XS = T::XS, BC = T::BC;
+    constexpr int NS = T::NS, BC = T::BC;
     extern __shared__ __align__(1024) uint8_t dsmem[];
     const uint32_t sbase = smem_u32(dsmem);
     if (sbase & 1023u) {
@@ -122,12 +129,10 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
         return;
     }
     uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
-    auto b_w_full = [&](int x) { return smem_u32(&bars[x]); };
-    auto b_w_empty = [&](int x) { return smem_u32(&bars[2 + x]); };
-    auto b_x_full = [&](int st) { return smem_u32(&bars[4 + st]); };
-    auto b_x_empty = [&](int st) { return smem_u32(&bars[4 + XS + st]); };
-    const uint32_t b_done = smem_u32(&bars[4 + 2 * XS]);
-    const uint32_t b_drain = smem_u32(&bars[5 + 2 * XS]);
+    auto b_full = [&](int st) { return smem_u32(&bars[st]); };
+    auto b_empty = [&](int st) { return smem_u32(&bars[NS + st]); };
+    const uint32_t b_done = smem_u32(&bars[2 * NS]);
+    const uint32_t b_drain = smem_u32(&bars[2 * NS + 1]);
     uint32_t *s_tmem_base = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC + 4);
 
@@ -139,17 +144,12 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     const int h = idx / a.nChunks;
     const int t0 = tile * 128, b0 = chunk * BC;
     const int nb = min(BC, a.B - b0);
-    const int nR = a.nT;            // reduction tiles (the problem is square)
-    const int K = nR * nb;          // steps (r, s), k = r * nb + s
+    const int nK = (a.N + T::KH - 1) / T::KH;   // reduction stages (the problem is square)
 
     if (threadIdx.x == 0) {
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(b_w_full(x), 1);
-            mbar_init(b_w_empty(x), 1);
-        }
-        for (int st = 0; st < XS; ++st) {
-            mbar_init(b_x_full(st), 1);
-            mbar_init(b_x_empty(st), 1);
+        for (int st = 0; st < NS; ++st) {
+            mbar_init(b_full(st), 1);
+            mbar_init(b_empty(st), 1);
         }
         mbar_init(b_done, 1);
         mbar_init(b_drain, 1);
@@ -164,7 +164,7 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *s_tmem_base;
-    int w_done = 0, x_done = 0;   // loads issued: W tiles [0, w_done), X tiles [0, x_done)
+    int k_done = 0;   // stages loaded: [0, k_done)
 
     if (warp == 4) {
         // ------------------------------------------------------------------ producer
@@ -172,59 +172,48 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
             tma_prefetch_desc(&tmW);
             tma_prefetch_desc(&tmX);
             bool ok = true;
-            int k = 0;
-            for (int r = 0; r < nR && ok; ++r) {
-                const int wb = r & 1;
-                if (r >= 2) ok = mbar_wait(b_w_empty(wb), ((r >> 1) - 1) & 1, abort_flag, SITE_PWA_PROD | 0x10 | (r << 12));
+            for (int r = 0; r < nK && ok; ++r) {
+                const int st = r % NS;
+                if (r >= NS) ok = mbar_wait(b_empty(st), ((r / NS) - 1) & 1, abort_flag, SITE_PWA_PROD | (r << 12));
                 if (!ok) break;
-                // the 128 x 128 block of w: rows i, columns j (two 64-column boxes)
-                const int wi = DV ? r * 128 : t0, wj = DV ? t0 : r * 128;
-                const uint32_t dst = sbase + T::OFF_W + wb * T::W_BYTES;
-                mbar_arrive_tx(b_w_full(wb), T::W_BYTES);
-                tma_load_3d(dst, &tmW, b_w_full(wb), wj, wi, h);
-                tma_load_3d(dst + 16384, &tmW, b_w_full(wb), wj + 64, wi, h);
-                w_done = r + 1;
-                for (int s = 0; s < nb && ok; ++s, ++k) {
-                    const int st = k % XS, use = k / XS;
-                    if (use >= 1) ok = mbar_wait(b_x_empty(st), (use - 1) & 1, abort_flag, SITE_PWA_PROD | (k << 12));
-                    if (!ok) break;
-                    mbar_arrive_tx(b_x_full(st), T::TILE_BYTES);
-                    tma_load_4d(sbase + T::OFF_X + st * T::TILE_BYTES, &tmX, b_x_full(st), 0, h, r * 128, b0 + s);
-                    x_done = k + 1;
+                const uint32_t sw = sbase + T::OFF_ST + st * T::STAGE_BYTES;
+                mbar_arrive_tx(b_full(st), T::W_BYTES + nb * T::XT_BYTES);
+                if (DV) {
+                    // w rows i = reduction rows [64 r, 64 r + 64), columns j = output rows
+                    tma_load_3d(sw, &tmW, b_full(st), t0, r * 64, h);
+                    tma_load_3d(sw + 8192, &tmW, b_full(st), t0 + 64, r * 64, h);
+                } else {
+                    // w rows i = output rows, columns j = reduction rows [64 r, 64 r + 64)
+                    tma_load_3d(sw, &tmW, b_full(st), r * 64, t0, h);
                 }
+                for (int s = 0; s < nb; ++s)
+                    tma_load_4d(sw + T::W_BYTES + s * T::XT_BYTES, &tmX, b_full(st), 0, h, r * 64, b0 + s);
+                k_done = r + 1;
             }
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            // forward: A = W (rows i, K = j) K-major; dv: A = W^T (rows j, K = i) MN-major;
-            // B = V / dOa tile (K = reduction rows, N = channels) MN-major
-            constexpr uint32_t idesc = idesc_bf16(128, CP, DV, true);
+            // forward: A = w (rows i, K = j) K-major; dv: A = w^T (rows j, K = i) MN-major;
+            // B = the chunk's V / dOa tiles (K = reduction rows, N = rows b x channels)
+            constexpr uint32_t idesc = idesc_bf16(128, 256, DV, true);
             constexpr uint32_t SBO = 8 * T::ROWB;
             bool ok = true;
-            int k = 0;
-            for (int r = 0; r < nR && ok; ++r) {
-                const int wb = r & 1;
-                ok = mbar_wait(b_w_full(wb), (r >> 1) & 1, abort_flag, SITE_PWA_MMA | 0x10 | (r << 12));
+            for (int r = 0; r < nK && ok; ++r) {
+                const int st = r % NS;
+                ok = mbar_wait(b_full(st), (r / NS) & 1, abort_flag, SITE_PWA_MMA | (r << 12));
                 if (!ok) break;
-                const uint32_t sW = sbase + T::OFF_W + wb * T::W_BYTES;
-                for (int s = 0; s < nb && ok; ++s, ++k) {
-                    const int st = k % XS;
-                    ok = mbar_wait(b_x_full(st), (k / XS) & 1, abort_flag, SITE_PWA_MMA | (k << 12));
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sX = sbase + T::OFF_X + st * T::TILE_BYTES;
+                tc_fence_after();
+                const uint32_t sw = sbase + T::OFF_ST + st * T::STAGE_BYTES;
+                const uint32_t sx = sw + T::W_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t adesc =
-                            DV ? sdesc(sW + kk * 2048, 16384, 1024, kSw128)
-                               : sdesc(sW + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-                        umma_ss(tbase + s * CP, adesc, sdesc(sX + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ),
-                                idesc, (r > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(b_x_empty(st));
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t adesc = DV ? sdesc(sw + kk * 2048, 8192, 1024, kSw128)
+                                              : sdesc(sw + kk * 32, 16, 1024, kSw128);
+                    umma_ss(tbase, adesc, sdesc(sx + kk * 16 * T::ROWB, T::XT_BYTES, SBO, T::SWZ), idesc,
+                            (r > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (ok) umma_commit(b_w_empty(wb));
+                umma_commit(b_empty(st));
             }
             if (ok) umma_commit(b_done);
         }
@@ -293,8 +282,7 @@ pba_pwa_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     __syncthreads();
     if (*abort_flag) {
         if (warp == 4 && lane == 0) {
-            for (int rr = max(0, w_done - 2); rr < w_done; ++rr) mbar_wait_drain(b_w_full(rr & 1), (rr >> 1) & 1);
-            for (int kk = max(0, x_done - XS); kk < x_done; ++kk) mbar_wait_drain(b_x_full(kk % XS), (kk / XS) & 1);
+            for (int rr = max(0, k_done - NS); rr < k_done; ++rr) mbar_wait_drain(b_full(rr % NS), (rr / NS) & 1);
         }
         if (warp == 5 && lane == 0) {
             umma_commit(b_drain);

@@ -130,3 +130,30 @@ def make_inputs(cfg: Config, seed: int = 0, with_dout: bool = True,
     if with_dout:
         d["dout"] = normal_bf16(seed, STREAM["dout"], (B, N, H, c))
     return d
+
+
+# ----------------------------------------------------------------------------------------
+# pair-bias projection inputs (pair representation and LayerNorm / projection parameters)
+# ----------------------------------------------------------------------------------------
+
+PAIR_STREAM = {"z": 11, "zshift": 12, "zscale": 13, "gamma": 14, "beta": 15, "w": 16, "dbias": 17}
+CZ_PAIR = 128   # channels of the pair representation in the AlphaFold3 family
+
+
+def make_pair_bias_inputs(Ni: int, Nj: int, Cz: int, H: int, seed: int = 0) -> Dict[str, np.ndarray]:
+    """z as bf16 bits [Ni, Nj, Cz]: N(0, 1) channels with a per-position offset N(0, 1) and
+    scale U(0.5, 2) (so that the normalisation has work to do); gamma ~ 1 + N(0, 0.1^2),
+    beta ~ N(0, 0.1^2), w ~ N(0, 1/Cz) [Cz, H] and dbias ~ N(0, 1) [H, Ni, Nj], all fp32."""
+    def rng(name):
+        return np.random.default_rng([seed, PAIR_STREAM[name]])
+    x = rng("z").standard_normal((Ni, Nj, Cz), dtype=np.float32)
+    shift = rng("zshift").standard_normal((Ni, Nj, 1), dtype=np.float32)
+    scale = rng("zscale").uniform(0.5, 2.0, (Ni, Nj, 1)).astype(np.float32)
+    z = f32_to_bf16_bits(x * scale + shift).reshape(Ni, Nj, Cz)
+    return {
+        "z": z,
+        "gamma": (1.0 + 0.1 * rng("gamma").standard_normal(Cz)).astype(np.float32),
+        "beta": (0.1 * rng("beta").standard_normal(Cz)).astype(np.float32),
+        "w": (rng("w").standard_normal((Cz, H)) / np.sqrt(Cz)).astype(np.float32),
+        "dbias": rng("dbias").standard_normal((H, Ni, Nj), dtype=np.float32),
+    }

@@ -92,3 +92,38 @@ def test_empty_problem_is_a_no_op(pba):
     assert _fwd_status(pba, d, q=None, k=None, v=None, out=None, lse=None)[0] == 0
     d = pba.dims_dense(2, 2, 0, 64, 32)
     assert _fwd_status(pba, d, q=None, k=None, v=None, out=None, lse=None)[0] == 0
+
+
+def _pb_dims(pba, Ni=8, Nj=8, Cz=128, H=4, eps=1e-5):
+    d = pba.PbaPairBiasDims()
+    d.Ni, d.Nj, d.Cz, d.H, d.eps = Ni, Nj, Cz, H, eps
+    d.sz[0], d.sz[1] = Nj * Cz, Cz
+    d.sbias[0], d.sbias[1] = Ni * Nj, Nj
+    d.sdbias[0], d.sdbias[1] = Ni * Nj, Nj
+    return d
+
+
+def _pb_fwd_status(pba, d, z=16, bias=16):
+    st = pba.lib.pba_pair_bias_fwd(z, 16, 16, 16, bias, ctypes.byref(d), None)
+    return st, pba.lib.pba_last_error().decode()
+
+
+def test_pair_bias_host_side_argument_errors(pba):
+    assert _pb_fwd_status(pba, _pb_dims(pba, Cz=100))[0] == 2          # Cz not supported
+    assert _pb_fwd_status(pba, _pb_dims(pba, H=17))[0] == 2            # too many heads
+    assert _pb_fwd_status(pba, _pb_dims(pba, eps=0.0))[0] == 1         # eps must be > 0
+    assert _pb_fwd_status(pba, _pb_dims(pba, eps=float("nan")))[0] == 1
+    assert _pb_fwd_status(pba, _pb_dims(pba, Ni=-1))[0] == 1
+    d = _pb_dims(pba)
+    d.sz[1] = 100                                                        # not a multiple of 8
+    st, msg = _pb_fwd_status(pba, d)
+    assert st == 1 and "stride" in msg
+    assert _pb_fwd_status(pba, _pb_dims(pba), z=None)[0] == 1
+    assert _pb_fwd_status(pba, _pb_dims(pba), z=24)[0] == 1             # misaligned z
+    assert _pb_fwd_status(pba, _pb_dims(pba, Ni=0), z=None, bias=None)[0] == 0   # empty: no-op
+    d = _pb_dims(pba)
+    need = pba.lib.pba_pair_bias_bwd_workspace_size(ctypes.byref(d))
+    assert need > 0
+    st = pba.lib.pba_pair_bias_bwd(16, 16, 16, 16, 16, 16, 16, 16, 16, 256, need - 4, ctypes.byref(d), None)
+    assert st == 5                                                       # workspace too small
+    assert pba.lib.pba_pair_bias_bwd_workspace_size(ctypes.byref(_pb_dims(pba, Cz=100))) == 0
