@@ -231,6 +231,23 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def max_over_ranks(pg, values, device="cuda"):
+    """Every rank's timings -> their maximum over the ranks (the slowest replica sets the
+    job's time); `pg` is torch.distributed or None for one process."""
+    if pg is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(world, units_per_step, steps, elapsed_ms):
+    """Whole-job units per second: every replica processed `steps` steps of `units_per_step`
+    within the slowest rank's `elapsed_ms`."""
+    return world * units_per_step * steps / (elapsed_ms / 1e3)
+
+
 def run_ours(args, cfg):
     import torch
     rank, world, local = dist_env()
@@ -346,15 +363,12 @@ def run_ours(args, cfg):
     e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
     pba.pba_device_status()
 
-    if pg:
-        t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+    elapsed_ms, e2e_ms = max_over_ranks(pg, [elapsed_ms, e2e_ms])
 
     w = work(cfg)
     step_flops = w["fwd_flops"] + w["bwd_flops"]
-    value = world * step_flops * K / (elapsed_ms / 1e3) / 1e12
-    e2e_value = world * step_flops * K2 / (e2e_ms / 1e3) / 1e12
+    value = job_throughput(world, step_flops, K, elapsed_ms) / 1e12
+    e2e_value = job_throughput(world, step_flops, K2, e2e_ms) / 1e12
 
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
