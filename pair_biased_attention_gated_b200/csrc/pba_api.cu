@@ -456,7 +456,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         const long long grid = items < num_sms() ? items : num_sms();
         {
             ProfScope ps(K_BWD_MAIN, s);
-            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 352, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, tdq, a);
+            pba::pba_bwd_main_kernel<CP><<<(unsigned)grid, 512, MT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, tdq, a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {

@@ -51,7 +51,7 @@ struct BwdArgs {
 };
 
 enum : unsigned {
-    SITE_BWD_PROD = 0x201, SITE_BWD_MMA = 0x202, SITE_BWD_EW = 0x203,
+    SITE_BWD_PROD = 0x201, SITE_BWD_MMA = 0x202, SITE_BWD_EW = 0x203, SITE_BWD_EPI = 0x204,
     SITE_DB_PROD = 0x301, SITE_DB_MMA = 0x302, SITE_DB_EW = 0x303
 };
 
@@ -156,32 +156,36 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
     }
 }
 
-// P and dS of 64 keys (one half of a 128-key tile) for one query row, in 32-key chunks.
+// P and dS of 64 keys (one half of a 128-key tile) for one query row, in KC-key chunks.
 //   tS, tdP: this lane's S and dP columns in TMEM; bias_row: the row's 64 bf16 bias values
 //   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
 //   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
 //   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
 // For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS.
-template <typename Use>
+template <int KC, typename Use>
 __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
                                           bool has_bias, uint32_t mw0, uint32_t mw1, bool full,
                                           float sl2e, float lse2, float D, Use &&use) {
+    // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers; the main kernel
+    // uses 16 to stay within the 128 registers a thread has at 512 threads per CTA
+    static_assert(KC == 16 || KC == 32, "chunk");
     const float2 sl2 = make_float2(sl2e, sl2e), l2e2 = make_float2(kLog2eB, kLog2eB);
     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        uint32_t r[64];   // S of keys 32 q .. 32 q + 31 in r[0..31], dP in r[32..63]
-        tmem_ld32x2(tS + q * 32, tdP + q * 32, r);
-        const uint32_t mw = q == 0 ? mw0 : mw1;
+    for (int q = 0; q < 64 / KC; ++q) {
+        uint32_t r[2 * KC];   // S of keys KC q .. KC q + KC - 1 in r[0, KC), dP in r[KC, 2 KC)
+        if constexpr (KC == 32) tmem_ld32x2(tS + q * KC, tdP + q * KC, r);
+        else tmem_ld16x2(tS + q * KC, tdP + q * KC, r);
+        const uint32_t mw = ((q * KC) < 32 ? mw0 : mw1) >> ((q * KC) & 31);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int c8 = q * 4 + c4;
+        for (int c2 = 0; c2 < KC / 8; ++c2) {
+            const int c8 = q * (KC / 8) + c2;
             uint4 bw = make_uint4(0, 0, 0, 0);
             if (has_bias) bw = lds128(bias_row + ((c8 ^ (row & 7)) << 4));
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int k = c4 * 8 + 2 * e;   // key within the chunk
+                const int k = c2 * 8 + 2 * e;   // key within the chunk
                 float2 u = ffma2(make_float2(bf16lo(bb[e]), bf16hi(bb[e])), l2e2, nl2);
                 u = ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, u);
                 float2 p = make_float2(ex2(u.x), ex2(u.y));
@@ -189,8 +193,8 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
                     p.x = ((mw >> k) & 1u) ? p.x : 0.f;
                     p.y = ((mw >> (k + 1)) & 1u) ? p.y : 0.f;
                 }
-                const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(r[32 + k]), __uint_as_float(r[33 + k])), nD2));
-                use(q * 32 + k, p, ds);
+                const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(r[KC + k]), __uint_as_float(r[KC + 1 + k])), nD2));
+                use(q * KC + k, p, ds);
             }
         }
     }
@@ -203,8 +207,9 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
 // blockIdx.x + gridDim.x, ...; an item's steps are its query tiles.  The step pipeline
 // (S/dP -> P/dS -> dV, dK, dQ) runs on across item boundaries: the next item's K/V tiles
 // load into the other stage while the current item finishes, and dK/dV accumulate in one
-// of two TMEM buffers, so an item's dK/dV epilogue (written by the element-wise warps right
-// after the next item's first step) overlaps the next item's MMAs.
+// of two TMEM buffers, so an item's dK/dV epilogue overlaps the next item's MMAs.  The dQ
+// flushes and the dK/dV epilogues belong to a warpgroup of their own, so the element-wise
+// warps only turn S/dP into P/dS.
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct BwdTraits {
@@ -237,13 +242,14 @@ struct BwdTraits {
 };
 static_assert(BwdTraits<64>::SMEM_BYTES <= 232448 && BwdTraits<32>::SMEM_BYTES <= 232448, "smem");
 
-// Warp roles (352 threads): warps 0-7 element-wise (two warpgroups, one 64-key half each),
-// warp 8 TMA producer, warp 9 TMEM allocator and (lane 0) issuer of the dV, dK, dQ
-// products, warp 10 (lane 0) issuer of S = Q K^T and dP = dOa V^T.  A tcgen05.mma issue
+// Warp roles (512 threads, four warpgroups): warps 0-7 element-wise (two warpgroups, one
+// 64-key half each), warp 8 TMA producer, warp 9 TMEM allocator and (lane 0) issuer of the
+// dV, dK, dQ products, warp 10 (lane 0) issuer of S = Q K^T and dP = dOa V^T, warp 11 idle,
+// warps 12-15 the dQ flushes and dK/dV epilogues (thread = TMEM lane).  A tcgen05.mma issue
 // holds its thread about as long as the MMA runs, so S/dP of the next step do not wait
-// behind this step's 24 products.
+// behind this step's 24 products.  Every thread has 128 registers (512 threads on one SM).
 template <int CP>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(512, 1)
 pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmBias, const __grid_constant__ CUtensorMap tmDQ,
@@ -303,7 +309,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(b_drain, 2);   // one commit from each issuer
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_dq_full(x), 1);
-            mbar_init(b_dq_free(x), 256);
+            mbar_init(b_dq_free(x), 128);
         }
         for (int x = 0; x < QS; ++x) {
             mbar_init(b_q_full(x), 1);
@@ -319,9 +325,9 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         for (int x = 0; x < DKB; ++x) {
             mbar_init(b_dkv_full(x), 1);
-            mbar_init(b_dkv_free(x), 256);
+            mbar_init(b_dkv_free(x), 128);
         }
-        mbar_init(b_stg_full, 256);
+        mbar_init(b_stg_full, 128);
         mbar_init(b_stg_free, 1);
         s_abort = 0;
         fence_mbar_init();
@@ -481,7 +487,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------------------ elementwise
         // warpgroup e owns keys [64 e, 64 e + 64) of the tile for all 128 query rows
         const int e = warp >> 2;
@@ -489,105 +495,11 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const float sl2e = a.scale * kLog2eB;
         bool ok = true;
-        // items of the current and the previous step (decoded once per item)
-        Item cur = {0, 0, 0}, last = {0, 0, 0};
-        auto flush_dq = [&](int t, const Item &it) -> bool {
-            // dQ(t): this thread's query row, channels [e CP/2, (e+1) CP/2), added to dqacc
-            bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EW | 0x10 | (t << 12));
-            okf = __all_sync(0xffffffffu, okf);
-            if (!okf) return false;
-            tc_fence_after();
-            uint32_t r[CP / 2];
-            const uint32_t taddr = tbase + T::T_DQ + (t & 1) * CP + e * (CP / 2) + lane_off;
-            if constexpr (CP / 2 == 8) {
-                uint32_t r16[16];
-                tmem_ld16(taddr, r16);  // reads 16 columns; only the first 8 are this half's
-#pragma unroll
-                for (int c = 0; c < 8; ++c) r[c] = r16[c];
-            } else if constexpr (CP / 2 == 16) {
-                tmem_ld16(taddr, r);
-            } else {
-                tmem_ld32(taddr, r);
-            }
-            tc_fence_before();
-            mbar_arrive(b_dq_free(t & 1));
-            const int i = (t % nI) * 128 + row;
-            if constexpr (T::DQ_TMA) {
-                // the staging tile of the previous flush has been read by its TMA reduction:
-                // thread 0, which issued it, checks that here (a step later, so it no longer
-                // waits) and releases the tile
-                if (t > 0) {
-                    if (threadIdx.x == 0) {
-                        bulk_wait_read_all();
-                        mbar_arrive(b_stg_free);
-                    }
-                    okf = mbar_wait(b_stg_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x70 | (t << 12));
-                    okf = __all_sync(0xffffffffu, okf);
-                    if (!okf) return false;
-                }
-                // this thread's 16 channels = 16-byte chunks 4 e .. 4 e + 3 of row `row`
-                const uint32_t srow = sbase + T::OFF_DQS + row * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    sts128(srow + (((e * 4 + q4) ^ (row & 7)) << 4),
-                           make_uint4(r[q4 * 4], r[q4 * 4 + 1], r[q4 * 4 + 2], r[q4 * 4 + 3]));
-                fence_proxy_async();
-                mbar_arrive(b_stg_full);
-                if (threadIdx.x == 0) {
-                    // rows >= Nq and channels >= C fall outside the map and are skipped
-                    okf = mbar_wait(b_stg_full, t & 1, abort_flag, SITE_BWD_EW | 0x80 | (t << 12));
-                    if (!okf) return false;
-                    tma_reduce_add_4d(&tmDQ, sbase + T::OFF_DQS, 0, it.h, (t % nI) * 128, it.b);
-                    bulk_commit();
-                }
-            } else if (i < a.Nq) {
-                float *dst = a.dqacc + (((long long)it.b * a.Nq + i) * a.H + it.h) * a.C;
-#pragma unroll
-                for (int c4 = 0; c4 < CP / 8; ++c4) {
-                    const int c = e * (CP / 2) + c4 * 4;
-                    if (c < a.C)
-                        red_add_v4(dst + c, __uint_as_float(r[c4 * 4]), __uint_as_float(r[c4 * 4 + 1]),
-                                   __uint_as_float(r[c4 * 4 + 2]), __uint_as_float(r[c4 * 4 + 3]));
-                }
-            }
-            return true;
-        };
-        auto epilogue = [&](int m, const Item &it) -> bool {
-            // dK/dV of item m: warpgroup 0 writes dK (times scale), warpgroup 1 dV; lane = key
-            bool oke = mbar_wait(b_dkv_full(m % DKB), (m / DKB) & 1, abort_flag, SITE_BWD_EW | 0x20 | (m << 12));
-            oke = __all_sync(0xffffffffu, oke);
-            if (!oke) return false;
-            tc_fence_after();
-            uint32_t r[CP];
-            tmem_ld_cols<CP>(tbase + T::T_DK + (m % DKB) * 2 * CP + e * CP + lane_off, r);
-            tc_fence_before();
-            mbar_arrive(b_dkv_free(m % DKB));
-            const int j = it.jt * 128 + row;
-            if (j < a.Nk) {
-                __nv_bfloat16 *dst = e == 0 ? a.dk + it.b * a.sk0 + (long long)j * a.sk1 + it.h * a.sk2
-                                            : a.dv + it.b * a.sv0 + (long long)j * a.sv1 + it.h * a.sv2;
-                const float mul = e == 0 ? a.scale : 1.f;
-#pragma unroll
-                for (int c8 = 0; c8 < CP / 8; ++c8) {
-                    if (c8 * 8 < a.C) {
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            ow[q] = pack_bf16x2(__uint_as_float(r[c8 * 8 + 2 * q]) * mul,
-                                                __uint_as_float(r[c8 * 8 + 2 * q + 1]) * mul);
-                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
-                }
-            }
-            return true;
-        };
         uint32_t mw0 = 0, mw1 = 0;
         bool full = true;
         for (int t = 0; t < Tn && ok; ++t) {
             const int m = t / nI, i = t % nI, st = t % QS, bs = t % BS;
             if (i == 0) {
-                last = cur;
-                cur = item(m);
                 // this item's mask words come with its K/V tiles
                 ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
                 ok = __all_sync(0xffffffffu, ok);
@@ -606,7 +518,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
             uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
             const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
-            p_ds_half(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
+            p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
                       row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
                       [&](int c, float2 p, float2 ds) {
                           pp[c >> 1] = pack_bf16x2(p.x, p.y);
@@ -633,12 +545,132 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // generic-proxy writes -> visible to the tensor core's async proxy
             fence_proxy_async();
             mbar_arrive(b_ps_full);
-            if (t > 0) ok = flush_dq(t - 1, i == 0 ? last : cur);
-            if (ok && i == 0 && m > 0) ok = epilogue(m - 1, last);
         }
-        if (ok && Tn > 0) ok = flush_dq(Tn - 1, cur);
-        if (ok && M > 0) ok = epilogue(M - 1, cur);
-        if (T::DQ_TMA && threadIdx.x == 0) bulk_wait_all();   // its TMA reductions are done
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------------ dQ and dK/dV
+        // thread = TMEM lane = query row (dQ) or key row (dK/dV); the warpgroup's first
+        // thread issues the dQ tile's TMA reductions
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
+        const bool issuer = threadIdx.x == 384;
+        bool ok = true;
+        auto flush_dq = [&](int t, const Item &it) -> bool {
+            // dQ(t): this thread's query row, all CP channels, added to dqacc
+            bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EPI | 0x10 | (t << 12));
+            okf = __all_sync(0xffffffffu, okf);
+            if (!okf) return false;
+            tc_fence_after();
+            const uint32_t tq = tbase + T::T_DQ + (t & 1) * CP + lane_off;
+            const int i = (t % nI) * 128 + row;
+            if constexpr (T::DQ_TMA) {
+                uint32_t r[32];
+                tmem_ld32(tq, r);
+                tc_fence_before();
+                mbar_arrive(b_dq_free(t & 1));
+                // the staging tile of the previous flush has been read by its TMA reduction:
+                // the thread that issued it checks that here (a step later, so it no longer
+                // waits) and releases the tile
+                if (t > 0) {
+                    if (issuer) {
+                        bulk_wait_read_all();
+                        mbar_arrive(b_stg_free);
+                    }
+                    okf = mbar_wait(b_stg_free, (t - 1) & 1, abort_flag, SITE_BWD_EPI | 0x70 | (t << 12));
+                    okf = __all_sync(0xffffffffu, okf);
+                    if (!okf) return false;
+                }
+                // row `row` of the 128 x 32 fp32 staging tile: eight 16-byte chunks, swizzled
+                const uint32_t srow = sbase + T::OFF_DQS + row * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4)
+                    sts128(srow + ((q4 ^ (row & 7)) << 4),
+                           make_uint4(r[q4 * 4], r[q4 * 4 + 1], r[q4 * 4 + 2], r[q4 * 4 + 3]));
+                fence_proxy_async();
+                mbar_arrive(b_stg_full);
+                bool oki = true;
+                if (issuer) {
+                    // rows >= Nq and channels >= C fall outside the map and are skipped
+                    oki = mbar_wait(b_stg_full, t & 1, abort_flag, SITE_BWD_EPI | 0x80 | (t << 12));
+                    if (oki) {
+                        tma_reduce_add_4d(&tmDQ, sbase + T::OFF_DQS, 0, it.h, (t % nI) * 128, it.b);
+                        bulk_commit();
+                    }
+                }
+                if (!__all_sync(0xffffffffu, oki)) return false;   // the issuer's warp leaves together
+            } else {
+                float *dst = a.dqacc + (((long long)it.b * a.Nq + i) * a.H + it.h) * a.C;
+#pragma unroll
+                for (int h32 = 0; h32 < (CP + 31) / 32; ++h32) {
+                    constexpr int W = CP < 32 ? CP : 32;   // columns per TMEM load
+                    uint32_t r[W];
+                    if constexpr (W == 16) tmem_ld16(tq, r);
+                    else tmem_ld32(tq + h32 * 32, r);
+                    if (h32 == (CP + 31) / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(b_dq_free(t & 1));
+                    }
+                    if (i < a.Nq) {
+#pragma unroll
+                        for (int c4 = 0; c4 < W / 4; ++c4) {
+                            const int c = h32 * 32 + c4 * 4;
+                            if (c < a.C)
+                                red_add_v4(dst + c, __uint_as_float(r[c4 * 4]), __uint_as_float(r[c4 * 4 + 1]),
+                                           __uint_as_float(r[c4 * 4 + 2]), __uint_as_float(r[c4 * 4 + 3]));
+                        }
+                    }
+                }
+            }
+            return true;
+        };
+        auto epilogue = [&](int m, const Item &it) -> bool {
+            // dK (times scale) and dV of item m; lane = key row
+            bool oke = mbar_wait(b_dkv_full(m % DKB), (m / DKB) & 1, abort_flag, SITE_BWD_EPI | 0x20 | (m << 12));
+            oke = __all_sync(0xffffffffu, oke);
+            if (!oke) return false;
+            tc_fence_after();
+            const int j = it.jt * 128 + row;
+            const uint32_t tdk = tbase + T::T_DK + (m % DKB) * 2 * CP + lane_off;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                __nv_bfloat16 *dst = e == 0 ? a.dk + it.b * a.sk0 + (long long)j * a.sk1 + it.h * a.sk2
+                                            : a.dv + it.b * a.sv0 + (long long)j * a.sv1 + it.h * a.sv2;
+                const float mul = e == 0 ? a.scale : 1.f;
+#pragma unroll
+                for (int h32 = 0; h32 < (CP + 31) / 32; ++h32) {
+                    constexpr int W = CP < 32 ? CP : 32;
+                    uint32_t r[W];
+                    if constexpr (W == 16) tmem_ld16(tdk + e * CP, r);
+                    else tmem_ld32(tdk + e * CP + h32 * 32, r);
+                    if (e == 1 && h32 == (CP + 31) / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(b_dkv_free(m % DKB));
+                    }
+                    if (j < a.Nk) {
+#pragma unroll
+                        for (int c8 = 0; c8 < W / 8; ++c8) {
+                            const int c = h32 * 32 + c8 * 8;
+                            if (c < a.C) {
+                                uint32_t ow[4];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    ow[q] = pack_bf16x2(__uint_as_float(r[c8 * 8 + 2 * q]) * mul,
+                                                        __uint_as_float(r[c8 * 8 + 2 * q + 1]) * mul);
+                                *reinterpret_cast<uint4 *>(dst + c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            }
+                        }
+                    }
+                }
+            }
+            return true;
+        };
+        Item cur = {0, 0, 0};
+        for (int t = 0; t < Tn && ok; ++t) {
+            const int m = t / nI, i = t % nI;
+            if (i == 0) cur = item(m);
+            ok = flush_dq(t, cur);
+            if (ok && i == nI - 1) ok = epilogue(m, cur);
+        }
+        if (T::DQ_TMA && issuer) bulk_wait_all();   // its TMA reductions are done
     }
 
     tc_fence_before();
@@ -832,7 +864,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
             const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
             const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
-            p_ds_half(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
+            p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
                       bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
                       rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
             tc_fence_before();

@@ -343,6 +343,18 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
         : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
         : "memory");
 }
+// Two 16-column loads from two addresses with a single wait: r[0..15] from a0, r[16..31] from a1.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t a0, uint32_t a1, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : PBA_R32(r, 0)
+        : "r"(a0), "r"(a1)
+        : "memory");
+}
 // Two 32-column loads from two addresses with a single wait: r[0..31] from a0, r[32..63] from a1.
 __device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t a1, uint32_t (&r)[64]) {
     asm volatile(

@@ -145,7 +145,6 @@ __device__ __forceinline__ void pb_row_stats(const float *sW, uint32_t buf, int 
         }
     }
     mu = (s0 + s1) * (1.f / CZ);
-#pragma unroll
     float2 acc2[HP];   // (even channel, odd channel) partial sums of acc_h
 #pragma unroll
     for (int h = 0; h < HP; ++h) acc2[h] = make_float2(0.f, 0.f);
