@@ -42,12 +42,25 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # algorithmic work (unmasked keys only; c is the true head dim)
 # ---------------------------------------------------------------------------------------
 
+def oracle_inputs(cfg: pi.Config, d):
+    """The oracle's fp64 view of one draw; under a tile window the bias carries -inf at the
+    pairs the window excludes, which is what local attention computes."""
+    f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+    if cfg.window >= 0 and "bias" in f:
+        f["bias"] = np.where(pi.window_pair_mask(cfg.N, cfg.N, cfg.window)[None], f["bias"], -np.inf)
+    return f
+
+
 def work(cfg: pi.Config, B=None):
+    """Algorithmic flops and bytes: products over attended (query, key) pairs only (unmasked
+    keys, and under a tile window only the pairs it keeps); the bias read where it is used."""
     B = cfg.B if B is None else B
-    H, N, c, nv = cfg.H, cfg.N, cfg.c, cfg.n_valid_keys
-    unit = B * H * N * nv * c
+    H, N, c = cfg.H, cfg.N, cfg.c
+    pairs = pi.window_pair_mask(N, N, cfg.window)
+    attended = int((pairs & (cfg.keep()[None, :] != 0)).sum())   # sum over rows of attended keys
+    unit = B * H * attended * c
     e = B * N * H * c                       # elements of one [B, N, H, c] tensor
-    bias_b = H * N * N * 2
+    bias_b = H * int(pairs.sum()) * 2
     lse_b = B * H * N * 4
     mask_b = N
     f = {
@@ -192,7 +205,7 @@ def time_oracle(cfg: pi.Config, target_s: float, seed: int = 0, max_rows=None):
 
     def run(Bs):
         d = pi.make_inputs(cfg, seed=seed, B=Bs)
-        f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+        f = oracle_inputs(cfg, d)
         t0 = time.perf_counter()
         oracle.fwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"))
         oracle.bwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"), f["dout"])
@@ -294,8 +307,8 @@ def run_ours(args, cfg):
     stream = torch.cuda.current_stream()
 
     def step():
-        pba.pba_fwd(q, kk, v, bias, keep, g, out, lse)
-        pba.pba_bwd(q, kk, v, bias, keep, g, out, lse, dout, dq, dk, dv, db, dg, ws)
+        pba.pba_fwd(q, kk, v, bias, keep, g, out, lse, window=cfg.window)
+        pba.pba_bwd(q, kk, v, bias, keep, g, out, lse, dout, dq, dk, dv, db, dg, ws, window=cfg.window)
 
     def l2_flush(i):
         flush.fill_(i & 0xFF)
@@ -445,7 +458,7 @@ def run_reference(args, cfg):
     import oracle
     import numpy as np  # noqa: F401
     d = pi.make_inputs(cfg, seed=args.seed, B=Bs)
-    f = {k: (pi.bf16_bits_to_f64(v) if k != "keep" else v) for k, v in d.items()}
+    f = oracle_inputs(cfg, d)
 
     def step():
         oracle.fwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f.get("g"))

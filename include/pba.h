@@ -111,6 +111,30 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                    void *stream);
 
 /*
+ * Block-sparse local attention (the sequence-local atom attention of the AlphaFold3 family,
+ * "AlphaFold3 open-source implementation" page, Model Efficiency section, which names the
+ * atom attention encoder and decoder among the attention-with-pair-bias modules): query
+ * tile t (rows 128 t .. 128 t + 127) attends only the key tiles [t - window, t + window]
+ * (clamped to the problem); every other key is masked for its rows and never read.  A
+ * finer local pattern inside the visited tiles is expressed through the bias (-inf) or the
+ * key mask.  The results equal pba_fwd / pba_bwd with those keys masked; dbias is 0 for the
+ * pairs outside the band.  window < 0 is pba_fwd / pba_bwd.  Every query tile must keep a
+ * key tile and every key tile a query tile (ceil(Nq/128) <= ceil(Nk/128) + window and the
+ * reverse), else PBA_ERR_UNSUPPORTED.  Other arguments, layouts and errors as pba_fwd /
+ * pba_bwd; the workspace is pba_bwd_workspace_size(dims).
+ */
+pba_status pba_fwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                         pba_bf16 *out, float *lse, const pba_dims *dims, int window,
+                         void *stream);
+pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                         const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                         pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                         void *workspace, size_t workspace_bytes, const pba_dims *dims,
+                         int window, void *stream);
+
+/*
  * Backward pass for callers that cannot allocate device memory.  The paper has no
  * counterpart: this entry point exists for users of the library, not for the method.
  * Some callers have no way to obtain scratch memory: a plugin running inside another

@@ -48,6 +48,10 @@ lib.pba_bwd_workspace_size.restype = ctypes.c_size_t
 lib.pba_bwd.argtypes = [_vp] * 14 + [_vp, ctypes.c_size_t, ctypes.POINTER(PbaDims), _vp]
 lib.pba_bwd.restype = ctypes.c_int
 lib.pba_bwd_noalloc.argtypes = [_vp] * 14 + [ctypes.POINTER(PbaDims), _vp]
+lib.pba_fwd_local.argtypes = [_vp] * 8 + [ctypes.POINTER(PbaDims), ctypes.c_int, _vp]
+lib.pba_fwd_local.restype = ctypes.c_int
+lib.pba_bwd_local.argtypes = [_vp] * 14 + [_vp, ctypes.c_size_t, ctypes.POINTER(PbaDims), ctypes.c_int, _vp]
+lib.pba_bwd_local.restype = ctypes.c_int
 lib.pba_bwd_noalloc.restype = ctypes.c_int
 lib.pba_pwa_fwd_workspace_size.argtypes = [ctypes.POINTER(PbaDims)]
 lib.pba_pwa_fwd_workspace_size.restype = ctypes.c_size_t
@@ -152,11 +156,14 @@ def dims_dense(B, H, Nq, Nk, C, scale=0.0) -> PbaDims:
     return d
 
 
-def pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale: float = 0.0, stream=None) -> None:
-    """Forward pass into preallocated `out` (bf16, like q) and `lse` (fp32 [B,H,Nq])."""
+def pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale: float = 0.0, stream=None,
+            window: int = -1) -> None:
+    """Forward pass into preallocated `out` (bf16, like q) and `lse` (fp32 [B,H,Nq]).
+    `window` >= 0: block-sparse local attention, query tile t (128 rows) attends key tiles
+    [t - window, t + window] only (pba_fwd_local)."""
     d = make_dims(q, k, v, gate, out, bias, key_mask, scale)
-    _check(lib.pba_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
-                       _ptr(out), _ptr(lse), ctypes.byref(d), _stream(stream)))
+    _check(lib.pba_fwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
+                             _ptr(out), _ptr(lse), ctypes.byref(d), int(window), _stream(stream)))
 
 
 def pba_bwd_workspace_size(dims: PbaDims) -> int:
@@ -164,7 +171,7 @@ def pba_bwd_workspace_size(dims: PbaDims) -> int:
 
 
 def pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
-            workspace, scale: float = 0.0, stream=None) -> None:
+            workspace, scale: float = 0.0, stream=None, window: int = -1) -> None:
     """Backward pass into preallocated dq, dk, dv (like q/k/v), dbias (fp32 [H,Nq,Nk] or
     None), dgate (like gate, or None).  `workspace`: a uint8 CUDA tensor of at least
     pba_bwd_workspace_size(dims) bytes."""
@@ -174,10 +181,10 @@ def pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dg
         if a is not None and b is not None and a.stride() != b.stride():
             raise ValueError("%s must have the same strides as its forward tensor" % name)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.pba_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
-                       _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                       _ptr(dbias), _ptr(dgate), _ptr(workspace), ws_bytes, ctypes.byref(d),
-                       _stream(stream)))
+    _check(lib.pba_bwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
+                             _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(dbias), _ptr(dgate), _ptr(workspace), ws_bytes, ctypes.byref(d),
+                             int(window), _stream(stream)))
 
 
 def pba_bwd_noalloc(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
@@ -235,17 +242,17 @@ def pba_device_status(stream=None) -> None:
 # ---------------------------------------------------------------------------------------
 
 def attention_fwd(q, k, v, bias=None, key_mask=None, gate=None, scale: float = 0.0,
-                  stream=None):
+                  stream=None, window: int = -1):
     import torch
     B, Nq, H, C = q.shape
     out = torch.empty_like(q)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale, stream)
+    pba_fwd(q, k, v, bias, key_mask, gate, out, lse, scale, stream, window)
     return out, lse
 
 
 def attention_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, scale: float = 0.0,
-                  want_dbias: bool = True, stream=None):
+                  want_dbias: bool = True, stream=None, window: int = -1):
     import torch
     B, Nq, H, C = q.shape
     Nk = k.shape[1]
@@ -256,7 +263,7 @@ def attention_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, scale: float = 
     d = make_dims(q, k, v, gate, out, bias, key_mask, scale, dout=dout)
     ws = torch.empty(max(pba_bwd_workspace_size(d), 1), dtype=torch.uint8, device=q.device)
     pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, ws,
-            scale, stream)
+            scale, stream, window)
     return dq, dk, dv, dgate, dbias
 
 

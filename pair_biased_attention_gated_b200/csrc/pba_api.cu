@@ -220,6 +220,18 @@ float eff_scale(const pba_dims *d) {
     return d->scale > 0.f ? d->scale : 1.0f / std::sqrt((float)d->C);
 }
 
+// Local attention: query tile t visits key tiles [t - window, t + window]; every query tile
+// must keep at least one key tile and every key tile at least one query tile (window < 0:
+// dense, always fine).
+pba_status check_window(const pba_dims *d, int window) {
+    if (window < 0) return PBA_OK;
+    const long long nI = (d->Nq + 127) / 128, nJ = (d->Nk + 127) / 128;
+    if (d->Nq > 0 && d->Nk > 0 && (nI > nJ + window || nJ > nI + window))
+        return fail(PBA_ERR_UNSUPPORTED, "window %d leaves a query or key tile with no partner "
+                                         "(%lld query tiles, %lld key tiles)", window, nI, nJ);
+    return PBA_OK;
+}
+
 template <typename K>
 pba_status set_smem(K kernel, int bytes) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -232,7 +244,7 @@ long long num_sms();
 template <int CP>
 pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                       const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
-                      pba_bf16 *out, float *lse, const pba_dims *d, cudaStream_t stream) {
+                      pba_bf16 *out, float *lse, const pba_dims *d, int win, cudaStream_t stream) {
     using T = pba::FwdTraits<CP>;
     CUtensorMap tq, tk, tv, tb;
     pba_status st;
@@ -261,6 +273,7 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.so0 = d->so[0]; a.so1 = d->so[1]; a.so2 = d->so[2];
     a.lse = lse;
     a.skip_step = g_debug_skip_step;
+    a.win = win;
     if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
     // two CTAs per SM need (almost) all of the unified L1 / shared memory as shared memory
     cudaError_t ce = cudaFuncSetAttribute(pba::pba_fwd_kernel<CP>,
@@ -383,7 +396,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                       const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
                       const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
                       pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
-                      void *ws, const BwdPlan &pl, const pba_dims *d, cudaStream_t s) {
+                      void *ws, const BwdPlan &pl, const pba_dims *d, int win, cudaStream_t s) {
     using MT = pba::BwdTraits<CP>;
     using DT = pba::DbTraits<CP>;
     uint8_t *w = static_cast<uint8_t *>(ws);
@@ -392,6 +405,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.B = d->B; a.H = d->H; a.Nq = d->Nq; a.Nk = d->Nk; a.C = d->C;
     a.nI = pl.nI; a.nJ = pl.nJ; a.NqPad = pl.NqPad; a.NkPad = pl.NkPad;
     a.splits = pl.splits; a.rows_per_split = pl.rows_per_split;
+    a.win = win;
     a.scale = eff_scale(d);
     a.has_bias = bias != nullptr;
     a.has_gate = gate != nullptr;
@@ -859,9 +873,16 @@ void pba_dims_dense(pba_dims *d, int32_t B, int32_t H, int32_t Nq, int32_t Nk, i
 pba_status pba_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                    const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
                    pba_bf16 *out, float *lse, const pba_dims *d, void *stream) {
+    return pba_fwd_local(q, k, v, bias, key_mask, gate, out, lse, d, -1, stream);
+}
+
+pba_status pba_fwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                         pba_bf16 *out, float *lse, const pba_dims *d, int window, void *stream) {
     g_last_error.clear();
     pba_status st = check_dims(d);
     if (st != PBA_OK) return st;
+    if ((st = check_window(d, window)) != PBA_OK) return st;
     if (d->B == 0 || d->Nq == 0) return PBA_OK;  // nothing to compute
     if ((st = check_layouts(d)) != PBA_OK) return st;
     if (!q || !k || !v || !out || !lse) return fail(PBA_ERR_INVALID_ARG, "q, k, v, out and lse are required");
@@ -880,9 +901,9 @@ pba_status pba_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     if ((st = get_encoder()) != PBA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (padded_c(d->C)) {
-        case 16: return launch_fwd<16>(q, k, v, bias, key_mask, gate, out, lse, d, s);
-        case 32: return launch_fwd<32>(q, k, v, bias, key_mask, gate, out, lse, d, s);
-        default: return launch_fwd<64>(q, k, v, bias, key_mask, gate, out, lse, d, s);
+        case 16: return launch_fwd<16>(q, k, v, bias, key_mask, gate, out, lse, d, window, s);
+        case 32: return launch_fwd<32>(q, k, v, bias, key_mask, gate, out, lse, d, window, s);
+        default: return launch_fwd<64>(q, k, v, bias, key_mask, gate, out, lse, d, window, s);
     }
 }
 
@@ -896,9 +917,20 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                    const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
                    pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
                    void *workspace, size_t workspace_bytes, const pba_dims *d, void *stream) {
+    return pba_bwd_local(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
+                         workspace, workspace_bytes, d, -1, stream);
+}
+
+pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                         const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                         pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                         void *workspace, size_t workspace_bytes, const pba_dims *d, int window,
+                         void *stream) {
     g_last_error.clear();
     pba_status st = check_dims(d);
     if (st != PBA_OK) return st;
+    if ((st = check_window(d, window)) != PBA_OK) return st;
     if (d->B == 0) return PBA_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d->Nq == 0) {
@@ -935,9 +967,12 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         return fail(PBA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     if ((st = get_encoder()) != PBA_OK) return st;
     switch (padded_c(d->C)) {
-        case 16: return launch_bwd<16>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
-        case 32: return launch_bwd<32>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
-        default: return launch_bwd<64>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d, s);
+        case 16: return launch_bwd<16>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d,
+                                  window, s);
+        case 32: return launch_bwd<32>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d,
+                                  window, s);
+        default: return launch_bwd<64>(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate, workspace, pl, d,
+                                  window, s);
     }
 }
 

@@ -30,6 +30,8 @@ struct BwdArgs {
     int B, H, Nq, Nk, C;
     int nI, nJ, NqPad, NkPad;
     int splits, rows_per_split;
+    int win;                   // local attention: key tile j is seen by query tiles [j - win,
+                               // j + win] (clamped); < 0: every query tile
     float scale;
     int has_bias, has_gate;
     const uint8_t *mask;
@@ -285,12 +287,11 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint8_t *gbase = dsmem + (sbase - raw);
 
     const int warp = warp_id(), lane = lane_id();
-    const int nI = a.nI;
     const long long n_items = (long long)a.B * a.H * a.nJ;
-    // items of this CTA: blockIdx.x + m * gridDim.x, m < M; steps t = m * nI + i
+    // items of this CTA: blockIdx.x + m * gridDim.x, m < M; an item's steps are its query
+    // tiles ilo .. ilo + ni - 1, and t counts the CTA's steps
     const int M = blockIdx.x < n_items ? (int)((n_items - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
-    const int Tn = M * nI;
-    struct Item { int b, h, jt; };
+    struct Item { int b, h, jt, ilo, ni; };
     auto item = [&](int m) {   // n_items < 2^31 (checked on the host)
         int n = (int)blockIdx.x + m * (int)gridDim.x;
         Item it;
@@ -298,6 +299,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         n /= a.nJ;
         it.h = n % a.H;
         it.b = n / a.H;
+        it.ilo = a.win < 0 ? 0 : max(0, it.jt - a.win);
+        it.ni = (a.win < 0 ? a.nI : min(a.nI, it.jt + a.win + 1)) - it.ilo;   // >= 1 (host check)
         return it;
     };
 
@@ -354,6 +357,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (a.has_bias) tma_prefetch_desc(&tmBias);
         }
         bool ok = true;
+        int t = 0;
         for (int m = 0; m < M && ok; ++m) {
             const Item it = item(m);
             const int x = m % KVB, j0 = it.jt * 128;
@@ -373,8 +377,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tma_load_4d(sbase + T::OFF_V + x * T::TILE_BYTES, &tmV, b_kv_full(x), 0, it.h, j0, it.b);
             }
             kv_done = m + 1;
-            for (int i = 0; i < nI && ok; ++i) {
-                const int t = m * nI + i, st = t % QS, bs = t % BS, i0 = i * 128;
+            for (int ii = 0; ii < it.ni && ok; ++ii, ++t) {
+                const int st = t % QS, bs = t % BS, i0 = (it.ilo + ii) * 128;
                 if (t >= QS) ok = mbar_wait(b_q_empty(st), ((t / QS) - 1) & 1, abort_flag, SITE_BWD_PROD | (t << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -410,26 +414,30 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);   // S = Q K^T, dP = dOa V^T
             bool ok = true;
             // step t: its item's K/V, its Q/dOa, and S/dP of step t - 1 read out
-            for (int t = 0; t < Tn && ok; ++t) {
-                const int m = t / nI, st = t % QS, x = m % KVB;
-                if (t % nI == 0)
-                    ok = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
-                if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
-                if (ok && t > 0) ok = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                const uint32_t sDO = sQ + T::TILE_BYTES;
-                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
-                const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
+            int t = 0;
+            for (int m = 0; m < M && ok; ++m) {
+                const int ni = item(m).ni;
+                for (int ii = 0; ii < ni && ok; ++ii, ++t) {
+                    const int st = t % QS, x = m % KVB;
+                    if (ii == 0)
+                        ok = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
+                    if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
+                    if (ok && t > 0) ok = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
+                    const uint32_t sDO = sQ + T::TILE_BYTES;
+                    const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                    const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < CP / 16; ++kk) {
-                    umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(sK + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
-                    umma_ss(tbase + T::T_DP, sdesc(sDO + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                    for (int kk = 0; kk < CP / 16; ++kk) {
+                        umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
+                                sdesc(sK + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                        umma_ss(tbase + T::T_DP, sdesc(sDO + kk * 32, 16, SBO, T::SWZ),
+                                sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                    }
+                    umma_commit(b_sd_full);
                 }
-                umma_commit(b_sd_full);
             }
         }
     } else if (warp == 9) {
@@ -442,48 +450,52 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             bool ok = true;
             // step t: P/dS written (S/dP of the step were read out before that, so its
             // S/dP MMAs are complete); this item's dK/dV buffer and the dQ buffer free
-            for (int t = 0; t < Tn && ok; ++t) {
-                const int m = t / nI, i = t % nI, st = t % QS;
-                const int x = m % KVB, d = m % DKB;
-                ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
-                if (!ok) break;
-                if (i == 0 && m >= DKB) {
-                    // this item's dK/dV buffer: the epilogue of item m - DKB has read it
-                    ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
+            int t = 0;
+            for (int m = 0; m < M && ok; ++m) {
+                const int ni = item(m).ni;
+                for (int i = 0; i < ni && ok; ++i, ++t) {   // i: the item's step (query tile ilo + i)
+                    const int st = t % QS;
+                    const int x = m % KVB, d = m % DKB;
+                    ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
                     if (!ok) break;
-                }
-                if (t >= 2) {
-                    ok = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
-                    if (!ok) break;
-                }
-                tc_fence_after();
-                const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                const uint32_t sDO = sQ + T::TILE_BYTES;
-                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
-                const uint32_t tDK = tbase + T::T_DK + d * 2 * CP, tDV = tDK + CP;
+                    if (i == 0 && m >= DKB) {
+                        // this item's dK/dV buffer: the epilogue of item m - DKB has read it
+                        ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
+                        if (!ok) break;
+                    }
+                    if (t >= 2) {
+                        ok = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
+                    const uint32_t sDO = sQ + T::TILE_BYTES;
+                    const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                    const uint32_t tDK = tbase + T::T_DK + d * 2 * CP, tDV = tDK + CP;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
-                    // B (dOa / Q, MN-major) rows advance 16 rows
-                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                    umma_ss(tDV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
-                            sdesc(sDO + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                    umma_ss(tDK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
-                            sdesc(sQ + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                }
+                    for (int kk = 0; kk < 8; ++kk) {
+                        // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
+                        // B (dOa / Q, MN-major) rows advance 16 rows
+                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                        umma_ss(tDV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
+                                sdesc(sDO + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
+                        umma_ss(tDK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
+                                sdesc(sQ + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
+                    }
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half
-                    const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
-                            sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
-                }
-                umma_commit(b_ps_free);
-                umma_commit(b_q_empty(st));
-                umma_commit(b_dq_full(t & 1));
-                if (i == nI - 1) {
-                    umma_commit(b_dkv_full(d));
-                    umma_commit(b_kv_empty(x));
+                    for (int kk = 0; kk < 8; ++kk) {
+                        // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half
+                        const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
+                                sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
+                    }
+                    umma_commit(b_ps_free);
+                    umma_commit(b_q_empty(st));
+                    umma_commit(b_dq_full(t & 1));
+                    if (i == ni - 1) {
+                        umma_commit(b_dkv_full(d));
+                        umma_commit(b_kv_empty(x));
+                    }
                 }
             }
         }
@@ -497,54 +509,58 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         bool ok = true;
         uint32_t mw0 = 0, mw1 = 0;
         bool full = true;
-        for (int t = 0; t < Tn && ok; ++t) {
-            const int m = t / nI, i = t % nI, st = t % QS, bs = t % BS;
-            if (i == 0) {
-                // this item's mask words come with its K/V tiles
-                ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
+        int t = 0;
+        for (int m = 0; m < M && ok; ++m) {
+            const int ni = item(m).ni;
+            for (int i = 0; i < ni && ok; ++i, ++t) {
+                const int st = t % QS, bs = t % BS;
+                if (i == 0) {
+                    // this item's mask words come with its K/V tiles
+                    ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + (m % KVB) * 8;
+                    mw0 = mw[2 * e];
+                    mw1 = mw[2 * e + 1];
+                    full = mw[4 + e] != 0;
+                }
+                ok = mbar_wait(b_sd_full, t & 1, abort_flag, SITE_BWD_EW | (t << 12));
+                if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_EW | 0x40 | (t << 12));
+                if (ok) ok = mbar_wait(b_bias_full(bs), (t / BS) & 1, abort_flag, SITE_BWD_EW | 0x50 | (t << 12));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + (m % KVB) * 8;
-                mw0 = mw[2 * e];
-                mw1 = mw[2 * e + 1];
-                full = mw[4 + e] != 0;
-            }
-            ok = mbar_wait(b_sd_full, t & 1, abort_flag, SITE_BWD_EW | (t << 12));
-            if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_EW | 0x40 | (t << 12));
-            if (ok) ok = mbar_wait(b_bias_full(bs), (t / BS) & 1, abort_flag, SITE_BWD_EW | 0x50 | (t << 12));
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
-            uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
-            const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
-            p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
-                      row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
-                      [&](int c, float2 p, float2 ds) {
-                          pp[c >> 1] = pack_bf16x2(p.x, p.y);
-                          dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
-                      });
-            tc_fence_before();
-            mbar_arrive(b_sd_free);
-            mbar_arrive(b_bias_empty(bs));
-            mbar_arrive(b_q_empty(st));
-            if (t > 0) {
-                ok = mbar_wait(b_ps_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x60 | (t << 12));
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-            }
-            // P and dS (bf16) into their 128-byte swizzled tiles: half e, row `row`
-            const uint32_t prow = sbase + T::OFF_P + e * 16384 + row * 128;
-            const uint32_t drow = sbase + T::OFF_DS + e * 16384 + row * 128;
+                tc_fence_after();
+                const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
+                uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
+                const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
+                p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
+                          row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
+                          [&](int c, float2 p, float2 ds) {
+                              pp[c >> 1] = pack_bf16x2(p.x, p.y);
+                              dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
+                          });
+                tc_fence_before();
+                mbar_arrive(b_sd_free);
+                mbar_arrive(b_bias_empty(bs));
+                mbar_arrive(b_q_empty(st));
+                if (t > 0) {
+                    ok = mbar_wait(b_ps_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x60 | (t << 12));
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                }
+                // P and dS (bf16) into their 128-byte swizzled tiles: half e, row `row`
+                const uint32_t prow = sbase + T::OFF_P + e * 16384 + row * 128;
+                const uint32_t drow = sbase + T::OFF_DS + e * 16384 + row * 128;
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                const uint32_t sw = (uint32_t)((c8 ^ (row & 7)) << 4);
-                sts128(prow + sw, make_uint4(pp[c8 * 4], pp[c8 * 4 + 1], pp[c8 * 4 + 2], pp[c8 * 4 + 3]));
-                sts128(drow + sw, make_uint4(dsp[c8 * 4], dsp[c8 * 4 + 1], dsp[c8 * 4 + 2], dsp[c8 * 4 + 3]));
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint32_t sw = (uint32_t)((c8 ^ (row & 7)) << 4);
+                    sts128(prow + sw, make_uint4(pp[c8 * 4], pp[c8 * 4 + 1], pp[c8 * 4 + 2], pp[c8 * 4 + 3]));
+                    sts128(drow + sw, make_uint4(dsp[c8 * 4], dsp[c8 * 4 + 1], dsp[c8 * 4 + 2], dsp[c8 * 4 + 3]));
+                }
+                // generic-proxy writes -> visible to the tensor core's async proxy
+                fence_proxy_async();
+                mbar_arrive(b_ps_full);
             }
-            // generic-proxy writes -> visible to the tensor core's async proxy
-            fence_proxy_async();
-            mbar_arrive(b_ps_full);
         }
     } else if (warp >= 12) {
         // ------------------------------------------------------------------ dQ and dK/dV
@@ -554,14 +570,14 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const bool issuer = threadIdx.x == 384;
         bool ok = true;
-        auto flush_dq = [&](int t, const Item &it) -> bool {
+        auto flush_dq = [&](int t, int i0, const Item &it) -> bool {
             // dQ(t): this thread's query row, all CP channels, added to dqacc
             bool okf = mbar_wait(b_dq_full(t & 1), (t >> 1) & 1, abort_flag, SITE_BWD_EPI | 0x10 | (t << 12));
             okf = __all_sync(0xffffffffu, okf);
             if (!okf) return false;
             tc_fence_after();
             const uint32_t tq = tbase + T::T_DQ + (t & 1) * CP + lane_off;
-            const int i = (t % nI) * 128 + row;
+            const int i = i0 + row;
             if constexpr (T::DQ_TMA) {
                 uint32_t r[32];
                 tmem_ld32(tq, r);
@@ -592,7 +608,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     // rows >= Nq and channels >= C fall outside the map and are skipped
                     oki = mbar_wait(b_stg_full, t & 1, abort_flag, SITE_BWD_EPI | 0x80 | (t << 12));
                     if (oki) {
-                        tma_reduce_add_4d(&tmDQ, sbase + T::OFF_DQS, 0, it.h, (t % nI) * 128, it.b);
+                        tma_reduce_add_4d(&tmDQ, sbase + T::OFF_DQS, 0, it.h, i0, it.b);
                         bulk_commit();
                     }
                 }
@@ -663,12 +679,13 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             return true;
         };
-        Item cur = {0, 0, 0};
-        for (int t = 0; t < Tn && ok; ++t) {
-            const int m = t / nI, i = t % nI;
-            if (i == 0) cur = item(m);
-            ok = flush_dq(t, cur);
-            if (ok && i == nI - 1) ok = epilogue(m, cur);
+        int t = 0;
+        for (int m = 0; m < M && ok; ++m) {
+            const Item cur = item(m);
+            for (int i = 0; i < cur.ni && ok; ++i, ++t) {
+                ok = flush_dq(t, (cur.ilo + i) * 128, cur);
+                if (ok && i == cur.ni - 1) ok = epilogue(m, cur);
+            }
         }
         if (T::DQ_TMA && issuer) bulk_wait_all();   // its TMA reductions are done
     }
@@ -749,6 +766,17 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int i0 = it * 128, j0 = jt * 128;
     const int bstart = sp * a.rows_per_split;
     const int nb = max(0, min(a.rows_per_split, a.B - bstart));
+    if (a.win >= 0 && (it < jt - a.win || it > jt + a.win)) {
+        // local attention: no query of this tile sees a key of it, dS = 0; split 0 writes
+        // the zero tile, the other splits have nothing to do
+        if (sp == 0) {
+            for (int v = threadIdx.x; v < 128 * 128; v += blockDim.x) {
+                const int i = i0 + (v >> 7), j = j0 + (v & 127);
+                if (i < a.Nq && j < a.Nk) a.dbias[((long long)h * a.Nq + i) * a.Nk + j] = 0.f;
+            }
+        }
+        return;
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(b_bias, 1);

@@ -43,6 +43,8 @@ struct FwdArgs {
     int B, H, Nq, Nk, C;
     int nI, nJ, nChunks;
     int items;       // H * nI * nChunks work items, walked by a grid of at most 2 CTAs per SM
+    int win;         // local attention: query tile t visits key tiles [t - win, t + win] (clamped);
+                     // < 0: every key tile
     float scale;
     int has_bias;
     int mask_shared;  // the key mask (if any) is one row shared by every b
@@ -144,12 +146,12 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC + 4);
 
     const int warp = warp_id(), lane = lane_id();
-    const int nJ = a.nJ;
     const bool row_mask = a.mask != nullptr && !a.mask_shared;
     // item n of this CTA is blockIdx.x + n gridDim.x: query tile fastest, then the chunk of
     // rows, then the head (CTAs running at the same time share K/V and bias tiles in L2)
     struct FItem {
         int h, i0, b0, nb;
+        int jlo, nj;   // the item's key tiles [jlo, jlo + nj)
     };
     auto item = [&](int n) {
         int idx = blockIdx.x + n * gridDim.x;
@@ -161,10 +163,13 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         it.i0 = itile * 128;
         it.b0 = chunk * BC;
         it.nb = min(BC, a.B - it.b0);
+        it.jlo = a.win < 0 ? 0 : max(0, itile - a.win);
+        it.nj = (a.win < 0 ? a.nJ : min(a.nJ, itile + a.win + 1)) - it.jlo;   // >= 1 (host check)
         return it;
     };
     const int n_items = (int)blockIdx.x < a.items ? (a.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    // steps of an item: (j, s), local index j * nb + s; k below is the CTA's step count
+    // steps of an item: (key tile jlo + j, row s), local index j * nb + s; k below is the
+    // CTA's step count
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
@@ -261,7 +266,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (lane == 0 && k != a.skip_step) {
                 mbar_arrive_tx(b_k_full(st), T::TILE_BYTES);
                 tma_load_4d(sbase + T::OFF_K + st * T::TILE_BYTES, &tmK, b_k_full(st), 0, it.h,
-                            (kl / it.nb) * 128, it.b0 + kl % it.nb);
+                            (it.jlo + kl / it.nb) * 128, it.b0 + kl % it.nb);
             }
             k_done = k + 1;
             return true;
@@ -273,7 +278,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 ok = mbar_wait(b_v_empty(st), (use - 1) & 1, abort_flag, SITE_FWD_PROD | 0x10 | (k << 12));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return false;
-            const int j = kl / it.nb, b = it.b0 + kl % it.nb;
+            const int j = it.jlo + kl / it.nb, b = it.b0 + kl % it.nb;
             if (row_mask) {
                 // words of row b: word q bit t <-> key 128 j + 32 q + t attended
                 uint32_t w[4];
@@ -303,16 +308,16 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         int kg = 0, jg = 0;   // the CTA's steps and bias tiles before this item
         for (int n = 0; n < n_items && ok; ++n) {
             const FItem it = item(n);
-            const int Kn = nJ * it.nb;
-            ok = load_bias(jg, 0, it) && load_k(kg, 0, it) && load_q(n, it);
+            const int Kn = it.nj * it.nb;
+            ok = load_bias(jg, it.jlo, it) && load_k(kg, 0, it) && load_q(n, it);
             for (int kl = 0; kl < Kn && ok; ++kl) {
                 if (kl + 1 < Kn) ok = load_k(kg + kl + 1, kl + 1, it);
                 if (ok) ok = load_v(kg + kl, kl, it);
                 if (ok && kl + 1 < Kn && (kl + 1) % it.nb == 0)
-                    ok = load_bias(jg + (kl + 1) / it.nb, (kl + 1) / it.nb, it);
+                    ok = load_bias(jg + (kl + 1) / it.nb, it.jlo + (kl + 1) / it.nb, it);
             }
             kg += Kn;
-            jg += nJ;
+            jg += it.nj;
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------------ Q K^T issuer
@@ -322,7 +327,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             bool ok = true;
             int kg = 0;
             for (int n = 0; n < n_items && ok; ++n) {
-                const int nb = item(n).nb, Kn = nJ * nb;
+                const FItem it = item(n);
+                const int nb = it.nb, Kn = it.nj * nb;
                 ok = mbar_wait(b_q_full, n & 1, abort_flag, SITE_FWD_MMA | 0x50 | (n << 12));
                 // step k: S must have been read out by the softmax of step k - 1
                 for (int kl = 0; kl < Kn && ok; ++kl) {
@@ -352,7 +358,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             bool ok = true;
             int kg = 0;
             for (int n = 0; n < n_items && ok; ++n) {
-                const int nb = item(n).nb, Kn = nJ * nb;
+                const FItem it = item(n);
+                const int nb = it.nb, Kn = it.nj * nb;
                 // step k: P of step k written (and O[s] rescaled) by the softmax, V landed
                 for (int kl = 0; kl < Kn && ok; ++kl) {
                     const int k = kg + kl, j = kl / nb, s = kl % nb, st = k % KVS;
@@ -378,59 +385,62 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // ------------------------------------------------------------------ mask fold
         const int t = lane;   // rows t, t + 32, t + 64, t + 96 of every bias tile
         bool ok = true;
-        const int n_tiles = n_items * nJ;   // the CTA's bias tiles; tile jg has key tile jg % nJ
-        for (int jg = 0; jg < n_tiles && ok; ++jg) {
-            const int bs = jg % BS, j = jg % nJ;
-            // word q bit l <-> key 128 j + 32 q + l attended by every row of the chunk
-            uint32_t w[4];
+        int jg = 0;   // the CTA's bias tiles
+        for (int n = 0; n < n_items && ok; ++n) {
+            const FItem it = item(n);
+            for (int jl = 0; jl < it.nj && ok; ++jl, ++jg) {
+                const int bs = jg % BS, j = it.jlo + jl;
+                // word q bit l <-> key 128 j + 32 q + l attended by every row of the chunk
+                uint32_t w[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int key = j * 128 + q * 32 + lane;
-                bool valid = key < a.Nk;
-                if (valid && a.mask && !row_mask) valid = a.mask[key] != 0;
-                w[q] = __ballot_sync(0xffffffffu, valid);
-            }
-            ok = mbar_wait(b_bias_full(bs), (jg / BS) & 1, abort_flag, SITE_FWD_FOLD | (jg << 12));
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            uint8_t *tile = dsmem + T::OFF_BIAS + bs * T::BIAS_BYTES;
-            if (a.has_bias) {
-                if ((w[0] & w[1] & w[2] & w[3]) != 0xffffffffu) {
+                for (int q = 0; q < 4; ++q) {
+                    const int key = j * 128 + q * 32 + lane;
+                    bool valid = key < a.Nk;
+                    if (valid && a.mask && !row_mask) valid = a.mask[key] != 0;
+                    w[q] = __ballot_sync(0xffffffffu, valid);
+                }
+                ok = mbar_wait(b_bias_full(bs), (jg / BS) & 1, abort_flag, SITE_FWD_FOLD | (jg << 12));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                uint8_t *tile = dsmem + T::OFF_BIAS + bs * T::BIAS_BYTES;
+                if (a.has_bias) {
+                    if ((w[0] & w[1] & w[2] & w[3]) != 0xffffffffu) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t m = ~w[q];
-                        while (m) {
-                            const int c = q * 32 + __ffs(m) - 1;
-                            m &= m - 1;
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t m = ~w[q];
+                            while (m) {
+                                const int c = q * 32 + __ffs(m) - 1;
+                                m &= m - 1;
 #pragma unroll
-                            for (int r = t; r < 128; r += 32)
-                                *reinterpret_cast<uint16_t *>(tile + bias_off(r, c)) = 0xFF80u;
+                                for (int r = t; r < 128; r += 32)
+                                    *reinterpret_cast<uint16_t *>(tile + bias_off(r, c)) = 0xFF80u;
+                            }
                         }
                     }
-                }
-            } else {
-                // no bias: 0 for attended keys, -inf for the rest
+                } else {
+                    // no bias: 0 for attended keys, -inf for the rest
 #pragma unroll 1
-                for (int ch = 0; ch < 16; ++ch) {   // 16-byte chunk ch: keys 8 ch .. 8 ch + 7
-                    const int qw = ch >> 2;
-                    const uint32_t wq = qw == 0 ? w[0] : qw == 1 ? w[1] : qw == 2 ? w[2] : w[3];
-                    const uint32_t bits = wq >> ((ch & 3) * 8);
-                    uint32_t v4[4];
+                    for (int ch = 0; ch < 16; ++ch) {   // 16-byte chunk ch: keys 8 ch .. 8 ch + 7
+                        const int qw = ch >> 2;
+                        const uint32_t wq = qw == 0 ? w[0] : qw == 1 ? w[1] : qw == 2 ? w[2] : w[3];
+                        const uint32_t bits = wq >> ((ch & 3) * 8);
+                        uint32_t v4[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t lo = ((bits >> (2 * e)) & 1u) ? 0u : 0xFF80u;
-                        const uint32_t hi = ((bits >> (2 * e + 1)) & 1u) ? 0u : 0xFF80u;
-                        v4[e] = lo | (hi << 16);
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t lo = ((bits >> (2 * e)) & 1u) ? 0u : 0xFF80u;
+                            const uint32_t hi = ((bits >> (2 * e + 1)) & 1u) ? 0u : 0xFF80u;
+                            v4[e] = lo | (hi << 16);
+                        }
+                        const uint4 val = make_uint4(v4[0], v4[1], v4[2], v4[3]);
+                        const uint32_t tb = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
+#pragma unroll
+                        for (int r = t; r < 128; r += 32) sts128(tb + bias_off(r, ch * 8), val);
                     }
-                    const uint4 val = make_uint4(v4[0], v4[1], v4[2], v4[3]);
-                    const uint32_t tb = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES;
-#pragma unroll
-                    for (int r = t; r < 128; r += 32) sts128(tb + bias_off(r, ch * 8), val);
                 }
+                // these generic writes precede a later TMA refill of the same buffer
+                fence_proxy_async();
+                mbar_arrive(b_bias_ready(bs));
             }
-            // these generic writes precede a later TMA refill of the same buffer
-            fence_proxy_async();
-            mbar_arrive(b_bias_ready(bs));
         }
     } else {
         // ------------------------------------------------------------------ softmax
@@ -452,7 +462,7 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 m_run[t] = -INFINITY;
                 l_run[t] = 0.f;
             }
-            for (int j = 0; j < nJ && ok; ++j, ++jg) {
+            for (int j = 0; j < it.nj && ok; ++j, ++jg) {   // j: the item's key tile jlo + j
                 const int bs = jg % BS;
                 for (int s = 0; s < nb; ++s, ++k) {
                     const int st = k % KVS;

@@ -38,6 +38,7 @@ class Config:
     passes: str       # "fwd" or "fwdbwd": which passes the workload names
     gate: bool = True
     desc: str = ""
+    window: int = -1  # local attention: query tile t sees key tiles [t - window, t + window]
 
     def keep(self) -> np.ndarray:
         keep = np.ones(self.N, dtype=np.uint8)
@@ -70,13 +71,28 @@ CONFIGS: Dict[str, Config] = {
                  masked=((160, 198), (448, 486), (729, 768)), passes="fwdbwd",
                  desc="large triangle attention: 768 rows x 768 keys, 15% keys masked in "
                       "three contiguous padding blocks"),
+    "C6": Config("C6", B=48, H=4, N=3072, c=32, bias_std=1.0, masked=((3040, 3072),),
+                 passes="fwdbwd", window=1,
+                 desc="sequence-local atom attention of the diffusion module: 48 noise-level "
+                      "copies, 3072 atoms, 4 heads, each 128-atom query tile sees the key tiles "
+                      "within one tile of it (block-sparse), last 32 atoms padding"),
 }
 
 
+def window_pair_mask(Nq: int, Nk: int, window: int) -> np.ndarray:
+    """[Nq, Nk] bool: True where query i may attend key j under a tile window (query tile
+    i // 128 sees key tiles within `window` of it; window < 0: every pair)."""
+    if window < 0:
+        return np.ones((Nq, Nk), dtype=bool)
+    ti = np.arange(Nq)[:, None] // 128
+    tj = np.arange(Nk)[None, :] // 128
+    return np.abs(ti - tj) <= window
+
+
 def custom(name: str, B: int, H: int, N: int, c: int, bias_std: float = 1.0,
-           masked=(), gate: bool = True) -> Config:
+           masked=(), gate: bool = True, window: int = -1) -> Config:
     return Config(name, B=B, H=H, N=N, c=c, bias_std=bias_std, masked=tuple(masked),
-                  passes="fwdbwd", gate=gate)
+                  passes="fwdbwd", gate=gate, window=window)
 
 
 # ----------------------------------------------------------------------------------------

@@ -127,3 +127,15 @@ def test_pair_bias_host_side_argument_errors(pba):
     st = pba.lib.pba_pair_bias_bwd(16, 16, 16, 16, 16, 16, 16, 16, 16, 256, need - 4, ctypes.byref(d), None)
     assert st == 5                                                       # workspace too small
     assert pba.lib.pba_pair_bias_bwd_workspace_size(ctypes.byref(_pb_dims(pba, Cz=100))) == 0
+
+
+def test_local_window_refusals(pba):
+    d = pba.dims_dense(2, 2, 128, 1024, 32)          # 1 query tile, 8 key tiles
+    st = pba.lib.pba_fwd_local(16, 16, 16, None, None, None, 16, 16, ctypes.byref(d), 0, None)
+    assert st == 2 and "window" in pba.lib.pba_last_error().decode()
+    st = pba.lib.pba_bwd_local(*([16] * 9), 16, 16, 16, None, None, 256, 1 << 30, ctypes.byref(d), 0, None)
+    assert st == 2
+    d0 = pba.dims_dense(0, 2, 128, 1024, 32)         # empty problem, but the window is still checked
+    assert pba.lib.pba_fwd_local(None, None, None, None, None, None, None, None, ctypes.byref(d0), 0, None) == 2
+    # window -1 is the dense operator: the same empty problem is a no-op
+    assert pba.lib.pba_fwd_local(None, None, None, None, None, None, None, None, ctypes.byref(d0), -1, None) == 0
