@@ -45,7 +45,7 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 // ---------------------------------------------------------------------------- profiling
 enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS,
                 K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS,
-                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_COUNT };
+                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_DBIAS_ZERO, K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
                                            "pba_dbias_kernel",
                                            "pba_dq_convert_kernel", "zero_rows_kernel",
@@ -53,7 +53,8 @@ const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel
                                            "pba_pwa_pre_kernel", "pba_pwa_gemm_kernel (dv)",
                                            "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel",
                                            "pba_pair_bias_fwd_kernel", "pba_pair_bias_bwd_kernel",
-                                           "pba_pair_bias_reduce_kernel", "pba_pair_bias_param_kernel"};
+                                           "pba_pair_bias_reduce_kernel", "pba_pair_bias_param_kernel",
+                                           "pba_dbias_zero_kernel"};
 struct ProfRec {
     int kid;
     cudaEvent_t a, b;
@@ -298,38 +299,43 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
 constexpr long long kSmCount = 148;   // SMs of a B200
 
 struct BwdPlan {
-    int nI, nJ, NqPad, NkPad, splits, rows_per_split;
+    int nI, nJ, NqPad, NkPad, splits, rows_per_split, ntiles;
     size_t off_rs, off_doa, off_dq, off_cnt, off_part, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-BwdPlan plan_bwd(const pba_dims *d) {
+// the split count that minimises waves x (rows + 3) for `tiles` dbias tiles, at most
+// `max_part` split partial tiles (splits x tiles)
+void choose_splits(const pba_dims *d, long long tiles, long long max_part, int *splits, int *rows_per_split);
+
+BwdPlan plan_bwd(const pba_dims *d, int win = -1) {
     BwdPlan p;
     p.nI = (d->Nq + 127) / 128;
     p.nJ = (d->Nk + 127) / 128;
     p.NqPad = p.nI * 128;
     p.NkPad = p.nJ * 128;
+    p.ntiles = p.nI * p.nJ;
+    if (win >= 0) {   // local attention: the (query tile, key tile) pairs within the window
+        long long n = 0;
+        for (int i = 0; i < p.nI; ++i) n += std::min(p.nJ, i + win + 1) - std::max(0, i - win);
+        p.ntiles = (int)n;
+    }
     // splits of the broadcast rows for the dbias kernel: a fixed function of the sizes,
     // so the reduction order (and every bit of dbias) depends on nothing else.  A CTA
     // handles one (head, query tile, key tile, split); its time grows with the rows of its
     // split plus a fixed cost (bias tile, pipeline fill, the partial tile's store) of about
     // three rows, so pick the split count that minimises waves x (rows + 3) on 148 SMs.
-    const long long tiles = (long long)d->H * p.nI * p.nJ;
-    const long long maxs = d->B < 64 ? (d->B > 0 ? d->B : 1) : 64;
-    long long best_cost = -1;
-    p.splits = 1;
-    p.rows_per_split = d->B > 0 ? d->B : 1;
-    for (long long sp = 1; sp <= maxs; ++sp) {
-        const long long rows = d->B > 0 ? (d->B + sp - 1) / sp : 1;
-        const long long actual = d->B > 0 ? (d->B + rows - 1) / rows : 1;
-        const long long waves = (tiles * actual + kSmCount - 1) / kSmCount;
-        const long long cost = waves * (rows + 3);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            p.splits = (int)actual;
-            p.rows_per_split = (int)rows;
-        }
+    // The workspace is sized for the dense problem, so a window's plan holds at most as many
+    // partial tiles as the dense plan.
+    int dense_splits, dense_rows;
+    choose_splits(d, (long long)d->H * p.nI * p.nJ, -1, &dense_splits, &dense_rows);
+    if (win < 0) {
+        p.splits = dense_splits;
+        p.rows_per_split = dense_rows;
+    } else {
+        choose_splits(d, (long long)d->H * p.ntiles, (long long)dense_splits * p.nI * p.nJ * d->H,
+                      &p.splits, &p.rows_per_split);
     }
     const size_t rows = (size_t)d->B * d->H * p.NqPad;
     const size_t elems = (size_t)d->B * d->Nq * d->H * d->C;
@@ -339,8 +345,27 @@ BwdPlan plan_bwd(const pba_dims *d) {
     // per-tile counters of the dbias kernel (cleared by the pre kernel)
     p.off_cnt = align256(p.off_dq + elems * 4);
     p.off_part = align256(p.off_cnt + (size_t)d->H * p.nI * p.nJ * sizeof(int));
-    p.total = align256(p.off_part + (size_t)p.splits * d->H * p.NqPad * p.NkPad * 4);
+    p.total = align256(p.off_part + (size_t)p.splits * d->H * p.ntiles * 128 * 128 * 4);
     return p;
+}
+
+void choose_splits(const pba_dims *d, long long tiles, long long max_part, int *splits, int *rows_per_split) {
+    const long long maxs = d->B < 64 ? (d->B > 0 ? d->B : 1) : 64;
+    long long best_cost = -1;
+    *splits = 1;
+    *rows_per_split = d->B > 0 ? d->B : 1;
+    for (long long sp = 1; sp <= maxs; ++sp) {
+        const long long rows = d->B > 0 ? (d->B + sp - 1) / sp : 1;
+        const long long actual = d->B > 0 ? (d->B + rows - 1) / rows : 1;
+        if (max_part >= 0 && actual * tiles > max_part) break;
+        const long long waves = (tiles * actual + kSmCount - 1) / kSmCount;
+        const long long cost = waves * (rows + 3);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            *splits = (int)actual;
+            *rows_per_split = (int)rows;
+        }
+    }
 }
 
 __global__ void zero_rows_kernel(__nv_bfloat16 *dk, __nv_bfloat16 *dv, pba::BwdArgs a) {
@@ -406,6 +431,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.nI = pl.nI; a.nJ = pl.nJ; a.NqPad = pl.NqPad; a.NkPad = pl.NkPad;
     a.splits = pl.splits; a.rows_per_split = pl.rows_per_split;
     a.win = win;
+    a.ntiles = pl.ntiles;
     a.scale = eff_scale(d);
     a.has_bias = bias != nullptr;
     a.has_gate = gate != nullptr;
@@ -475,7 +501,13 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {
             if ((st = set_smem(pba::pba_dbias_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
-            const long long g2 = (long long)pl.splits * d->H * pl.nI * pl.nJ;
+            const long long g2 = (long long)pl.splits * d->H * pl.ntiles;
+            if (win >= 0) {
+                ProfScope ps(K_DBIAS_ZERO, s);
+                const long long rows = (long long)d->H * d->Nq;
+                pba::pba_dbias_zero_kernel<<<(unsigned)std::min<long long>(rows, 8 * kSmCount), 256, 0, s>>>(a);
+            }
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_zero_kernel launch");
             {
                 ProfScope ps(K_DBIAS, s);
                 pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
@@ -959,7 +991,7 @@ pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v
         if ((st = check_bias(d)) != PBA_OK) return st;
     }
     if (key_mask && d->smask_b < 0) return fail(PBA_ERR_INVALID_ARG, "smask_b must be >= 0");
-    const BwdPlan pl = plan_bwd(d);
+    const BwdPlan pl = plan_bwd(d, window);
     if (!workspace || workspace_bytes < pl.total)
         return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
                     pl.total);

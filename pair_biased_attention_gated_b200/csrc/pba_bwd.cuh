@@ -48,7 +48,8 @@ struct BwdArgs {
     float2 *rowstats;          // [B][H][NqPad]: (lse * log2 e, or +inf for a dead row; D)
     __nv_bfloat16 *doa;        // [B][Nq][H][C] (only with a gate)
     float *dqacc;              // [B][Nq][H][C]
-    float *dbias_part;         // [splits][H][NqPad][NkPad]
+    float *dbias_part;         // [splits][H][ntiles][128][128]
+    int ntiles;                // dbias tiles computed: nI nJ, or those within the window
     int *tile_count;           // [H][nI][nJ]: splits done (zeroed before the launch)
 };
 
@@ -716,8 +717,42 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 }
 
+// dbias tile number bt -> (query tile, key tile): row-major over the tile pairs the kernels
+// visit (every pair, or under a window the pairs with |query tile - key tile| <= win)
+__device__ __forceinline__ void dbias_tile(const BwdArgs &a, int bt, int &it, int &jt) {
+    if (a.win < 0) {
+        it = bt / a.nJ;
+        jt = bt % a.nJ;
+        return;
+    }
+    it = a.nI - 1;
+    jt = a.nJ - 1;
+    for (int i = 0; i < a.nI; ++i) {
+        const int lo = max(0, i - a.win), hi = min(a.nJ, i + a.win + 1);
+        if (bt < hi - lo) {
+            it = i;
+            jt = lo + bt;
+            return;
+        }
+        bt -= hi - lo;
+    }
+}
+
+// local attention: dbias is 0 at every pair outside the window (no query of such a pair's
+// tile sees its key); the dbias kernel writes the tiles inside it
+__global__ void __launch_bounds__(256) pba_dbias_zero_kernel(const BwdArgs a) {
+    // one dbias row (h, i) per block: the keys before and after the row's window
+    for (long long r = blockIdx.x; r < (long long)a.H * a.Nq; r += gridDim.x) {
+        const int t = (int)(r % a.Nq) >> 7;
+        const int lo = max(0, t - a.win) * 128, hi = min(a.Nk, (t + a.win + 1) * 128);
+        float *row = a.dbias + r * a.Nk;
+        for (int j = threadIdx.x; j < lo; j += blockDim.x) row[j] = 0.f;
+        for (int j = hi + threadIdx.x; j < a.Nk; j += blockDim.x) row[j] = 0.f;
+    }
+}
+
 // ---------------------------------------------------------------------------------------
-// dbias kernel: CTA = (h, query tile, key tile, split s); loops over its rows b
+// dbias kernel: CTA = (h, dbias tile, split s); loops over its rows b
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct DbTraits {
@@ -757,26 +792,15 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     const int warp = warp_id(), lane = lane_id();
     int idx = blockIdx.x;
-    const int jt = idx % a.nJ;
-    idx /= a.nJ;
-    const int it = idx % a.nI;
-    idx /= a.nI;
+    const int bt = idx % a.ntiles;   // the tile, in dbias_tile order
+    idx /= a.ntiles;
     const int h = idx % a.H;
     const int sp = idx / a.H;
+    int it, jt;
+    dbias_tile(a, bt, it, jt);
     const int i0 = it * 128, j0 = jt * 128;
     const int bstart = sp * a.rows_per_split;
     const int nb = max(0, min(a.rows_per_split, a.B - bstart));
-    if (a.win >= 0 && (it < jt - a.win || it > jt + a.win)) {
-        // local attention: no query of this tile sees a key of it, dS = 0; split 0 writes
-        // the zero tile, the other splits have nothing to do
-        if (sp == 0) {
-            for (int v = threadIdx.x; v < 128 * 128; v += blockDim.x) {
-                const int i = i0 + (v >> 7), j = j0 + (v & 127);
-                if (i < a.Nq && j < a.Nk) a.dbias[((long long)h * a.Nq + i) * a.Nk + j] = 0.f;
-            }
-        }
-        return;
-    }
 
     if (threadIdx.x == 0) {
         mbar_init(b_bias, 1);
@@ -900,9 +924,9 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_arrive(b_empty(st));
         }
         if (ok) {
-            // this split's partial tile, padded layout: [split][h][NqPad][NkPad]
+            // this split's partial tile: [split][h][tile][128][128]
             float *dst = a.dbias_part +
-                         ((((long long)sp * a.H + h) * a.NqPad + i0 + row) * a.NkPad + j0 + e * 64);
+                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 64;
 #pragma unroll
             for (int c = 0; c < 32; c += 2)
                 *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
@@ -941,11 +965,11 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const long long plane = (long long)a.H * a.NqPad * a.NkPad;
+    const long long plane = (long long)a.H * a.ntiles * 128 * 128;
     for (int v = threadIdx.x; v < 128 * 32; v += blockDim.x) {
         const int i = i0 + (v >> 5), j = j0 + (v & 31) * 4;
         if (i >= a.Nq || j >= a.Nk) continue;
-        const float *src = a.dbias_part + ((long long)h * a.NqPad + i) * a.NkPad + j;
+        const float *src = a.dbias_part + (((long long)h * a.ntiles + bt) * 128 + (i - i0)) * 128 + (j - j0);
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int q = 0; q < a.splits; ++q) {
             const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + q * plane));
