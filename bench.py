@@ -8,11 +8,16 @@ like the MSA row attention workload (128 MSA rows share one [8, 256, 256] pair b
 starts; L2 is flushed before every timed step, outside the timed events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+                  [--op attention|pwa|pairbias]
 
 N > 1 runs under torchrun, one process per GPU, each an independent replica of the
 workload (the path has no exchange step); rank 0 prints one JSON line.  `--impl
 reference` times the fp64 CPU oracle (the only other implementation of the operation)
-on the host cores instead.
+on the host cores instead.  `--config C6` is the block-sparse local (atom) attention
+workload; `--op pwa` times MSA pair-weighted averaging and `--op pairbias` the LayerNorm +
+projection that makes the bias, each with its own metric line.  The end-to-end figure
+copies every step's inputs in and results out of pinned host memory, pipelined over a
+copy-in, a compute and a copy-out stream.
 """
 from __future__ import annotations
 
