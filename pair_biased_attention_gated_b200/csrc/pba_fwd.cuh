@@ -545,6 +545,21 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     const float nm = (m_use == -INFINITY) ? 0.f : -m_use * kLog2e;
                     const float2 nm2 = make_float2(nm, nm);
 
+                    // The exponentials go into registers first: only the store of P (and a
+                    // rescale of O[s]) has to wait for the previous P V, so the exponential
+                    // unit's share of the step overlaps that product instead of following it.
+                    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+                    uint32_t p0[32], p1[32];   // P of keys 0..63 and 64..127 as bf16 pairs
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const float2 tt = ffma2(make_float2(x[2 * c], x[2 * c + 1]), l2e2, nm2);
+                        const float2 pv = make_float2(ex2(tt.x), ex2(tt.y));
+                        if (c & 1) acc1 = fadd2(acc1, pv);
+                        else acc0 = fadd2(acc0, pv);
+                        if (c < 32) p0[c] = pack_bf16x2(pv.x, pv.y);
+                        else p1[c - 32] = pack_bf16x2(pv.x, pv.y);
+                    }
+                    const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
                     // P and O[s] may only be written once the previous P V is done
                     if (k > 0) {
                         ok = mbar_wait(b_p_free, (k - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x30 | (k << 12));
@@ -552,22 +567,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         if (!ok) break;
                         tc_fence_after();
                     }
-                    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        uint32_t p[32];
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int i2 = hf * 64 + 2 * c;
-                            const float2 tt = ffma2(make_float2(x[i2], x[i2 + 1]), l2e2, nm2);
-                            const float2 pv = make_float2(ex2(tt.x), ex2(tt.y));
-                            if (c & 1) acc1 = fadd2(acc1, pv);
-                            else acc0 = fadd2(acc0, pv);
-                            p[c] = pack_bf16x2(pv.x, pv.y);
-                        }
-                        tmem_st32(tP + hf * 32, p);
-                    }
-                    const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+                    tmem_st32(tP, p0);
+                    tmem_st32(tP + 32, p1);
                     if (__any_sync(0xffffffffu, resc)) {
                         const uint32_t tO = tbase + T::T_O + s * CP + lane_off;
                         uint32_t o[CP];
