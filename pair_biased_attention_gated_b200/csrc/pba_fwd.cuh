@@ -462,6 +462,15 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 m_run[t] = -INFINITY;
                 l_run[t] = 0.f;
             }
+            // the epilogue's gate rows: into L2 now, so that their loads after the item's
+            // last step do not wait for DRAM
+            if (a.gate && it.i0 + row < a.Nq) {
+#pragma unroll
+                for (int t = 0; t < BC; ++t)
+                    if (t < nb)
+                        prefetch_l2(a.gate + (it.b0 + t) * a.sg0 + (long long)(it.i0 + row) * a.sg1 +
+                                    it.h * a.sg2);
+            }
             for (int j = 0; j < it.nj && ok; ++j, ++jg) {   // j: the item's key tile jlo + j
                 const int bs = jg % BS;
                 for (int s = 0; s < nb; ++s, ++k) {
