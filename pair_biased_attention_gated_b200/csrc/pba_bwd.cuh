@@ -473,19 +473,20 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const uint32_t sDO = sQ + T::TILE_BYTES;
                     const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
                     const uint32_t tDK = tbase + T::T_DK + d * 2 * CP, tDV = tDK + CP;
+                    // The three products interleaved, one K step of each in turn: consecutive
+                    // MMAs into one accumulator wait on each other, three accumulators in
+                    // rotation keep the tensor pipe fed.
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
-                        // B (dOa / Q, MN-major) rows advance 16 rows
+                        // dV, dK: K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance
+                        // 2 KB, B (dOa / Q, MN-major) rows advance 16 rows
                         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                         umma_ss(tDV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
                                 sdesc(sDO + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
                         umma_ss(tDK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
                                 sdesc(sQ + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half
+                        // dQ: K steps over 16 keys: A (dS, K-major) advances 32 B within a
+                        // 64-key half
                         const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
                         umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
                                 sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
