@@ -110,14 +110,22 @@ def kernel_source_file(kernel: str) -> str:
     return KERNEL_SOURCES.get(kernel, "pba_bwd.cuh")
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines: a comment edit is not a kernel change."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources one kernel is compiled from: its own file and the shared device
-    header (launch configuration in the API file is not covered)."""
+    """Hash of the code one kernel is compiled from: its own file and the shared device
+    header, comments left out (launch configuration in the API file is not covered)."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc")
     for name in (kernel_source_file(kernel), "pba_device.cuh"):
-        with open(os.path.join(cdir, name), "rb") as fh:
-            h.update(name.encode() + fh.read())
+        with open(os.path.join(cdir, name), encoding="utf-8") as fh:
+            h.update(name.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

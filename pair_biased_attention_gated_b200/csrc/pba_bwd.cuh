@@ -12,14 +12,17 @@
 //
 // Kernels, in launch order on one stream:
 //   pba_bwd_pre_kernel      per query row: dOa (bf16), dg, and (lse * log2 e, D) row stats
-//   pba_bwd_main_kernel     CTA = (b, h, 128-key tile): loops over query tiles; dK, dV
-//                           accumulate in TMEM; each step's dQ partial is added to an fp32
-//                           accumulator in global memory
-//   pba_dbias_kernel        CTA = (h, query tile, key tile, split of b): loops over its rows
-//                           b with the bias tile resident; dS summed in registers; one fp32
-//                           partial tile per split; the tile's last CTA to finish sums the
-//                           partials in split order (bit-stable dbias)
+//   pba_bwd_main_kernel     persistent, items (b, h, 128-key tile): steps over query tiles;
+//                           dK, dV accumulate in TMEM; each step's dQ partial is added to an
+//                           fp32 accumulator in global memory
+//   pba_dbias_zero_kernel   local attention only: zeros of dbias outside the window
+//   pba_dbias_kernel        CTA = (h, dbias tile, split of b): loops over its rows b with the
+//                           bias tile resident; dS summed in registers; one fp32 partial tile
+//                           per split; the tile's last CTA to finish sums the partials in
+//                           split order (bit-stable dbias)
 //   pba_dq_convert_kernel   fp32 dQ accumulator -> bf16 dq (times scale)
+// Local attention (win >= 0): key tile j is seen only by query tiles [j - win, j + win]; the
+// main kernel's items step over those, the dbias kernel covers only those tile pairs.
 #pragma once
 
 #include "pba_device.cuh"
