@@ -133,3 +133,28 @@ def test_atom_attention_size_sampled(pba):
                                             f["keep"], f["g"][b, rows, h])
             assert_out_close(got[b, rows, h], r_out)
             assert_lse_close(gl[b, h, rows], r_lse)
+
+
+def test_local_attention_per_row_key_mask(pba):
+    """A key mask with one row per b (its words travel with each row's K/V tiles) under a window."""
+    B, H, N, C, window = 4, 2, 512, 32, 1
+    cfg = pi.custom("lrow", B=B, H=H, N=N, c=C)
+    d = pi.make_inputs(cfg, seed=7)
+    keep = np.ones((B, N), dtype=np.uint8)
+    for b in range(B):
+        keep[b, 480 - 37 * b:] = 0          # a different padding tail per row
+        keep[b, 100 + 50 * b: 110 + 50 * b] = 0
+    d["keep"] = keep
+    t = to_dev(d)
+    out, lse = pba.attention_fwd(t["q"], t["k"], t["v"], t["bias"], t["keep"], t["g"], window=window)
+    dq, dk, dv, dg, db = pba.attention_bwd(t["q"], t["k"], t["v"], t["bias"], t["keep"], t["g"], out, lse,
+                                           t["dout"], window=window)
+    pba.pba_device_status()
+    f = _ref(d, window, N, N)
+    r_out, r_lse = oracle.fwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f["g"])
+    assert_out_close(bf16_to_f64_tensor(out), r_out)
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), r_lse)
+    r_dq, r_dk, r_dv, r_dg, r_db = oracle.bwd(f["q"], f["k"], f["v"], f["bias"], f["keep"], f["g"], f["dout"])
+    for name, got, ref in (("dq", dq, r_dq), ("dk", dk, r_dk), ("dv", dv, r_dv), ("dgate", dg, r_dg)):
+        assert_grad_close(bf16_to_f64_tensor(got), ref, name)
+    assert_grad_close(db.cpu().numpy().astype(np.float64), r_db, "dbias")
