@@ -41,6 +41,14 @@ import pba_inputs as pi  # noqa: E402
 METRIC = "pair-bias attention fwd / fwd+bwd TFLOP/s and %roofline on 1 B200"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 data-sheet figures (dense bf16, HBM3e), reported beside the measured-peak fractions
+NOMINAL_PEAKS = {"hbm": (8000.0, "GB/s"), "tensor": (2250.0, "TFLOP/s")}
+
+
+def nominal(achieved, bound):
+    """The achieved rate as a fraction of the data-sheet peak of its bound."""
+    peak, unit = NOMINAL_PEAKS[bound]
+    return {"peak": peak, "unit": unit, "frac": round(achieved / peak, 4)}
 
 
 # ---------------------------------------------------------------------------------------
@@ -441,7 +449,8 @@ def run_ours(args, cfg):
                 "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
                 "algorithmic_per_launch": {"flops": kf, "bytes": kb},
                 "avg_launch_us": round(avg_s * 1e6, 2),
-                "traffic": ncu_traffic(dom, cfg.name)}
+                "traffic": ncu_traffic(dom, cfg.name),
+                "nominal": nominal(achieved, bound)}
     # the whole step against its own roofline
     t_step_roof = max(step_flops / (tens * 1e12),
                       (w["fwd_bytes"] + w["bwd_bytes"]) / (hbm * 1e9))
@@ -680,7 +689,7 @@ def run_pwa(args, cfg):
                 "frac": round(achieved / peak, 4),
                 "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
                 "algorithmic_per_launch": {"flops": kf, "bytes": kb}, "avg_launch_us": round(avg_s * 1e6, 2),
-                "traffic": ncu_traffic(dom, "pwa-" + cfg.name)}
+                "traffic": ncu_traffic(dom, "pwa-" + cfg.name), "nominal": nominal(achieved, bound)}
     ms_per_step = elapsed_ms / K
     t_step_roof = max(step_flops / (tens * 1e12), (w["fwd_bytes"] + w["bwd_bytes"]) / (hbm * 1e9))
     kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
@@ -831,7 +840,7 @@ def run_pairbias(args, cfg):
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_source": "%s (copy)" % peak_src,
                 "algorithmic_per_launch": {"flops": 0, "bytes": kb}, "avg_launch_us": round(avg_s * 1e6, 2),
-                "traffic": ncu_traffic(dom, "pairbias-" + cfg.name)}
+                "traffic": ncu_traffic(dom, "pairbias-" + cfg.name), "nominal": nominal(achieved, "hbm")}
     ms_per_step = elapsed_ms / K
     kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
                for n, (l, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1])}

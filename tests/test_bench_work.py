@@ -43,3 +43,9 @@ def test_window_pair_mask():
     assert pi.window_pair_mask(5, 7, -1).all()
     d = pi.window_pair_mask(640, 640, 0)
     assert np.array_equal(d, d.T) and d.sum() == 5 * 128 * 128
+
+
+def test_nominal_peak_fractions():
+    import bench
+    assert bench.nominal(4000.0, "hbm") == {"peak": 8000.0, "unit": "GB/s", "frac": 0.5}
+    assert bench.nominal(225.0, "tensor") == {"peak": 2250.0, "unit": "TFLOP/s", "frac": 0.1}
