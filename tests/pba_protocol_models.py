@@ -1,5 +1,5 @@
-"""Randomised models of the barrier protocols of the persistent forward kernel and the
-persistent dq/dk/dv kernel (pba_fwd.cuh, pba_bwd.cuh): every role (TMA producer, MMA
+"""Randomised models of the barrier protocols of the persistent forward kernel, the
+persistent dq/dk/dv kernel and the dbias kernel (pba_fwd.cuh, pba_bwd.cuh): every role (TMA producer, MMA
 issuers, softmax / element-wise warps, epilogue warpgroup) is a generator that waits on
 mbarrier phases exactly as the kernel does; TMA copies and MMAs complete asynchronously in a
 random order (MMAs of one issuer in issue order).  The models check that the protocol never
@@ -457,3 +457,100 @@ class BwdSim:
             idle += 1
             if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
         assert self.epi_done == list(range(self.M)) and self.dq_flushed == list(range(self.T))
+
+
+class DbiasSim:
+    """The dbias kernel (pba_bwd.cuh): one producer fills NS stages (Q, dOa, K and V tiles, row
+    statistics and mask words of one broadcast row each) after the bias tile; one MMA issuer
+    computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; two
+    element-wise warpgroups (128 arrivals each) read the TMEM buffer, the stage's row
+    statistics and mask words, and release both."""
+
+    def __init__(self, nb, NS, seed, plant=None):
+        self.rng = random.Random(seed)
+        self.plant = plant
+        self.nb, self.NS = nb, NS
+        B = Bar
+        self.bias = B("bias", 1)
+        self.full = [B("full%d" % x, 1) for x in range(NS)]
+        self.empty = [B("empty%d" % x, 1 + 256) for x in range(NS)]   # MMA commit + 256 threads
+        self.sd_full = [B("sd_full%d" % x, 1) for x in range(2)]
+        self.sd_free = [B("sd_free%d" % x, 256) for x in range(2)]
+        self.tma, self.mq = [], []
+        self.stage_row = [None] * NS; self.stage_readers = [0] * NS; self.mask_row = [None] * NS
+        self.tm_row = [None, None]; self.tm_readers = [0, 0]; self.tm_pending = [0, 0]
+        self.summed = [[], []]
+
+    def step_async(self):
+        opts = (["tma"] if self.tma else []) + (["mma"] if self.mq else [])
+        if not opts: return
+        if self.rng.choice(opts) == "tma":
+            bar, n, fn = self.tma.pop(self.rng.randrange(len(self.tma)))
+            fn(); bar.complete_tx(n)
+        else:
+            kind, x = self.mq.pop(0)
+            if kind == "mma": x()
+            else: x.arrive()
+
+    def producer(self):
+        self.bias.arrive_tx(1)
+        self.tma.append((self.bias, 1, lambda: None))
+        yield
+        for n in range(self.nb):
+            st = n % self.NS
+            if n >= self.NS and self.plant != "no_empty_wait":
+                while not self.empty[st].test(n // self.NS - 1): yield
+            assert self.stage_readers[st] == 0, "stage refilled while it is read"
+            self.mask_row[st] = n          # plain shared stores, ordered by the arrive below
+            self.stage_row[st] = None
+            self.full[st].arrive_tx(1)
+            self.tma.append((self.full[st], 1, lambda st=st, n=n: self.stage_row.__setitem__(st, n)))
+            yield
+
+    def issuer(self):
+        for n in range(self.nb):
+            st, x = n % self.NS, n & 1
+            while not self.full[st].test(n // self.NS): yield
+            if n >= 2 and self.plant != "no_sd_free_wait":
+                while not self.sd_free[x].test((n >> 1) - 1): yield
+            assert self.stage_row[st] == n
+            self.stage_readers[st] += 1; self.tm_pending[x] += 1
+            def ex(st=st, x=x, n=n):
+                assert self.stage_row[st] == n, "stage changed under the MMA"
+                assert self.tm_readers[x] == 0, "S/dP overwritten while the element-wise warps read them"
+                self.stage_readers[st] -= 1; self.tm_pending[x] -= 1
+                self.tm_row[x] = n
+            self.mq.append(("mma", ex))
+            self.mq.append(("commit", self.sd_full[x]))
+            self.mq.append(("commit", self.empty[st]))
+            yield
+
+    def ew(self, e):
+        while not self.bias.test(0): yield
+        for n in range(self.nb):
+            st, x = n % self.NS, n & 1
+            while not self.sd_full[x].test(n >> 1): yield
+            while not self.full[st].test(n // self.NS): yield
+            assert self.tm_row[x] == n and self.tm_pending[x] == 0
+            assert self.stage_row[st] == n and self.mask_row[st] == n
+            self.tm_readers[x] += 1; self.stage_readers[st] += 1
+            yield
+            assert self.tm_row[x] == n and self.stage_row[st] == n and self.mask_row[st] == n, \
+                "inputs changed under the element-wise warps"
+            self.tm_readers[x] -= 1; self.stage_readers[st] -= 1
+            self.summed[e].append(n)
+            self.sd_free[x].arrive(128); self.empty[st].arrive(128)
+
+    def run(self):
+        live = {"prod": self.producer(), "mma": self.issuer(), "ew0": self.ew(0), "ew1": self.ew(1)}
+        idle = 0
+        while live or self.tma or self.mq:
+            opts = list(live) + (["async"] * 2 if (self.tma or self.mq) else [])
+            c = self.rng.choice(opts)
+            if c == "async":
+                self.step_async(); idle = 0; continue
+            try: next(live[c])
+            except StopIteration: del live[c]
+            idle += 1
+            if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
+        assert self.summed == [list(range(self.nb))] * 2

@@ -3,7 +3,7 @@ many interleavings per configuration, ring and buffer depths as the kernels inst
 and planted mistakes that the checks must catch."""
 import pytest
 
-from pba_protocol_models import BwdSim, FwdSim
+from pba_protocol_models import BwdSim, DbiasSim, FwdSim
 
 
 # ring depths as the forward instantiates them: c=16 -> (3, 2), c=32 -> (2, 2), c=64 -> (2, 1)
@@ -46,3 +46,19 @@ def test_planted_backward_mistakes_are_caught():
     assert _caught(lambda seed: BwdSim(4, 2, 2, 2, 2, 2, seed, plant="no_ps_free_wait"))
     # a dK/dV accumulator reused before its epilogue has read it (one buffer, one step per item)
     assert _caught(lambda seed: BwdSim(4, 1, 2, 2, 2, 1, seed, plant="no_dkv_free_wait"))
+
+
+# dbias kernel stages: c=64 -> 2, otherwise 3
+@pytest.mark.parametrize("NS", [2, 3])
+def test_dbias_protocol(NS):
+    for nb in (0, 1, 2, 3, 4, 7):
+        for seed in range(40):
+            DbiasSim(nb, NS, seed).run()
+
+
+def test_planted_dbias_mistakes_are_caught():
+    # a stage refilled before the MMA and both warpgroups are done with it
+    assert _caught(lambda seed: DbiasSim(6, 2, seed, plant="no_empty_wait"))
+    # S/dP of row n + 2 issued into the TMEM buffer row n is still read from (with two stages
+    # the stage's own empty barrier happens to cover this; with three it does not)
+    assert _caught(lambda seed: DbiasSim(6, 3, seed, plant="no_sd_free_wait"))
