@@ -1,5 +1,6 @@
 """Randomised models of the barrier protocols of the persistent forward kernel, the
-persistent dq/dk/dv kernel and the dbias kernel (pba_fwd.cuh, pba_bwd.cuh): every role (TMA producer, MMA
+persistent dq/dk/dv kernel, the dbias kernel and the pair-weighted averaging GEMM kernel
+(pba_fwd.cuh, pba_bwd.cuh, pba_pwa.cuh): every role (TMA producer, MMA
 issuers, softmax / element-wise warps, epilogue warpgroup) is a generator that waits on
 mbarrier phases exactly as the kernel does; TMA copies and MMAs complete asynchronously in a
 random order (MMAs of one issuer in issue order).  The models check that the protocol never
@@ -554,3 +555,80 @@ class DbiasSim:
             idle += 1
             if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
         assert self.summed == [list(range(self.nb))] * 2
+
+
+class PwaGemmSim:
+    """The pair-weighted averaging GEMM kernel (pba_pwa.cuh): one producer fills NS stages
+    (a 64-deep block of w and the chunk's value tiles) over the nK reduction stages; one MMA
+    issuer accumulates every stage into one TMEM accumulator, releases each stage by a commit
+    and signals the epilogue by a last commit; the epilogue reads the accumulator once."""
+
+    def __init__(self, nK, NS, seed, plant=None):
+        self.rng = random.Random(seed)
+        self.plant = plant
+        self.nK, self.NS = nK, NS
+        self.full = [Bar("full%d" % x, 1) for x in range(NS)]
+        self.empty = [Bar("empty%d" % x, 1) for x in range(NS)]
+        self.done = Bar("done", 1)
+        self.tma, self.mq = [], []
+        self.stage = [None] * NS; self.readers = [0] * NS
+        self.acc = []          # reduction stages added to the accumulator, in order
+        self.read = None
+
+    def step_async(self):
+        opts = (["tma"] if self.tma else []) + (["mma"] if self.mq else [])
+        if not opts: return
+        if self.rng.choice(opts) == "tma":
+            bar, n, fn = self.tma.pop(self.rng.randrange(len(self.tma)))
+            fn(); bar.complete_tx(n)
+        else:
+            kind, x = self.mq.pop(0)
+            if kind == "mma": x()
+            else: x.arrive()
+
+    def producer(self):
+        for r in range(self.nK):
+            st = r % self.NS
+            if r >= self.NS and self.plant != "no_empty_wait":
+                while not self.empty[st].test(r // self.NS - 1): yield
+            assert self.readers[st] == 0, "stage refilled while the MMA reads it"
+            self.stage[st] = None
+            self.full[st].arrive_tx(1)
+            self.tma.append((self.full[st], 1, lambda st=st, r=r: self.stage.__setitem__(st, r)))
+            yield
+
+    def issuer(self):
+        for r in range(self.nK):
+            st = r % self.NS
+            while not self.full[st].test(r // self.NS): yield
+            assert self.stage[st] == r
+            self.readers[st] += 1
+            def ex(st=st, r=r):
+                assert self.stage[st] == r, "stage changed under the MMA"
+                self.readers[st] -= 1
+                self.acc.append(r)
+            self.mq.append(("mma", ex))
+            self.mq.append(("commit", self.empty[st]))
+            yield
+        if self.plant != "early_done":
+            self.mq.append(("commit", self.done))
+        else:
+            self.mq.insert(0, ("commit", self.done))
+
+    def epilogue(self):
+        while not self.done.test(0): yield
+        self.read = list(self.acc)
+
+    def run(self):
+        live = {"prod": self.producer(), "mma": self.issuer(), "epi": self.epilogue()}
+        idle = 0
+        while live or self.tma or self.mq:
+            opts = list(live) + (["async"] * 2 if (self.tma or self.mq) else [])
+            c = self.rng.choice(opts)
+            if c == "async":
+                self.step_async(); idle = 0; continue
+            try: next(live[c])
+            except StopIteration: del live[c]
+            idle += 1
+            if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
+        assert self.read == list(range(self.nK)), "the epilogue read an unfinished accumulator"

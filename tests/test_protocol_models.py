@@ -3,7 +3,7 @@ many interleavings per configuration, ring and buffer depths as the kernels inst
 and planted mistakes that the checks must catch."""
 import pytest
 
-from pba_protocol_models import BwdSim, DbiasSim, FwdSim
+from pba_protocol_models import BwdSim, DbiasSim, FwdSim, PwaGemmSim
 
 
 # ring depths as the forward instantiates them: c=16 -> (3, 2), c=32 -> (2, 2), c=64 -> (2, 1)
@@ -62,3 +62,15 @@ def test_planted_dbias_mistakes_are_caught():
     # S/dP of row n + 2 issued into the TMEM buffer row n is still read from (with two stages
     # the stage's own empty barrier happens to cover this; with three it does not)
     assert _caught(lambda seed: DbiasSim(6, 3, seed, plant="no_sd_free_wait"))
+
+
+def test_pwa_gemm_protocol():
+    for nK in (1, 2, 3, 4, 7):
+        for seed in range(40):
+            PwaGemmSim(nK, 2, seed).run()
+
+
+def test_planted_pwa_gemm_mistakes_are_caught():
+    assert _caught(lambda seed: PwaGemmSim(5, 2, seed, plant="no_empty_wait"))
+    # the epilogue signalled before the last products are done
+    assert _caught(lambda seed: PwaGemmSim(5, 2, seed, plant="early_done"))
