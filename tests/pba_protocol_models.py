@@ -558,8 +558,9 @@ class DbiasSim:
 
 
 class PwaGemmSim:
-    """The pair-weighted averaging GEMM kernel (pba_pwa.cuh): one producer fills NS stages
-    (a 64-deep block of w and the chunk's value tiles) over the nK reduction stages; one MMA
+    """The pair-weighted averaging GEMM and dW kernels (pba_pwa.cuh, one protocol): one producer
+    fills NS stages (GEMM: a 64-deep block of w and the chunk's value tiles; dW: one row's dOa
+    and V tiles) over the nK reduction stages; one MMA
     issuer accumulates every stage into one TMEM accumulator, releases each stage by a commit
     and signals the epilogue by a last commit; the epilogue reads the accumulator once."""
 
