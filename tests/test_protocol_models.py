@@ -64,10 +64,12 @@ def test_planted_dbias_mistakes_are_caught():
     assert _caught(lambda seed: DbiasSim(6, 3, seed, plant="no_sd_free_wait"))
 
 
-def test_pwa_gemm_protocol():
-    for nK in (1, 2, 3, 4, 7):
+# GEMM: 2 stages; dW: 4 stages (and possibly no rows in a split)
+@pytest.mark.parametrize("NS", [2, 4])
+def test_pwa_gemm_protocol(NS):
+    for nK in (0, 1, 2, 3, 4, 5, 9):
         for seed in range(40):
-            PwaGemmSim(nK, 2, seed).run()
+            PwaGemmSim(nK, NS, seed).run()
 
 
 def test_planted_pwa_gemm_mistakes_are_caught():
