@@ -126,14 +126,50 @@ def _code_only(text: str) -> str:
     return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
 
 
+def _without_other_kernels(code: str, kernel: str) -> str:
+    """`code` without the definitions of its __global__ functions other than `kernel`
+    (helpers, structures and the kernel itself stay); the whole of `code` if it cannot be
+    parsed."""
+    import re
+    try:
+        out, pos = [], 0
+        for m in re.finditer(r"__global__\s+void\s+(?:__launch_bounds__\s*\([^)]*\)\s*)?(\w+)\s*\(", code):
+            i, depth = m.end(), 1
+            while depth:                      # the parameter list
+                depth += (code[i] == "(") - (code[i] == ")")
+                i += 1
+            k = code.index("{", i) + 1
+            depth = 1
+            while depth:                      # the body
+                depth += (code[k] == "{") - (code[k] == "}")
+                k += 1
+            if m.group(1) != kernel:
+                out.append(code[pos:m.start()])
+                pos = k
+        out.append(code[pos:])
+        return "".join(out)
+    except (IndexError, ValueError):
+        return code
+
+
+def kernel_code(text: str, kernel: str) -> str:
+    """The part of a source file's text that one kernel is compiled from: no comments, and
+    none of the other kernels defined beside it (`kernel` may carry a suffix, e.g.
+    "pba_pwa_gemm_kernel (dv)")."""
+    return _without_other_kernels(_code_only(text), kernel.split()[0].split("<")[0])
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the code one kernel is compiled from: its own file and the shared device
-    header, comments left out (launch configuration in the API file is not covered)."""
+    """Hash of the code one kernel is compiled from: its own definition with the helpers of
+    its file, and the shared device header, comments left out (launch configuration in the
+    API file is not covered)."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc")
     for name in (kernel_source_file(kernel), "pba_device.cuh"):
         with open(os.path.join(cdir, name), encoding="utf-8") as fh:
-            h.update(name.encode() + _code_only(fh.read()).encode())
+            text = fh.read()
+        code = kernel_code(text, kernel) if name != "pba_device.cuh" else _code_only(text)
+        h.update(name.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

@@ -969,24 +969,63 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // Only the tile's valid part (rows i < Nq, four-key groups starting below Nk) is summed,
+    // four positions per thread at a time.  Every position adds its partials in split order,
+    // starting from zero; the loads of four splits of the four positions are all issued
+    // before their additions, so their latencies overlap.
     const long long plane = (long long)a.H * a.ntiles * 128 * 128;
-    for (int v = threadIdx.x; v < 128 * 32; v += blockDim.x) {
-        const int i = i0 + (v >> 5), j = j0 + (v & 31) * 4;
-        if (i >= a.Nq || j >= a.Nk) continue;
-        const float *src = a.dbias_part + (((long long)h * a.ntiles + bt) * 128 + (i - i0)) * 128 + (j - j0);
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < a.splits; ++q) {
-            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + q * plane));
-            sum.x += v4.x;
-            sum.y += v4.y;
-            sum.z += v4.z;
-            sum.w += v4.w;
+    const float *part = a.dbias_part + ((long long)h * a.ntiles + bt) * 128 * 128;
+    const int groups = (min(128, a.Nk - j0) + 3) >> 2;
+    const int nv = min(128, a.Nq - i0) * groups;
+    for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * blockDim.x) {
+        int off[4];   // row * 128 + column within the tile, or -1
+        float4 sum[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = v0 + u * blockDim.x;
+            off[u] = v < nv ? (v / groups) * 128 + (v % groups) * 4 : -1;
+            sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        float *dst = a.dbias + ((long long)h * a.Nq + i) * a.Nk + j;
-        dst[0] = sum.x;
-        if (j + 1 < a.Nk) dst[1] = sum.y;
-        if (j + 2 < a.Nk) dst[2] = sum.z;
-        if (j + 3 < a.Nk) dst[3] = sum.w;
+        int q = 0;
+        for (; q + 4 <= a.splits; q += 4) {
+            float4 x[4][4];
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    x[s][u] = off[u] >= 0 ? __ldcg(reinterpret_cast<const float4 *>(part + (q + s) * plane + off[u]))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    sum[u].x += x[s][u].x;
+                    sum[u].y += x[s][u].y;
+                    sum[u].z += x[s][u].z;
+                    sum[u].w += x[s][u].w;
+                }
+        }
+        for (; q < a.splits; ++q) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (off[u] < 0) continue;
+                const float4 x = __ldcg(reinterpret_cast<const float4 *>(part + q * plane + off[u]));
+                sum[u].x += x.x;
+                sum[u].y += x.y;
+                sum[u].z += x.z;
+                sum[u].w += x.w;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (off[u] < 0) continue;
+            const int i = i0 + (off[u] >> 7), j = j0 + (off[u] & 127);
+            float *dst = a.dbias + ((long long)h * a.Nq + i) * a.Nk + j;
+            dst[0] = sum[u].x;
+            if (j + 1 < a.Nk) dst[1] = sum[u].y;
+            if (j + 2 < a.Nk) dst[2] = sum[u].z;
+            if (j + 3 < a.Nk) dst[3] = sum[u].w;
+        }
     }
 }
 

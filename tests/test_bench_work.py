@@ -49,3 +49,25 @@ def test_nominal_peak_fractions():
     import bench
     assert bench.nominal(4000.0, "hbm") == {"peak": 8000.0, "unit": "GB/s", "frac": 0.5}
     assert bench.nominal(225.0, "tensor") == {"peak": 2250.0, "unit": "TFLOP/s", "frac": 0.1}
+
+
+def test_kernel_code_keeps_one_kernel_and_its_helpers():
+    import bench
+    path = os.path.join(ROOT, "pair_biased_attention_gated_b200", "csrc", "pba_bwd.cuh")
+    with open(path) as fh:
+        text = fh.read()
+    main = bench.kernel_code(text, "pba_bwd_main_kernel")
+    dbias = bench.kernel_code(text, "pba_dbias_kernel")
+    assert "pba_bwd_main_kernel(" in main and "pba_dbias_kernel(" not in main
+    assert "pba_dbias_kernel(" in dbias and "pba_bwd_main_kernel(" not in dbias
+    assert "struct BwdArgs" in main and "struct BwdArgs" in dbias   # shared helpers stay
+    # a change inside one kernel's body changes its code only; a comment changes nothing
+    marker = "if (!s_last) return;"
+    assert text.count(marker) == 1
+    edited = text.replace(marker, "if (!s_last) { return; }")
+    assert bench.kernel_code(edited, "pba_dbias_kernel") != dbias
+    assert bench.kernel_code(edited, "pba_bwd_main_kernel") == main
+    assert bench.kernel_code(text + "\n// a note\n", "pba_dbias_kernel") == dbias
+    # text that cannot be parsed is kept whole
+    broken = "__global__ void k(int a { x"
+    assert bench.kernel_code(broken, "other") == bench._code_only(broken)
