@@ -135,8 +135,8 @@ pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v
                          int window, void *stream);
 
 /*
- * Backward pass for callers that cannot allocate device memory.  The paper has no
- * counterpart: this entry point exists for users of the library, not for the method.
+ * Backward pass for callers that cannot allocate device memory.  The method's sources have
+ * no counterpart: this entry point exists for users of the library, not for the method.
  * Some callers have no way to obtain scratch memory: a plugin running inside another
  * framework's executor that owns all device memory and forbids cudaMalloc while it
  * runs, or a binding from a language with no device allocator.  This variant takes the
