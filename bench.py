@@ -2,13 +2,20 @@
 """Benchmark of pair-biased gated attention on B200: fwd+bwd TFLOP/s and % of roofline.
 
 A step is one pass of the whole hot path: the forward kernel (out, lse) and the backward
-kernels (dq, dk, dv, dgate, dbias) over one batch of synthetic, seeded bf16 input shaped
-like the MSA row attention workload (128 MSA rows share one [8, 256, 256] pair bias;
-`--config` selects another workload).  Inputs are resident in HBM when the timed region
-starts; L2 is flushed before every timed step, outside the timed events.
+kernels (dq, dk, dv, dgate, dbias) over one batch of synthetic, seeded bf16 input.  The
+default workload is the large triangle attention (768 rows x 768 keys, 4 heads, c = 32,
+the largest workload that the target names and that fits one GPU); `--config` selects
+another.  Inputs are resident in HBM when the timed region starts; L2 is flushed before
+every timed step, outside the timed events.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
-                  [--op attention|pwa|pairbias]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C5] [--impl ours|reference]
+                  [--op attention|pwa|pairbias] [--also C1,C2,C3,C4]
+
+The line reports the whole step (value, step_roofline), the dominant kernel's roofline,
+each pass's roofline fraction (fwd_roofline_frac, bwd_roofline_frac), and under
+`workloads` the same per-pass figures for the other workloads (`--also`, device timing
+only).  Tensor-bound fractions use the burst bf16 peak (kernels timed per launch); the
+sustained peak is reported beside it.
 
 N > 1 runs under torchrun, one process per GPU, each an independent replica of the
 workload (the path has no exchange step); rank 0 prints one JSON line.  `--impl
@@ -105,6 +112,85 @@ def load_peaks():
             d = json.load(fh)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def peak_rates(peaks):
+    """(HBM GB/s, burst bf16 TFLOP/s, sustained bf16 TFLOP/s).  The kernels are timed per
+    launch, each well under a millisecond, so a tensor-bound fraction is taken against the
+    burst figure; the sustained one is reported beside it."""
+    tens = float(peaks["bf16_tflops"])
+    return float(peaks["hbm_gbs"]), tens, float(peaks.get("bf16_tflops_sustained", tens))
+
+
+BWD_KERNELS = ("pba_bwd_pre_kernel", "pba_bwd_main_kernel", "pba_dbias_kernel",
+               "pba_dbias_zero_kernel", "pba_dq_convert_kernel")
+
+
+def pass_figures(w, kstats, steps, hbm, tens):
+    """Per-pass device time (the library's event timing of each kernel) and roofline
+    fraction: roofline time = max(flops / tensor peak, bytes / HBM peak) of the pass."""
+    fwd_ms = kstats.get("pba_fwd_kernel", (steps, 0.0))[1] / steps
+    bwd_ms = sum(kstats.get(k, (steps, 0.0))[1] for k in BWD_KERNELS) / steps
+    out = {}
+    for name, ms, fl, by in (("fwd", fwd_ms, w["fwd_flops"], w["fwd_bytes"]),
+                             ("bwd", bwd_ms, w["bwd_flops"], w["bwd_bytes"])):
+        t_roof = max(fl / (tens * 1e12), by / (hbm * 1e9))
+        out[name + "_us"] = round(ms * 1e3, 2) if ms > 0 else None
+        out[name + "_tflops"] = round(fl / (ms / 1e3) / 1e12, 3) if ms > 0 else None
+        out[name + "_roofline_us"] = round(t_roof * 1e6, 2)
+        out[name + "_roofline_bound"] = "tensor" if fl / (tens * 1e12) > by / (hbm * 1e9) else "hbm"
+        out[name + "_roofline_frac"] = round(t_roof * 1e3 / ms, 4) if ms > 0 else None
+    return out
+
+
+def time_workload(pba, cfg, args):
+    """Device timing of one more workload (fwd + bwd step, L2 flushed before each step):
+    per-pass time, TFLOP/s and roofline fraction from the library's per-kernel events."""
+    import torch
+    d = pi.make_inputs(cfg, seed=args.seed)
+    t = {}
+    for k, a in d.items():
+        t[k] = (torch.from_numpy(np.ascontiguousarray(a)) if k == "keep" else
+                torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)).cuda()
+    q, kk, v, g, bias, keep, dout = t["q"], t["k"], t["v"], t.get("g"), t["bias"], t["keep"], t["dout"]
+    B, N, H, C = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(kk), torch.empty_like(v)
+    dg = torch.empty_like(g) if g is not None else None
+    db = torch.empty(H, N, N, dtype=torch.float32, device="cuda")
+    dims = pba.make_dims(q, kk, v, g, out, bias, keep)
+    ws = torch.empty(pba.pba_bwd_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step():
+        pba.pba_fwd(q, kk, v, bias, keep, g, out, lse, window=cfg.window)
+        pba.pba_bwd(q, kk, v, bias, keep, g, out, lse, dout, dq, dk, dv, db, dg, ws, window=cfg.window)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    pba.pba_device_status()
+    K = max(3, min(args.steps, 20))
+    torch.cuda.synchronize()
+    pba.profile_read()
+    pba.profile_enable(True)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    pba.profile_enable(False)
+    kstats = pba.profile_read()
+    pba.pba_device_status()
+    peaks, _ = load_peaks()
+    hbm, tens, _ = peak_rates(peaks)
+    w = work(cfg)
+    res = {"workload": cfg.desc, "passes_named": "fwd+bwd" if cfg.passes == "fwdbwd" else "fwd",
+           "steps": K, **pass_figures(w, kstats, K, hbm, tens),
+           "kernels_us": {n: round(ms / l * 1e3, 2) for n, (l, ms) in kstats.items()}}
+    del q, kk, v, g, bias, keep, dout, out, lse, dq, dk, dv, dg, db, ws, flush, t
+    torch.cuda.empty_cache()
+    return res
 
 
 KERNEL_SOURCES = {"pba_fwd_kernel": "pba_fwd.cuh"}   # every other attention kernel: pba_bwd.cuh
@@ -465,8 +551,7 @@ def run_ours(args, cfg):
     e2e_value = job_throughput(world, step_flops, K2, e2e_ms) / 1e12
 
     peaks, peak_src = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    tens = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    hbm, tens, tens_sus = peak_rates(peaks)
     # dominant kernel and its roofline
     total_k = sum(ms for _, ms in kstats.values()) or 1.0
     dom = max(kstats.items(), key=lambda kv: kv[1][1])[0] if kstats else None
@@ -482,16 +567,17 @@ def run_ours(args, cfg):
             achieved, peak, unit, bound = kb / avg_s / 1e9, hbm, "GB/s", "hbm"
         roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
                 "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
-                "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
+                "peak_source": "%s (%s)" % (peak_src, "burst bf16" if bound == "tensor" else "copy"),
                 "algorithmic_per_launch": {"flops": kf, "bytes": kb},
                 "avg_launch_us": round(avg_s * 1e6, 2),
                 "traffic": ncu_traffic(dom, cfg.name),
                 "nominal": nominal(achieved, bound)}
+        if bound == "tensor":
+            roof["sustained"] = {"peak": tens_sus, "frac": round(achieved / tens_sus, 4)}
     # the whole step against its own roofline
     t_step_roof = max(step_flops / (tens * 1e12),
                       (w["fwd_bytes"] + w["bwd_bytes"]) / (hbm * 1e9))
     ms_per_step = elapsed_ms / K
-    fwd_ms = kstats.get("pba_fwd_kernel", (K, 0.0))[1] / K
     kernels = {n: {"launches": l, "avg_us": round(ms / l * 1e3, 2), "share": round(ms / total_k, 4)}
                for n, (l, ms) in sorted(kstats.items(), key=lambda kv: -kv[1][1])}
     launches_total = sum(l for l, _ in kstats.values())
@@ -510,16 +596,17 @@ def run_ours(args, cfg):
         "roofline": roof,
         "step_roofline": {"time_us": round(t_step_roof * 1e6, 2),
                           "frac": round(t_step_roof * 1e3 / ms_per_step, 4)},
-        "fwd_tflops": round(w["fwd_flops"] / (fwd_ms / 1e3) / 1e12, 3) if fwd_ms > 0 else None,
-        "fwd_roofline_frac": round(max(w["fwd_flops"] / (tens * 1e12),
-                                       w["fwd_bytes"] / (hbm * 1e9)) * 1e3 / fwd_ms, 4)
-        if fwd_ms > 0 else None,
+        **pass_figures(w, kstats, K, hbm, tens),
         "kernels": kernels,
         "gpu_launches": launches_total,
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2},
     }
+    if world == 1 and args.also:
+        res["workloads"] = {}
+        for name in [x for x in args.also.split(",") if x and x != cfg.name]:
+            res["workloads"][name] = time_workload(pba, pi.CONFIGS[name], args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = time_oracle(cfg, target_s=args.cpu_seconds, seed=args.seed)
     if pg:
@@ -708,8 +795,7 @@ def run_pwa(args, cfg):
     step_flops = w["fwd_flops"] + w["bwd_flops"]
     value = step_flops * K / (elapsed_ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    tens = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    hbm, tens, _ = peak_rates(peaks)
     total_k = sum(ms for _, ms in kstats.values()) or 1.0
     dom = max(kstats.items(), key=lambda kv: kv[1][1])[0] if kstats else None
     roof = None
@@ -723,7 +809,7 @@ def run_pwa(args, cfg):
             achieved, peak, unit, bound = kb / avg_s / 1e9, hbm, "GB/s", "hbm"
         roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                 "frac": round(achieved / peak, 4),
-                "peak_source": "%s (%s)" % (peak_src, "sustained bf16" if bound == "tensor" else "copy"),
+                "peak_source": "%s (%s)" % (peak_src, "burst bf16" if bound == "tensor" else "copy"),
                 "algorithmic_per_launch": {"flops": kf, "bytes": kb}, "avg_launch_us": round(avg_s * 1e6, 2),
                 "traffic": ncu_traffic(dom, "pwa-" + cfg.name), "nominal": nominal(achieved, bound)}
     ms_per_step = elapsed_ms / K
@@ -907,12 +993,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="C2", choices=sorted(pi.CONFIGS))
+    ap.add_argument("--config", default="C5", choices=sorted(pi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", default="C1,C2,C3,C4",
+                    help="other workloads whose per-pass device times and roofline fractions are "
+                         "added under `workloads` (one GPU; empty: none)")
     ap.add_argument("--op", default="attention", choices=["attention", "pwa", "pairbias"],
                     help="pwa: MSA pair-weighted averaging of the workload's value rows; pairbias: "
                          "the LayerNorm + projection that makes the workload's bias (one GPU each)")

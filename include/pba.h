@@ -143,11 +143,15 @@ pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v
  * same arguments as pba_bwd except the workspace, and uses instead a scratch array built
  * into the library (64 MiB in device global memory, held by every GPU that loads the
  * library until the process exits).  It allocates nothing: no cudaMalloc, no cudaFree.
- *  - Sizes whose workspace (pba_bwd_workspace_size) exceeds 64 MiB are rejected with
- *    PBA_ERR_UNSUPPORTED before anything is launched; use pba_bwd for those.
- *  - The first call on a device looks up the scratch array's device address with that
- *    device current (one cudaGetSymbolAddress per device); make that first call before
- *    any stream capture.
+ *  - Arguments are checked exactly as pba_bwd checks them (PBA_ERR_INVALID_ARG and the
+ *    like come first); then sizes whose workspace (pba_bwd_workspace_size) exceeds 64 MiB
+ *    are rejected with PBA_ERR_UNSUPPORTED before anything is launched; use pba_bwd for
+ *    those.
+ *  - The first call in a CUDA context looks up the scratch array's device address in that
+ *    context (one cudaGetSymbolAddress, with the calling thread's current device and
+ *    context) and keeps it under the context's unique id, so a context created later (a
+ *    second context on the device, or the one after cudaDeviceReset) gets its own lookup.
+ *    Make the first call in each context before any stream capture.
  *  - Every call on a device shares the one array and leaves the last call's contents in
  *    it (the parts that must start at zero are cleared by each call).  Calls whose
  *    execution overlaps on the GPU (different streams, no ordering between them) race on

@@ -527,26 +527,62 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
 // ---------------------------------------------------------------------------- no-alloc
 // Scratch of pba_bwd_noalloc: a file-scope device array, so callers that cannot allocate
 // can still run the backward pass.  In host code its name is only a stand-in; the
-// device address comes from cudaGetSymbolAddress, looked up once per device.
+// device address comes from cudaGetSymbolAddress.  A __device__ symbol's address belongs
+// to the CUDA context that loaded the module, so it is looked up once per context (the
+// first call in a context, with that context's device current) and cached under the
+// context's unique id, which a re-created context (after cudaDeviceReset, or another
+// context on the same device) does not share.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 __device__ __align__(256) unsigned char g_pba_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
-std::vector<void *> g_noalloc_addr;  // per device ordinal; nullptr until looked up
+std::vector<std::pair<unsigned long long, void *>> g_noalloc_addr;   // (context id, address)
+
+typedef CUresult (*PFN_ctxGetCurrent)(CUcontext *);
+typedef CUresult (*PFN_ctxGetId)(CUcontext, unsigned long long *);
+
+pba_status current_context_id(unsigned long long *id) {
+    static PFN_ctxGetCurrent get_cur = nullptr;
+    static PFN_ctxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<PFN_ctxGetCurrent>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_ctxGetId>(fn);
+    });
+    if (!get_cur || !get_id) return fail(PBA_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId unavailable");
+    CUcontext ctx = nullptr;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return fail(PBA_ERR_CUDA, "no current CUDA context");
+    if (get_id(ctx, id) != CUDA_SUCCESS) return fail(PBA_ERR_CUDA, "cuCtxGetId failed");
+    return PBA_OK;
+}
 
 pba_status noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    // makes the device's primary context current if the caller has none yet
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    unsigned long long ctx_id = 0;
+    pba_status st = current_context_id(&ctx_id);
+    if (st != PBA_OK) return st;
     std::lock_guard<std::mutex> g(g_noalloc_mu);
-    if ((int)g_noalloc_addr.size() <= dev) g_noalloc_addr.resize(dev + 1, nullptr);
-    if (!g_noalloc_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_pba_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    for (const auto &ent : g_noalloc_addr)
+        if (ent.first == ctx_id) {
+            *out = ent.second;
+            return PBA_OK;
+        }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_pba_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+    g_noalloc_addr.emplace_back(ctx_id, p);
+    *out = p;
     return PBA_OK;
 }
 
@@ -953,26 +989,22 @@ pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                          workspace, workspace_bytes, d, -1, stream);
 }
 
-pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
-                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
-                         const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
-                         pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
-                         void *workspace, size_t workspace_bytes, const pba_dims *d, int window,
-                         void *stream) {
-    g_last_error.clear();
+// Every check of the backward's arguments except the workspace: shared by pba_bwd_local and
+// pba_bwd_noalloc, so both report an argument error before any question of scratch size.
+pba_status check_bwd_args(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                          const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                          const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                          pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, pba_bf16 *dgate,
+                          const pba_dims *d, int window) {
     pba_status st = check_dims(d);
     if (st != PBA_OK) return st;
     if ((st = check_window(d, window)) != PBA_OK) return st;
     if (d->B == 0) return PBA_OK;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d->Nq == 0) {
-        // no query: every key gradient is zero, there is no dq, dgate or dbias element
         if (d->Nk == 0) return PBA_OK;
         if (!dk || !dv) return fail(PBA_ERR_INVALID_ARG, "dk and dv are required");
         if ((st = check_strides(d->sk, d->B, d->Nk, d->H, "k")) != PBA_OK) return st;
-        if ((st = check_strides(d->sv, d->B, d->Nk, d->H, "v")) != PBA_OK) return st;
-        if ((st = get_encoder()) != PBA_OK) return st;  // (keeps error handling uniform)
-        return launch_zero_rows(dk, dv, d, s);
+        return check_strides(d->sv, d->B, d->Nk, d->H, "v");
     }
     if ((st = check_layouts(d)) != PBA_OK) return st;
     if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
@@ -991,6 +1023,26 @@ pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v
         if ((st = check_bias(d)) != PBA_OK) return st;
     }
     if (key_mask && d->smask_b < 0) return fail(PBA_ERR_INVALID_ARG, "smask_b must be >= 0");
+    return PBA_OK;
+}
+
+pba_status pba_bwd_local(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
+                         const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
+                         const pba_bf16 *out, const float *lse, const pba_bf16 *dout,
+                         pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias, pba_bf16 *dgate,
+                         void *workspace, size_t workspace_bytes, const pba_dims *d, int window,
+                         void *stream) {
+    g_last_error.clear();
+    pba_status st = check_bwd_args(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dgate, d, window);
+    if (st != PBA_OK) return st;
+    if (d->B == 0) return PBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d->Nq == 0) {
+        // no query: every key gradient is zero, there is no dq, dgate or dbias element
+        if (d->Nk == 0) return PBA_OK;
+        if ((st = get_encoder()) != PBA_OK) return st;  // (keeps error handling uniform)
+        return launch_zero_rows(dk, dv, d, s);
+    }
     const BwdPlan pl = plan_bwd(d, window);
     if (!workspace || workspace_bytes < pl.total)
         return fail(PBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
@@ -1014,14 +1066,17 @@ pba_status pba_bwd_noalloc(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 
                            pba_bf16 *dq, pba_bf16 *dk, pba_bf16 *dv, float *dbias,
                            pba_bf16 *dgate, const pba_dims *d, void *stream) {
     g_last_error.clear();
-    pba_status st = check_dims(d);
+    // the same argument checks as pba_bwd first, then the scratch size
+    pba_status st = check_bwd_args(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dgate, d, -1);
     if (st != PBA_OK) return st;
-    const size_t need = plan_bwd(d).total;
-    if (need > kNoAllocScratchBytes)
-        return fail(PBA_ERR_UNSUPPORTED,
-                    "pba_bwd_noalloc: these sizes need %zu bytes of scratch, more than the %zu "
-                    "built into the library; call pba_bwd with a workspace instead",
-                    need, kNoAllocScratchBytes);
+    if (d->B > 0 && d->Nq > 0) {
+        const size_t need = plan_bwd(d).total;
+        if (need > kNoAllocScratchBytes)
+            return fail(PBA_ERR_UNSUPPORTED,
+                        "pba_bwd_noalloc: these sizes need %zu bytes of scratch, more than the %zu "
+                        "built into the library; call pba_bwd with a workspace instead",
+                        need, kNoAllocScratchBytes);
+    }
     void *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != PBA_OK) return st;
     return pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,

@@ -203,3 +203,27 @@ def test_bwd_full_config_sampled(pba, cfg_name):
     row_sums = db.double().sum(-1).abs()
     bound = (t["dout"].double() * out.double()).abs().sum(dim=(0, 3)).transpose(0, 1) * 2.0 ** -8
     assert bool((row_sums <= bound + 1e-6).all()), float((row_sums - bound).max())
+
+
+def test_dbias_whole_head_large_triangle(pba):
+    """Large triangle attention (768 rows x 768 keys, 4 heads, c = 32), the benchmark's
+    launch configuration: every one of the 768 dbias rows of head 0 (each the sum of dS over
+    all 768 broadcast rows) compared against the oracle, row by row and as a whole."""
+    from concurrent.futures import ThreadPoolExecutor
+    cfg = pi.CONFIGS["C5"]
+    d = pi.make_inputs(cfg, seed=0)
+    t = to_dev(d)
+    _, _, (_, _, _, _, db) = _gpu_fwd_bwd(pba, t)
+    h = 0
+    hs = lambda a: pi.bf16_bits_to_f64(a[:, :, h:h + 1])
+    args = (hs(d["q"]), hs(d["k"]), hs(d["v"]), pi.bf16_bits_to_f64(d["bias"][h:h + 1]), d["keep"],
+            hs(d["g"]), hs(d["dout"]))
+    # the oracle's C entry point runs without the GIL: one row per task
+    with ThreadPoolExecutor(max_workers=max(1, min(32, oracle.threads()))) as ex:
+        rows = list(ex.map(lambda i: oracle.dbias_row(*args, 0, i), range(cfg.N)))
+    ref = np.stack(rows)
+    got = db[h].cpu().numpy().astype(np.float64)
+    assert rel_l2(got, ref) <= GRAD_REL_L2, "dbias head 0 rel L2 %.3g" % rel_l2(got, ref)
+    worst = max(range(cfg.N), key=lambda i: rel_l2(got[i], ref[i]))
+    assert rel_l2(got[worst], ref[worst]) <= GRAD_REL_L2, \
+        "dbias[0,%d] rel L2 %.3g" % (worst, rel_l2(got[worst], ref[worst]))
