@@ -245,6 +245,21 @@ pba_status pba_pair_bias_bwd(const pba_bf16 *z, const float *gamma, const float 
                              void *stream);
 
 /*
+ * Ordered sum of bias-gradient partials, for the row-sharded backward pass across GPUs.
+ * The Design-CP page ("Context Parallelism for Design of Protein Nanoparticles", Method)
+ * shards each attention block's rows over GPUs and exchanges activations between blocks;
+ * for pair-biased attention the bias gradient is a sum over the broadcast rows
+ * ("AlphaFold3 open-source implementation" page, Model Efficiency), so row shards each
+ * hold a partial of it.  Given n_parts partials of n fp32 elements each, stored one after
+ * the other in `parts` (device memory, part p at parts + p * n), writes
+ *   out[i] = (...((parts[0][i] + parts[1][i]) + parts[2][i]) ... + parts[n_parts-1][i])
+ * in exactly that order, so the result depends only on the partials and their order, not
+ * on which GPU computed which.  `out` may not overlap `parts`.  n_parts >= 1, n >= 0;
+ * pointers 16-byte aligned.  Asynchronous on `stream`; allocates nothing.
+ */
+pba_status pba_dbias_sum(const float *parts, int n_parts, int64_t n, float *out, void *stream);
+
+/*
  * Synchronizes `stream`, then reports and clears the device watchdog word of the
  * current device: PBA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, PBA_ERR_CUDA if the synchronization itself failed, else PBA_OK.

@@ -75,6 +75,8 @@ lib.pba_pair_bias_bwd_workspace_size.argtypes = [ctypes.POINTER(PbaPairBiasDims)
 lib.pba_pair_bias_bwd_workspace_size.restype = ctypes.c_size_t
 lib.pba_pair_bias_bwd.argtypes = [_vp] * 10 + [ctypes.c_size_t, ctypes.POINTER(PbaPairBiasDims), _vp]
 lib.pba_pair_bias_bwd.restype = ctypes.c_int
+lib.pba_dbias_sum.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, _vp, _vp]
+lib.pba_dbias_sum.restype = ctypes.c_int
 lib.pba_device_status.argtypes = [_vp]
 lib.pba_device_status.restype = ctypes.c_int
 lib.pba_status_string.argtypes = [ctypes.c_int]

@@ -45,7 +45,7 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 // ---------------------------------------------------------------------------- profiling
 enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS,
                 K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS,
-                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_DBIAS_ZERO, K_COUNT };
+                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_DBIAS_ZERO, K_DBIAS_SUM, K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
                                            "pba_dbias_kernel",
                                            "pba_dq_convert_kernel", "zero_rows_kernel",
@@ -54,7 +54,7 @@ const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel
                                            "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel",
                                            "pba_pair_bias_fwd_kernel", "pba_pair_bias_bwd_kernel",
                                            "pba_pair_bias_reduce_kernel", "pba_pair_bias_param_kernel",
-                                           "pba_dbias_zero_kernel"};
+                                           "pba_dbias_zero_kernel", "pba_dbias_sum_kernel"};
 struct ProfRec {
     int kid;
     cudaEvent_t a, b;
@@ -275,20 +275,15 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.lse = lse;
     a.skip_step = g_debug_skip_step;
     a.win = win;
-    if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
-    // two CTAs per SM need (almost) all of the unified L1 / shared memory as shared memory
-    cudaError_t ce = cudaFuncSetAttribute(pba::pba_fwd_kernel<CP>,
-                                          cudaFuncAttributePreferredSharedMemoryCarveout,
-                                          cudaSharedmemCarveoutMaxShared);
-    if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute (carveout)");
+    if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_LAUNCH)) != PBA_OK) return st;
     const long long items = tiles * a.nChunks;
     if (items > INT_MAX) return fail(PBA_ERR_UNSUPPORTED, "too many forward work items");
     a.items = (int)items;
-    // persistent: at most two CTAs per SM (their shared memory allows no more)
-    const long long grid = std::min<long long>(items, 2LL * num_sms());
+    // persistent: one CTA per SM (its shared memory and tensor memory allow no more)
+    const long long grid = std::min<long long>(items, num_sms());
     {
         ProfScope ps(K_FWD, stream);
-        pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);
+        pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_LAUNCH, stream>>>(tq, tk, tv, tb, a);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pba_fwd_kernel launch");
@@ -510,7 +505,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_zero_kernel launch");
             {
                 ProfScope ps(K_DBIAS, s);
-                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+                pba::pba_dbias_kernel<CP><<<(unsigned)g2, DT::THREADS, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
             // (the last CTA of every tile sums the split partials in split order)
@@ -1081,6 +1076,25 @@ pba_status pba_bwd_noalloc(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 
     if ((st = noalloc_scratch(&scratch)) != PBA_OK) return st;
     return pba_bwd(q, k, v, bias, key_mask, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
                    scratch, kNoAllocScratchBytes, d, stream);
+}
+
+pba_status pba_dbias_sum(const float *parts, int n_parts, int64_t n, float *out, void *stream) {
+    g_last_error.clear();
+    if (n_parts < 1 || n < 0) return fail(PBA_ERR_INVALID_ARG, "n_parts must be >= 1 and n >= 0");
+    if (n == 0) return PBA_OK;
+    if (!parts || !out) return fail(PBA_ERR_INVALID_ARG, "parts and out are required");
+    if (!aligned16(parts) || !aligned16(out)) return fail(PBA_ERR_INVALID_ARG, "parts and out must be 16-byte aligned");
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(parts), hi = lo + (uintptr_t)n_parts * (uintptr_t)n * 4;
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out), o1 = o0 + (uintptr_t)n * 4;
+    if (o0 < hi && lo < o1) return fail(PBA_ERR_INVALID_ARG, "out overlaps parts");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int vec = (n & 3) == 0;
+    {
+        ProfScope ps(K_DBIAS_SUM, s);
+        pba::pba_dbias_sum_kernel<<<grid_for(vec ? n / 4 : n, 256), 256, 0, s>>>(parts, n_parts, n, out, vec);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PBA_OK : cuda_fail(e, "pba_dbias_sum_kernel launch");
 }
 
 pba_status pba_device_status(void *stream) {

@@ -162,30 +162,35 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
     }
 }
 
-// P and dS of 64 keys (one half of a 128-key tile) for one query row, in KC-key chunks.
-//   tS, tdP: this lane's S and dP columns in TMEM; bias_row: the row's 64 bf16 bias values
-//   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
-//   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
+// P and dS of NK keys (NK = 64: one half of a 128-key tile; NK = 32: one quarter) for one
+// query row, in KC-key chunks.
+//   tS, tdP: this lane's S and dP columns of those keys in TMEM; bias_row: the row's 64-key
+//   half of the bias tile (bf16, a 128-byte swizzled shared-memory row) and c8_base the
+//   first of its 16-byte chunks that the keys start at (0, or 4 for the second quarter of
+//   a half); mw0, mw1: mask words of keys 0-31 and 32-63 of the NK (all ones when `full`);
+//   sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
 //   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
 // For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS.
-template <int KC, typename Use>
-__device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
-                                          bool has_bias, uint32_t mw0, uint32_t mw1, bool full,
-                                          float sl2e, float lse2, float D, Use &&use) {
-    // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers; the main kernel
-    // uses 16 to stay within the 128 registers a thread has at 512 threads per CTA
+// The masked and the unmasked loop are separate instantiations (MASKED), chosen per call by
+// `full`, so that tiles without masked keys carry no per-key select.
+template <int NK, int KC, bool MASKED, typename Use>
+__device__ __forceinline__ void p_ds_keys_impl(uint32_t tS, uint32_t tdP, uint32_t bias_row, int c8_base,
+                                               int row, bool has_bias, uint32_t mw0, uint32_t mw1,
+                                               float sl2e, float lse2, float D, Use &&use) {
+    // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers
     static_assert(KC == 16 || KC == 32, "chunk");
+    static_assert(NK == 32 || NK == 64, "keys");
     const float2 sl2 = make_float2(sl2e, sl2e), l2e2 = make_float2(kLog2eB, kLog2eB);
     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
 #pragma unroll
-    for (int q = 0; q < 64 / KC; ++q) {
+    for (int q = 0; q < NK / KC; ++q) {
         uint32_t r[2 * KC];   // S of keys KC q .. KC q + KC - 1 in r[0, KC), dP in r[KC, 2 KC)
         if constexpr (KC == 32) tmem_ld32x2(tS + q * KC, tdP + q * KC, r);
         else tmem_ld16x2(tS + q * KC, tdP + q * KC, r);
         const uint32_t mw = ((q * KC) < 32 ? mw0 : mw1) >> ((q * KC) & 31);
 #pragma unroll
         for (int c2 = 0; c2 < KC / 8; ++c2) {
-            const int c8 = q * (KC / 8) + c2;
+            const int c8 = c8_base + q * (KC / 8) + c2;
             uint4 bw = make_uint4(0, 0, 0, 0);
             if (has_bias) bw = lds128(bias_row + ((c8 ^ (row & 7)) << 4));
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
@@ -195,7 +200,7 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
                 float2 u = ffma2(make_float2(bf16lo(bb[e]), bf16hi(bb[e])), l2e2, nl2);
                 u = ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, u);
                 float2 p = make_float2(ex2(u.x), ex2(u.y));
-                if (!full) {
+                if constexpr (MASKED) {
                     p.x = ((mw >> k) & 1u) ? p.x : 0.f;
                     p.y = ((mw >> (k + 1)) & 1u) ? p.y : 0.f;
                 }
@@ -204,6 +209,16 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
             }
         }
     }
+}
+
+template <int NK, int KC, typename Use>
+__device__ __forceinline__ void p_ds_keys(uint32_t tS, uint32_t tdP, uint32_t bias_row, int c8_base,
+                                          int row, bool has_bias, uint32_t mw0, uint32_t mw1,
+                                          bool full, float sl2e, float lse2, float D, Use &&use) {
+    if (full)
+        p_ds_keys_impl<NK, KC, false>(tS, tdP, bias_row, c8_base, row, has_bias, mw0, mw1, sl2e, lse2, D, use);
+    else
+        p_ds_keys_impl<NK, KC, true>(tS, tdP, bias_row, c8_base, row, has_bias, mw0, mw1, sl2e, lse2, D, use);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -250,10 +265,13 @@ static_assert(BwdTraits<64>::SMEM_BYTES <= 232448 && BwdTraits<32>::SMEM_BYTES <
 
 // Warp roles (512 threads, four warpgroups): warps 0-7 element-wise (two warpgroups, one
 // 64-key half each), warp 8 TMA producer, warp 9 TMEM allocator and (lane 0) issuer of the
-// dV, dK, dQ products, warp 10 (lane 0) issuer of S = Q K^T and dP = dOa V^T, warp 11 idle,
-// warps 12-15 the dQ flushes and dK/dV epilogues (thread = TMEM lane).  A tcgen05.mma issue
-// holds its thread about as long as the MMA runs, so S/dP of the next step do not wait
-// behind this step's 24 products.  Every thread has 128 registers (512 threads on one SM).
+// dV products, warp 10 (lane 0) issuer of S = Q K^T and dP = dOa V^T of each step and then
+// of the previous step's dQ products, warp 11 (lane 0) issuer of the dK products, warps
+// 12-15 the dQ flushes and dK/dV epilogues (thread = TMEM lane).  One thread issues a
+// tcgen05.mma only every ~200 cycles whatever the shape (measured: M = 128, K = 16, N = 32
+// to 256), while several issuing threads proceed at that rate each; the 28 MMAs of a step
+// are therefore spread over three threads (12, 8 and 8).  Every thread has 128 registers
+// (512 threads on one SM).
 template <int CP>
 __global__ void __launch_bounds__(512, 1)
 pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -312,15 +330,15 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(b_sd_full, 1);
         mbar_init(b_sd_free, 256);
         mbar_init(b_ps_full, 256);
-        mbar_init(b_ps_free, 1);
-        mbar_init(b_drain, 2);   // one commit from each issuer
+        mbar_init(b_ps_free, 3);   // the dV, dK and dQ issuers' commits
+        mbar_init(b_drain, 3);     // one commit from each issuer
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_dq_full(x), 1);
             mbar_init(b_dq_free(x), 128);
         }
         for (int x = 0; x < QS; ++x) {
             mbar_init(b_q_full(x), 1);
-            mbar_init(b_q_empty(x), 1 + 256);
+            mbar_init(b_q_empty(x), 2 + 256);   // the dV and dK commits, the element-wise warps
         }
         for (int x = 0; x < BS; ++x) {
             mbar_init(b_bias_full(x), 1);
@@ -331,7 +349,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_init(b_kv_empty(x), 1);
         }
         for (int x = 0; x < DKB; ++x) {
-            mbar_init(b_dkv_full(x), 1);
+            mbar_init(b_dkv_full(x), 2);   // the dV and dK commits
             mbar_init(b_dkv_free(x), 128);
         }
         mbar_init(b_stg_full, 128);
@@ -412,54 +430,92 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
         }
     } else if (warp == 10) {
-        // ------------------------------------------------------------------ S/dP issuer
+        // ------------------------------------------------------------------ S/dP and dQ issuer
+        // S/dP of step t, then the dQ products of step t - 1, so that the next step's scores
+        // are never queued behind this step's products.  With one K/V stage the previous
+        // item's last dQ (which frees the stage) goes first at an item's first step.
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);   // S = Q K^T, dP = dOa V^T
+            constexpr uint32_t id_q = idesc_bf16(128, CP, false, true);     // dQ = dS K
+            const uint32_t sDS = sbase + T::OFF_DS;
             bool ok = true;
-            // step t: its item's K/V, its Q/dOa, and S/dP of step t - 1 read out
+            // S/dP of step t: its item's K/V, its Q/dOa, and S/dP of step t - 1 read out
+            auto issue_sdp = [&](int t, int m, int ii) -> bool {
+                const int st = t % QS, x = m % KVB;
+                bool okk = true;
+                if (ii == 0)
+                    okk = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
+                if (okk) okk = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
+                if (okk && t > 0) okk = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
+                if (!okk) return false;
+                tc_fence_after();
+                const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
+                const uint32_t sDO = sQ + T::TILE_BYTES;
+                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < CP / 16; ++kk) {
+                    umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
+                            sdesc(sK + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                    umma_ss(tbase + T::T_DP, sdesc(sDO + kk * 32, 16, SBO, T::SWZ),
+                            sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                }
+                umma_commit(b_sd_full);
+                return true;
+            };
+            // dQ of step t (item m, its step i of ni): P/dS written, the dQ buffer free
+            auto issue_dq = [&](int t, int m, int i, int ni) -> bool {
+                const int x = m % KVB;
+                bool okk = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
+                if (okk && t >= 2)
+                    okk = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
+                if (!okk) return false;
+                tc_fence_after();
+                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half
+                    const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
+                            sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
+                }
+                umma_commit(b_ps_free);
+                umma_commit(b_dq_full(t & 1));
+                if (i == ni - 1) umma_commit(b_kv_empty(x));   // the item's last reader of K/V
+                return true;
+            };
             int t = 0;
+            int pm = -1, pi = 0, pni = 0;   // the previous step: item, step within it, its steps
             for (int m = 0; m < M && ok; ++m) {
                 const int ni = item(m).ni;
                 for (int ii = 0; ii < ni && ok; ++ii, ++t) {
-                    const int st = t % QS, x = m % KVB;
-                    if (ii == 0)
-                        ok = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
-                    if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
-                    if (ok && t > 0) ok = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                    const uint32_t sDO = sQ + T::TILE_BYTES;
-                    const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
-                    const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < CP / 16; ++kk) {
-                        umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
-                                sdesc(sK + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
-                        umma_ss(tbase + T::T_DP, sdesc(sDO + kk * 32, 16, SBO, T::SWZ),
-                                sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
-                    }
-                    umma_commit(b_sd_full);
+                    const bool dq_first = KVB == 1 && ii == 0;
+                    if (dq_first && t > 0) ok = issue_dq(t - 1, pm, pi, pni);
+                    if (ok) ok = issue_sdp(t, m, ii);
+                    if (ok && !dq_first && t > 0) ok = issue_dq(t - 1, pm, pi, pni);
+                    pm = m; pi = ii; pni = ni;
                 }
             }
+            if (ok && t > 0) issue_dq(t - 1, pm, pi, pni);
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------------------ products issuer
+    } else if (warp == 9 || warp == 11) {
+        // ------------------------------------------------------------------ dV / dK issuers
+        // warp 9 issues dV += P^T dOa, warp 11 dK += dS^T Q: one issuing thread per product,
+        // so that each MMA stream goes at its own thread's issue rate
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
-            constexpr uint32_t id_kv = idesc_bf16(128, CP, true, true);     // dV = P^T dOa, dK = dS^T Q
-            constexpr uint32_t id_q = idesc_bf16(128, CP, false, true);     // dQ = dS K
-            const uint32_t sP = sbase + T::OFF_P, sDS = sbase + T::OFF_DS;
+            constexpr uint32_t id_kv = idesc_bf16(128, CP, true, true);
+            const bool is_dv = warp == 9;
+            const uint32_t sA = sbase + (is_dv ? T::OFF_P : T::OFF_DS);
             bool ok = true;
-            // step t: P/dS written (S/dP of the step were read out before that, so its
-            // S/dP MMAs are complete); this item's dK/dV buffer and the dQ buffer free
+            // step t: P/dS written (S/dP of the step were read out before that, so its S/dP
+            // MMAs are complete); this item's dK/dV buffer free
             int t = 0;
             for (int m = 0; m < M && ok; ++m) {
                 const int ni = item(m).ni;
                 for (int i = 0; i < ni && ok; ++i, ++t) {   // i: the item's step (query tile ilo + i)
-                    const int st = t % QS;
-                    const int x = m % KVB, d = m % DKB;
+                    const int st = t % QS, d = m % DKB;
                     ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
                     if (!ok) break;
                     if (i == 0 && m >= DKB) {
@@ -467,40 +523,21 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
                         if (!ok) break;
                     }
-                    if (t >= 2) {
-                        ok = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
-                        if (!ok) break;
-                    }
                     tc_fence_after();
                     const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                    const uint32_t sDO = sQ + T::TILE_BYTES;
-                    const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
-                    const uint32_t tDK = tbase + T::T_DK + d * 2 * CP, tDV = tDK + CP;
-                    // The three products interleaved, one K step of each in turn: consecutive
-                    // MMAs into one accumulator wait on each other, three accumulators in
-                    // rotation keep the tensor pipe fed.
+                    const uint32_t sB = is_dv ? sQ + T::TILE_BYTES : sQ;   // dOa or Q
+                    const uint32_t tD = tbase + T::T_DK + d * 2 * CP + (is_dv ? CP : 0);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        // dV, dK: K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance
-                        // 2 KB, B (dOa / Q, MN-major) rows advance 16 rows
-                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                        umma_ss(tDV, sdesc(sP + kk * 2048, 16384, 1024, kSw128),
-                                sdesc(sDO + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                        umma_ss(tDK, sdesc(sDS + kk * 2048, 16384, 1024, kSw128),
-                                sdesc(sQ + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv, acc);
-                        // dQ: K steps over 16 keys: A (dS, K-major) advances 32 B within a
-                        // 64-key half
-                        const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
-                        umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
-                                sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
+                        // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
+                        // B (dOa / Q, MN-major) rows advance 16 rows
+                        umma_ss(tD, sdesc(sA + kk * 2048, 16384, 1024, kSw128),
+                                sdesc(sB + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv,
+                                (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(b_ps_free);
                     umma_commit(b_q_empty(st));
-                    umma_commit(b_dq_full(t & 1));
-                    if (i == ni - 1) {
-                        umma_commit(b_dkv_full(d));
-                        umma_commit(b_kv_empty(x));
-                    }
+                    if (i == ni - 1) umma_commit(b_dkv_full(d));
                 }
             }
         }
@@ -538,8 +575,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
                 uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
                 const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
-                p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
-                          row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
+                p_ds_keys<64, 16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
+                          0, row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
                           [&](int c, float2 p, float2 ds) {
                               pp[c >> 1] = pack_bf16x2(p.x, p.y);
                               dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
@@ -707,7 +744,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int tt = max(0, bias_done - BS); tt < bias_done; ++tt)
                 mbar_wait_drain(b_bias_full(tt % BS), (tt / BS) & 1);
         }
-        if ((warp == 9 || warp == 10) && lane == 0) {
+        if ((warp == 9 || warp == 10 || warp == 11) && lane == 0) {
             umma_commit(b_drain);   // each issuer's own MMAs
             mbar_wait_drain(b_drain, 0);
         }
@@ -769,10 +806,15 @@ struct DbTraits {
     static constexpr int SMEM_BYTES = OFF_MASK + NS * 32 + 1024;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
     static constexpr uint32_t ROWB = CP * 2;
+    // warps 0-15: element-wise, four warpgroups of one 32-key quarter each (four warps per
+    // scheduler keep the exponential unit fed); warp 16 TMA producer; warp 17 TMEM and MMA
+    static constexpr int EW_THREADS = 512;
+    static constexpr int THREADS = EW_THREADS + 64;
+    static constexpr int W_PROD = 16, W_MMA = 17;
 };
 
 template <int CP>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DbTraits<CP>::THREADS)
 pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
@@ -811,16 +853,16 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(b_drain, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_sd_full(x), 1);
-            mbar_init(b_sd_free(x), 256);
+            mbar_init(b_sd_free(x), T::EW_THREADS);
         }
         for (int x = 0; x < NS; ++x) {
             mbar_init(b_full(x), 1);
-            mbar_init(b_empty(x), 1 + 256);
+            mbar_init(b_empty(x), 1 + T::EW_THREADS);
         }
         s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == T::W_MMA) {
         tmem_alloc(smem_u32(&s_tmem_base), 512);
         tmem_relinquish();
     }
@@ -831,7 +873,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     volatile int *abort_flag = &s_abort;
     int n_done = 0;   // rows b whose stage loads were issued: [0, n_done)
 
-    if (warp == 8) {
+    if (warp == T::W_PROD) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -872,7 +914,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             n_done = n + 1;
         }
-    } else if (warp == 9) {
+    } else if (warp == T::W_MMA) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
@@ -900,16 +942,17 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------------ elementwise
+        // warpgroup e owns keys [32 e, 32 e + 32) of the tile for all 128 query rows
         const int e = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const float sl2e = a.scale * kLog2eB;
-        float2 acc[32];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
+        float2 acc[16];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
 #pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
+        for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.f, 0.f);
         bool ok = mbar_wait(b_bias, 0, abort_flag, SITE_DB_EW);
         ok = __all_sync(0xffffffffu, ok);
-        const uint32_t bias_row = sbase + T::OFF_BIAS + e * 16384 + row * 128;
+        const uint32_t bias_row = sbase + T::OFF_BIAS + (e >> 1) * 16384 + row * 128;
         for (int n = 0; n < nb && ok; ++n) {
             const int st = n % NS, x = n & 1;
             ok = mbar_wait(b_sd_full(x), (n >> 1) & 1, abort_flag, SITE_DB_EW);
@@ -919,10 +962,11 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc_fence_after();
             const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
             const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
-            const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
-            p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
-                      bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
-                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
+            const uint32_t mwe = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK)[st * 8 + e];
+            p_ds_keys<32, 16>(tbase + x * 256 + e * 32 + lane_off, tbase + x * 256 + 128 + e * 32 + lane_off,
+                              bias_row, (e & 1) * 4, row, a.has_bias != 0, mwe, 0u, mwe == 0xffffffffu,
+                              sl2e, rs.x, rs.y,
+                              [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
             tc_fence_before();
             mbar_arrive(b_sd_free(x));
             mbar_arrive(b_empty(st));
@@ -930,9 +974,9 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (ok) {
             // this split's partial tile: [split][h][tile][128][128]
             float *dst = a.dbias_part +
-                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 64;
+                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 32;
 #pragma unroll
-            for (int c = 0; c < 32; c += 2)
+            for (int c = 0; c < 16; c += 2)
                 *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
             __threadfence();   // this thread's partial row, before the tile counter moves
         }
@@ -941,18 +985,18 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) {
-        if (warp == 8 && lane == 0) {
+        if (warp == T::W_PROD && lane == 0) {
             mbar_wait_drain(b_bias, 0);
             for (int nn = max(0, n_done - NS); nn < n_done; ++nn) mbar_wait_drain(b_full(nn % NS), (nn / NS) & 1);
         }
-        if (warp == 9 && lane == 0) {
+        if (warp == T::W_MMA && lane == 0) {
             umma_commit(b_drain);
             mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
         __syncthreads();
     }
-    if (warp == 9) {
+    if (warp == T::W_MMA) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tbase, 512);
@@ -970,35 +1014,36 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (!s_last) return;
     __threadfence();
     // Only the tile's valid part (rows i < Nq, four-key groups starting below Nk) is summed,
-    // four positions per thread at a time.  Every position adds its partials in split order,
-    // starting from zero; the loads of four splits of the four positions are all issued
-    // before their additions, so their latencies overlap.
+    // U positions of four keys per thread at a time.  Every position adds its partials in
+    // split order, starting from zero; the loads of four splits of the U positions are all
+    // issued before their additions, so their latencies overlap.
+    constexpr int U = 2;
     const long long plane = (long long)a.H * a.ntiles * 128 * 128;
     const float *part = a.dbias_part + ((long long)h * a.ntiles + bt) * 128 * 128;
     const int groups = (min(128, a.Nk - j0) + 3) >> 2;
     const int nv = min(128, a.Nq - i0) * groups;
-    for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * blockDim.x) {
-        int off[4];   // row * 128 + column within the tile, or -1
-        float4 sum[4];
+    for (int v0 = threadIdx.x; v0 < nv; v0 += U * blockDim.x) {
+        int off[U];   // row * 128 + column within the tile, or -1
+        float4 sum[U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int v = v0 + u * blockDim.x;
             off[u] = v < nv ? (v / groups) * 128 + (v % groups) * 4 : -1;
             sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int q = 0;
         for (; q + 4 <= a.splits; q += 4) {
-            float4 x[4][4];
+            float4 x[4][U];
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < U; ++u)
                     x[s][u] = off[u] >= 0 ? __ldcg(reinterpret_cast<const float4 *>(part + (q + s) * plane + off[u]))
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < U; ++u) {
                     sum[u].x += x[s][u].x;
                     sum[u].y += x[s][u].y;
                     sum[u].z += x[s][u].z;
@@ -1007,7 +1052,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         for (; q < a.splits; ++q) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < U; ++u) {
                 if (off[u] < 0) continue;
                 const float4 x = __ldcg(reinterpret_cast<const float4 *>(part + q * plane + off[u]));
                 sum[u].x += x.x;
@@ -1017,7 +1062,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < U; ++u) {
             if (off[u] < 0) continue;
             const int i = i0 + (off[u] >> 7), j = j0 + (off[u] & 127);
             float *dst = a.dbias + ((long long)h * a.Nq + i) * a.Nk + j;
@@ -1026,6 +1071,34 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (j + 2 < a.Nk) dst[2] = sum[u].z;
             if (j + 3 < a.Nk) dst[3] = sum[u].w;
         }
+    }
+}
+
+// out[i] = ordered sum over the parts of parts[p][i] (part 0 first).  With `vec` (n a
+// multiple of 4, so that every part starts 16-byte aligned) four elements per thread and
+// load, otherwise one.
+__global__ void __launch_bounds__(256) pba_dbias_sum_kernel(const float *parts, int n_parts, long long n,
+                                                            float *out, int vec) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    if (vec) {
+        const long long n4 = n >> 2;
+        for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n4; e += stride) {
+            float4 acc = __ldcs(reinterpret_cast<const float4 *>(parts) + e);
+            for (int p = 1; p < n_parts; ++p) {
+                const float4 x = __ldcs(reinterpret_cast<const float4 *>(parts + p * n) + e);
+                acc.x += x.x;
+                acc.y += x.y;
+                acc.z += x.z;
+                acc.w += x.w;
+            }
+            reinterpret_cast<float4 *>(out)[e] = acc;
+        }
+        return;
+    }
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
+        float acc = parts[i];
+        for (int p = 1; p < n_parts; ++p) acc += parts[p * n + i];
+        out[i] = acc;
     }
 }
 

@@ -43,103 +43,121 @@ class Bar:
 
 
 class FwdSim:
-    def __init__(self, nJ, nbs, KVS, BS, seed, row_mask=False, plant=None):
+    """The persistent forward kernel (pba_fwd.cuh): a producer (Q tile per slot, K and V rings,
+    bias tiles), a mask-fold warp, one MMA issuer per row group, and two row groups g
+    (the slots s with s & 1 == g), each of two key halves e that exchange the row maximum
+    at every step and the row sums at every item's end through a two-slot buffer guarded
+    by one barrier per slot (two arrivals).  Each softmax half is its own role here (the
+    four row quads of a half behave alike and share every barrier but their exchange
+    barriers, so one quad stands for all)."""
+
+    def __init__(self, nJ, nbs, KVS, BS, BC, seed, row_mask=False, plant=None):
+        # KVS: K and V stages of each row group's own rings
         self.rng = random.Random(seed)
         self.plant = plant
-        self.nJ, self.nbs, self.KVS, self.BS = nJ, nbs, KVS, BS
+        self.nJ, self.nbs, self.KVS, self.BS, self.BC = nJ, nbs, KVS, BS, BC
+        assert all(1 <= nb <= BC for nb in nbs)
         self.row_mask = row_mask
         self.items = len(nbs)
-        # global step list: (item, j, s)
-        self.steps = [(n, j, s) for n, nb in enumerate(nbs) for j in range(nJ) for s in range(nb)]
-        self.K = len(self.steps)
         self.tiles = [(n, j) for n in range(self.items) for j in range(nJ)]
         B = Bar
-        self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
-        self.k_full = [B("k_full%d" % i, 1) for i in range(KVS)]
-        self.k_empty = [B("k_empty%d" % i, 1) for i in range(KVS)]
-        self.v_full = [B("v_full%d" % i, 1) for i in range(KVS)]
-        self.v_empty = [B("v_empty%d" % i, 1) for i in range(KVS)]
+        self.q_full = [B("q_full%d" % i, 1) for i in range(BC)]
+        self.q_empty = [B("q_empty%d" % i, 1) for i in range(BC)]
+        self.k_full = [[B("k_full%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
+        self.k_empty = [[B("k_empty%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
+        self.v_full = [[B("v_full%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
+        self.v_empty = [[B("v_empty%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
         self.bias_full = [B("bias_full%d" % i, 1) for i in range(BS)]
         self.bias_ready = [B("bias_ready%d" % i, 1) for i in range(BS)]
-        self.bias_empty = [B("bias_empty%d" % i, 1) for i in range(BS)]
-        self.s_full, self.s_free = B("s_full", 1), B("s_free", 1)
-        self.p_full, self.p_free = B("p_full", 1), B("p_free", 1)
-        self.ofinal = B("ofinal", 1)
-        self.tma, self.mq_qk, self.mq_pv = [], [], []
-        self.q_item = None; self.q_readers = 0
-        self.k_stage = [None] * KVS; self.k_readers = [0] * KVS
-        self.v_stage = [None] * KVS; self.v_readers = [0] * KVS
-        self.words = [None] * KVS; self.words_readers = [0] * KVS
+        self.bias_empty = [B("bias_empty%d" % i, 4) for i in range(BS)]   # 2 groups x 2 halves
+        self.s_full = [B("s_full%d" % g, 1) for g in range(2)]
+        self.s_free = [B("s_free%d" % g, 2) for g in range(2)]
+        self.p_full = [B("p_full%d" % g, 2) for g in range(2)]
+        self.p_free = [B("p_free%d" % g, 1) for g in range(2)]
+        self.ofinal = [B("ofinal%d" % g, 1) for g in range(2)]
+        self.xbar = [[B("xbar%d%d" % (g, par), 2) for par in range(2)] for g in range(2)]
+        self.tma, self.mq_g = [], [[], []]
+        self.q_slot = [None] * BC; self.q_readers = [0] * BC
+        self.k_stage = [[None] * KVS for _ in range(2)]; self.k_readers = [[0] * KVS for _ in range(2)]
+        self.v_stage = [[None] * KVS for _ in range(2)]; self.v_readers = [[0] * KVS for _ in range(2)]
+        self.words = [[None] * KVS for _ in range(2)]; self.words_readers = [[0] * KVS for _ in range(2)]
         self.bias_tile = [None] * BS; self.bias_state = ["free"] * BS; self.bias_left = [0] * BS
-        self.S_step = None; self.S_reading = False; self.S_pend = 0
-        self.P_step = None; self.P_pend = 0
-        self.O_item = {}       # slot -> item whose products it holds
-        self.O_pend = {}       # slot -> PVs in flight
-        self.O_reading = set()
-        self.done_items = []
+        self.S_step = [None, None]; self.S_reading = [0, 0]; self.S_pend = [0, 0]
+        self.P_step = [{}, {}]; self.P_pend = [0, 0]
+        self.O_item = {}; self.O_pend = {}; self.O_reading = set()
+        self.xval = [[[None, None] for _ in range(2)] for _ in range(2)]   # [g][par][e] = exchange id
+        self.done = [[[], []], [[], []]]
 
     def step_async(self):
         ch = []
         if self.tma: ch.append("tma")
-        if self.mq_qk: ch.append("qk")
-        if self.mq_pv: ch.append("pv")
+        for g in range(2):
+            if self.mq_g[g]: ch.append(g)
         if not ch: return
         c = self.rng.choice(ch)
         if c == "tma":
             bar, n, fn = self.tma.pop(self.rng.randrange(len(self.tma)))
             fn(); bar.complete_tx(n)
         else:
-            q = self.mq_qk if c == "qk" else self.mq_pv
-            kind, x = q.pop(0)
+            kind, x = self.mq_g[c].pop(0)
             if kind == "mma": x()
             else: x.arrive()
 
     def producer(self):
         KVS, BS = self.KVS, self.BS
-        kg = 0; jg = 0
+        kg = 0; jg = 0; qloads = [0] * self.BC
         def load_bias(jg, tile):
             bs = jg % BS
             if jg >= BS:
                 while not self.bias_empty[bs].test(jg // BS - 1): yield
-            assert self.bias_state[bs] in ("free", "folded") and self.bias_left[bs] == 0
+            assert self.bias_state[bs] in ("free", "folded") and self.bias_left[bs] == 0, \
+                "bias buffer refilled while it is read"
             self.bias_state[bs] = "loading"; self.bias_tile[bs] = tile
             self.bias_full[bs].arrive_tx(1)
             self.tma.append((self.bias_full[bs], 1, lambda bs=bs: self.bias_state.__setitem__(bs, "landed")))
             yield
-        def load_k(k):
-            st, use = k % KVS, k // KVS
+        gsteps = [0, 0]
+        def load_k(k, g, gs):
+            st, use = gs % KVS, gs // KVS
             if use >= 1:
-                while not self.k_empty[st].test(use - 1): yield
-            assert self.k_readers[st] == 0
-            self.k_stage[st] = None
-            self.k_full[st].arrive_tx(1)
-            self.tma.append((self.k_full[st], 1, lambda st=st, k=k: self.k_stage.__setitem__(st, k)))
+                while not self.k_empty[g][st].test(use - 1): yield
+            assert self.k_readers[g][st] == 0
+            self.k_stage[g][st] = None
+            self.k_full[g][st].arrive_tx(1)
+            self.tma.append((self.k_full[g][st], 1, lambda st=st, k=k, g=g: self.k_stage[g].__setitem__(st, k)))
             yield
-        def load_v(k):
-            st, use = k % KVS, k // KVS
+        def load_v(k, g, gs):
+            st, use = gs % KVS, gs // KVS
             if use >= 1:
-                while not self.v_empty[st].test(use - 1): yield
-            assert self.v_readers[st] == 0 and self.words_readers[st] == 0
-            self.v_stage[st] = None; self.words[st] = k
-            self.v_full[st].arrive_tx(1)
-            self.tma.append((self.v_full[st], 1, lambda st=st, k=k: self.v_stage.__setitem__(st, k)))
+                while not self.v_empty[g][st].test(use - 1): yield
+            assert self.v_readers[g][st] == 0 and self.words_readers[g][st] == 0
+            self.v_stage[g][st] = None; self.words[g][st] = k
+            self.v_full[g][st].arrive_tx(1)
+            self.tma.append((self.v_full[g][st], 1, lambda st=st, k=k, g=g: self.v_stage[g].__setitem__(st, k)))
             yield
         for n, nb in enumerate(self.nbs):
             Kn = self.nJ * nb
             k0 = kg
-            yield from load_bias(jg, (n, 0))
-            yield from load_k(k0)
-            # the item's Q tiles: the previous item's Q K^T products must be done
-            if n >= 1 and self.plant != "no_q_empty_wait":
-                while not self.q_empty.test(n - 1): yield
-            assert self.q_readers == 0, "Q refilled while a Q K^T reads it"
-            self.q_item = None
-            self.q_full.arrive_tx(1)
-            self.tma.append((self.q_full, 1, lambda n=n: setattr(self, "q_item", n)))
-            yield
+            # each step's group and its step count within the group
+            grp = [(kl % nb) & 1 for kl in range(Kn)]
+            gsk = []
             for kl in range(Kn):
-                if kl + 1 < Kn: yield from load_k(k0 + kl + 1)
-                yield from load_v(k0 + kl)
+                gsk.append(gsteps[grp[kl]]); gsteps[grp[kl]] += 1
+            yield from load_bias(jg, (n, 0))
+            yield from load_k(k0, grp[0], gsk[0])
+            for s in range(nb):
+                # slot s's Q tile: the previous item's last Q K^T on the slot must be done
+                if qloads[s] >= 1 and self.plant != "no_q_empty_wait":
+                    while not self.q_empty[s].test(qloads[s] - 1): yield
+                assert self.q_readers[s] == 0, "Q refilled while a Q K^T reads it"
+                self.q_slot[s] = None
+                self.q_full[s].arrive_tx(1)
+                self.tma.append((self.q_full[s], 1, lambda s=s, n=n: self.q_slot.__setitem__(s, n)))
+                qloads[s] += 1
+                yield
+            for kl in range(Kn):
+                if kl + 1 < Kn: yield from load_k(k0 + kl + 1, grp[kl + 1], gsk[kl + 1])
+                yield from load_v(k0 + kl, grp[kl], gsk[kl])
                 if kl + 1 < Kn and (kl + 1) % nb == 0:
                     yield from load_bias(jg + (kl + 1) // nb, (n, (kl + 1) // nb))
             kg += Kn; jg += self.nJ
@@ -149,111 +167,158 @@ class FwdSim:
             bs = jg % self.BS
             while not self.bias_full[bs].test(jg // self.BS): yield
             assert self.bias_state[bs] == "landed" and self.bias_tile[bs] == tile
-            self.bias_state[bs] = "folded"; self.bias_left[bs] = self.nbs[tile[0]]
+            self.bias_state[bs] = "folded"; self.bias_left[bs] = 4
             yield
             self.bias_ready[bs].arrive()
 
-    def issuer_qk(self):
-        kg = 0
+    def issuer(self, g):
+        # row group g's issuer: Q K^T of each of the group's steps, then P V of the group's
+        # previous step (so a step's scores never wait behind the previous step's P V)
+        kg = 0; gk = 0; quse = [0] * self.BC
+        q = self.mq_g[g]
+        pend = None
+        def pv(pk, pj, ps, pst, pn, pnb, pgk):
+            while not self.p_full[g].test(pgk): yield
+            while not self.v_full[g][pst].test(pgk // self.KVS): yield
+            assert self.v_stage[g][pst] == pk
+            if pj == 0:   # first tile: the slot starts over
+                assert not any(x[0] == ps for x in self.O_reading), "O overwritten while the epilogue reads it"
+                self.O_item[ps] = pn
+            assert self.O_item[ps] == pn
+            self.v_readers[g][pst] += 1; self.P_pend[g] += 1; self.O_pend[ps] = self.O_pend.get(ps, 0) + 1
+            def ex(st=pst, k=pk, s=ps, n=pn):
+                assert self.P_step[g] == {0: k, 1: k}, "P V read a P that is not this step's"
+                assert self.v_stage[g][st] == k and self.O_item[s] == n
+                assert not any(x[0] == s for x in self.O_reading)
+                self.v_readers[g][st] -= 1; self.P_pend[g] -= 1; self.O_pend[s] -= 1
+            q.append(("mma", ex))
+            q.append(("commit", self.p_free[g]))
+            q.append(("commit", self.v_empty[g][pst]))
+            if pj == self.nJ - 1 and ps + 2 >= pnb and self.plant != "early_ofinal":
+                q.append(("commit", self.ofinal[g]))
+            if self.plant == "early_ofinal" and pj == 0 and ps == g:
+                q.append(("commit", self.ofinal[g]))
+            yield
         for n, nb in enumerate(self.nbs):
             Kn = self.nJ * nb
-            while not self.q_full.test(n): yield
-            for kl in range(Kn):
-                k = kg + kl; st = k % self.KVS
-                if k > 0:
-                    while not self.s_free.test(k - 1): yield
-                while not self.k_full[st].test(k // self.KVS): yield
-                assert self.k_stage[st] == k and self.q_item == n
-                self.q_readers += 1; self.k_readers[st] += 1; self.S_pend += 1
-                def ex(st=st, k=k, n=n):
-                    assert not self.S_reading
-                    assert self.k_stage[st] == k and self.q_item == n
-                    self.q_readers -= 1; self.k_readers[st] -= 1; self.S_pend -= 1
-                    self.S_step = k
-                self.mq_qk.append(("mma", ex))
-                self.mq_qk.append(("commit", self.s_full))
-                self.mq_qk.append(("commit", self.k_empty[st]))
-                if kl == Kn - 1:
-                    self.mq_qk.append(("commit", self.q_empty))
+            if nb <= g:
+                # no row of this group in the item: its last P V goes out now (the group's
+                # epilogue waits for it, and the item's loads wait for that epilogue's group
+                # to hand back the item's bias tiles)
+                if pend is not None and self.plant != "keep_pending":
+                    yield from pv(*pend); pend = None
+                if self.plant == "idle_ofinal":
+                    # (a planted mistake: completing the barrier for an item without rows of
+                    # the group lets it run two phases ahead of the group's epilogue)
+                    q.append(("commit", self.ofinal[g]))
                 yield
-            kg += Kn
-
-    def issuer_pv(self):
-        kg = 0
-        for n, nb in enumerate(self.nbs):
-            Kn = self.nJ * nb
             for kl in range(Kn):
-                k = kg + kl; st = k % self.KVS; s = kl % nb
-                while not self.p_full.test(k): yield
-                while not self.v_full[st].test(k // self.KVS): yield
-                assert self.v_stage[st] == k
-                if kl < nb:   # first tile: the slot starts over
-                    assert s not in self.O_reading, "O overwritten while the epilogue reads it"
-                    self.O_item[s] = n
-                assert self.O_item[s] == n
-                self.v_readers[st] += 1; self.P_pend += 1; self.O_pend[s] = self.O_pend.get(s, 0) + 1
-                def ex(st=st, k=k, s=s, n=n):
-                    assert self.P_step == k and self.v_stage[st] == k and self.O_item[s] == n
-                    assert s not in self.O_reading
-                    self.v_readers[st] -= 1; self.P_pend -= 1; self.O_pend[s] -= 1
-                self.mq_pv.append(("mma", ex))
-                self.mq_pv.append(("commit", self.p_free))
-                self.mq_pv.append(("commit", self.v_empty[st]))
+                k = kg + kl; j, s = divmod(kl, nb)
+                if s & 1 != g: continue
+                st = gk % self.KVS
+                if gk > 0 and self.plant != "no_s_free_wait":
+                    while not self.s_free[g].test(gk - 1): yield
+                while not self.k_full[g][st].test(gk // self.KVS): yield
+                if j == 0:
+                    while not self.q_full[s].test(quse[s]): yield
+                assert self.k_stage[g][st] == k and self.q_slot[s] == n
+                self.q_readers[s] += 1; self.k_readers[g][st] += 1; self.S_pend[g] += 1
+                def ex(st=st, k=k, n=n, s=s):
+                    assert self.S_reading[g] == 0, "S overwritten while the softmax reads it"
+                    assert self.k_stage[g][st] == k and self.q_slot[s] == n
+                    self.q_readers[s] -= 1; self.k_readers[g][st] -= 1; self.S_pend[g] -= 1
+                    self.S_step[g] = k
+                q.append(("mma", ex))
+                q.append(("commit", self.s_full[g]))
+                q.append(("commit", self.k_empty[g][st]))
+                if j == self.nJ - 1:
+                    q.append(("commit", self.q_empty[s]))
                 yield
-            self.mq_pv.append(("commit", self.ofinal))
+                if pend is not None:
+                    yield from pv(*pend)
+                pend = (k, j, s, st, n, nb, gk)
+                gk += 1
+            for s in range(nb): quse[s] += 1
             kg += Kn
+        if pend is not None:
+            yield from pv(*pend)
 
-    def softmax(self):
-        kg = 0; jg = 0
+    def softmax(self, g, e):
+        kg = 0; jg = 0; gk = 0; xc = 0
+        gitems = 0   # items with a row of this group: the phases of its ofinal barrier
+        def exchange(tag):
+            nonlocal xc
+            par = xc & 1
+            self.xval[g][par][e] = (xc, tag)
+            self.xbar[g][par].arrive()
+            while not self.xbar[g][par].test(xc >> 1): yield
+            yield
+            assert self.xval[g][par][1 - e] == (xc, tag), "exchange slot rewritten before it was read"
+            xc += 1
         for n, nb in enumerate(self.nbs):
+            mine = [s for s in range(nb) if s % 2 == g]
             for j in range(self.nJ):
                 bs = (jg + j) % self.BS
-                for s in range(nb):
-                    k = kg + j * nb + s; st = k % self.KVS
-                    while not self.s_full.test(k): yield
-                    if s == 0:
+                if not mine:
+                    while not self.bias_ready[bs].test((jg + j) // self.BS): yield
+                    self.bias_left[bs] -= 1
+                    self.bias_empty[bs].arrive()
+                    yield
+                    continue
+                for t, s in enumerate(mine):
+                    k = kg + j * nb + s; st = gk % self.KVS
+                    while not self.s_full[g].test(gk): yield
+                    if t == 0:
                         while not self.bias_ready[bs].test((jg + j) // self.BS): yield
                     if self.row_mask:
-                        while not self.v_full[st].test(k // self.KVS): yield
-                        assert self.words[st] == k
-                        self.words_readers[st] += 1
-                    assert self.S_step == k and self.S_pend == 0
-                    self.S_reading = True
+                        while not self.v_full[g][st].test(gk // self.KVS): yield
+                        assert self.words[g][st] == k
+                        self.words_readers[g][st] += 1
+                    assert self.S_step[g] == k and self.S_pend[g] == 0
+                    self.S_reading[g] += 1
                     yield
-                    self.S_reading = False
-                    self.s_free.arrive()
+                    self.S_reading[g] -= 1
+                    self.s_free[g].arrive()
                     assert self.bias_tile[bs] == (n, j) and self.bias_state[bs] == "folded"
                     yield
-                    self.bias_left[bs] -= 1
-                    if s == nb - 1:
-                        assert self.bias_left[bs] == 0
+                    if t == len(mine) - 1:
+                        self.bias_left[bs] -= 1
                         self.bias_empty[bs].arrive()
-                    if k > 0:
-                        while not self.p_free.test(k - 1): yield
-                    assert self.P_pend == 0
+                    yield from exchange(("max", k))
+                    if gk > 0:
+                        while not self.p_free[g].test(gk - 1): yield
+                    assert self.P_pend[g] == 0, "P rewritten while a P V reads it"
                     assert self.O_pend.get(s, 0) == 0
-                    self.P_step = k
+                    self.P_step[g][e] = k
                     yield
                     if self.row_mask:
-                        assert self.words[st] == k
-                        self.words_readers[st] -= 1
-                    self.p_full.arrive()
-            # epilogue of item n
-            while not self.ofinal.test(n): yield
-            assert all(self.O_pend.get(s, 0) == 0 for s in range(nb))
-            assert all(self.O_item.get(s) == n for s in range(nb))
-            self.O_reading = set(range(nb))
+                        assert self.words[g][st] == k
+                        self.words_readers[g][st] -= 1
+                    self.p_full[g].arrive()
+                    gk += 1
+            # epilogue of item n: the group's slots (no wait when it had none)
+            if mine:
+                while not self.ofinal[g].test(gitems): yield
+                gitems += 1
+            assert all(self.O_pend.get(s, 0) == 0 and self.O_item.get(s) == n for s in mine), \
+                "O read before its products are done"
+            yield from exchange(("sum", n))
+            for s in mine: self.O_reading.add((s, e))
             yield
-            self.O_reading = set()
-            self.done_items.append(n)
+            for s in mine: self.O_reading.discard((s, e))
+            self.done[g][e].append(n)
             kg += self.nJ * nb; jg += self.nJ
 
     def run(self):
-        live = {"prod": self.producer(), "fold": self.fold(), "qk": self.issuer_qk(),
-                "pv": self.issuer_pv(), "smx": self.softmax()}
+        live = {"prod": self.producer(), "fold": self.fold(), "iss0": self.issuer(0),
+                "iss1": self.issuer(1)}
+        for g in range(2):
+            for e in range(2):
+                live["smx%d%d" % (g, e)] = self.softmax(g, e)
         idle = 0
-        while live or self.tma or self.mq_qk or self.mq_pv:
-            opts = list(live) + (["async"] * 2 if (self.tma or self.mq_qk or self.mq_pv) else [])
+        while live or self.tma or self.mq_g[0] or self.mq_g[1]:
+            busy = self.tma or self.mq_g[0] or self.mq_g[1]
+            opts = list(live) + (["async"] * 2 if busy else [])
             c = self.rng.choice(opts)
             if c == "async":
                 self.step_async(); idle = 0; continue
@@ -261,10 +326,16 @@ class FwdSim:
             except StopIteration: del live[c]
             idle += 1
             if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
-        assert self.done_items == list(range(self.items))
+        assert self.done == [[list(range(self.items))] * 2] * 2
 
 
 class BwdSim:
+    """The persistent dq/dk/dv kernel (pba_bwd.cuh): a producer (K/V per item; Q, dOa and row
+    statistics per step; a bias tile per step), one element-wise role (S/dP -> P/dS), the
+    dQ / dK-dV epilogue warpgroup, and three MMA issuers, each in issue order: one for the
+    dV products, one for the dK products, and one that issues S/dP of step t and then the
+    dQ products of step t - 1."""
+
     def __init__(self, M, nI, QS, BS, KVB, DKB, seed, plant=None):
         self.rng = random.Random(seed)
         self.plant = plant
@@ -274,20 +345,19 @@ class BwdSim:
         self.T = len(self.steps)
         B = Bar
         self.kv_full = [B("kv_full%d" % x, 1) for x in range(KVB)]
-        self.kv_empty = [B("kv_empty%d" % x, 1) for x in range(KVB)]
+        self.kv_empty = [B("kv_empty%d" % x, 1) for x in range(KVB)]          # dQ issuer
         self.q_full = [B("q_full%d" % x, 1) for x in range(QS)]
-        self.q_empty = [B("q_empty%d" % x, 2) for x in range(QS)]   # MMA commit + EW
+        self.q_empty = [B("q_empty%d" % x, 3) for x in range(QS)]             # dV, dK commits + EW
         self.bias_full = [B("bias_full%d" % x, 1) for x in range(BS)]
         self.bias_empty = [B("bias_empty%d" % x, 1) for x in range(BS)]
         self.sd_full, self.sd_free = B("sd_full", 1), B("sd_free", 1)
-        self.ps_full, self.ps_free = B("ps_full", 1), B("ps_free", 1)
+        self.ps_full, self.ps_free = B("ps_full", 1), B("ps_free", 3)        # dV, dK, dQ commits
         self.dq_full = [B("dq_full%d" % x, 1) for x in range(2)]
         self.dq_free = [B("dq_free%d" % x, 1) for x in range(2)]
-        self.dkv_full = [B("dkv_full%d" % x, 1) for x in range(DKB)]
+        self.dkv_full = [B("dkv_full%d" % x, 2) for x in range(DKB)]          # dV, dK commits
         self.dkv_free = [B("dkv_free%d" % x, 1) for x in range(DKB)]
         self.tma = []
-        self.mq = []      # products issuer (in order)
-        self.mq_s = []    # S/dP issuer (in order); the two interleave arbitrarily
+        self.mq = {"dv": [], "dk": [], "sdq": []}   # one in-order queue per issuer
         # resource state
         self.kv_item = [None] * KVB; self.kv_readers = [0] * KVB; self.words_item = [None] * KVB
         self.q_step = [None] * QS; self.q_readers = [0] * QS
@@ -295,23 +365,23 @@ class BwdSim:
         self.sd_step = None; self.sd_reading = False; self.sd_pending = 0
         self.ps_step = None; self.ps_pending = 0
         self.dq_step = [None, None]; self.dq_pending = [0, 0]
-        self.dkv_item = [None] * DKB; self.dkv_pending = [0] * DKB; self.dkv_steps = [0] * DKB
+        self.acc_item = {"dv": [None] * DKB, "dk": [None] * DKB}
+        self.acc_steps = {"dv": [0] * DKB, "dk": [0] * DKB}
+        self.dkv_pending = [0] * DKB
         self.dkv_reading = [False] * DKB
         self.epi_done = []
         self.dq_flushed = []
 
     def step_async(self):
-        opts = []
-        if self.tma: opts.append("tma")
-        if self.mq: opts.append("mma")
-        if self.mq_s: opts.append("mma_s")
+        opts = ["tma"] if self.tma else []
+        opts += [k for k, q in self.mq.items() if q]
         if not opts: return
         c = self.rng.choice(opts)
         if c == "tma":
             bar, n, fn = self.tma.pop(self.rng.randrange(len(self.tma)))
             fn(); bar.complete_tx(n)
         else:
-            kind, x = (self.mq if c == "mma" else self.mq_s).pop(0)
+            kind, x = self.mq[c].pop(0)
             if kind == "mma": x()
             else: x.arrive()
 
@@ -331,7 +401,7 @@ class BwdSim:
                 st, bs = t % self.QS, t % self.BS
                 if t >= self.QS:
                     while not self.q_empty[st].test(t // self.QS - 1): yield
-                assert self.q_readers[st] == 0
+                assert self.q_readers[st] == 0, "Q/dOa stage refilled while it is read"
                 self.q_step[st] = None
                 self.q_full[st].arrive_tx(1)
                 self.tma.append((self.q_full[st], 1, lambda st=st, t=t: self.q_step.__setitem__(st, t)))
@@ -343,63 +413,89 @@ class BwdSim:
                 self.tma.append((self.bias_full[bs], 1, lambda bs=bs, t=t: self.bias_step.__setitem__(bs, t)))
                 yield
 
-    def issue_sdp(self, t, q):
-        st, x = t % self.QS, self.steps[t][0] % self.KVB
-        assert self.q_step[st] == t and self.kv_item[x] == self.steps[t][0]
-        self.q_readers[st] += 1; self.kv_readers[x] += 1; self.sd_pending += 1
-        def ex():
-            assert not self.sd_reading, "S/dP overwritten while the EW reads them"
-            assert self.q_step[st] == t and self.kv_item[x] == self.steps[t][0]
-            self.q_readers[st] -= 1; self.kv_readers[x] -= 1; self.sd_pending -= 1
-            self.sd_step = t
-        q.append(("mma", ex))
-        q.append(("commit", self.sd_full))
-
-    def issuer_sdp(self):
+    def issuer_sdq(self):
+        # S/dP of step t, then the dQ products of step t - 1; with one K/V stage, a step that
+        # starts an item issues the previous item's last dQ first (that dQ frees the stage)
         T = self.T
-        for t in range(T):
-            m = self.steps[t][0]
-            if self.steps[t][1] == 0:
-                while not self.kv_full[m % self.KVB].test(m // self.KVB): yield
-            while not self.q_full[t % self.QS].test(t // self.QS): yield
-            if t > 0:
-                while not self.sd_free.test(t - 1): yield
-            self.issue_sdp(t, self.mq_s)
-            yield
+        for t in range(T + 1):
+            dq_first = self.KVB == 1 and t < T and self.steps[t][1] == 0 and self.plant != "sdp_before_dq"
+            for part in (("dq", "sdp") if dq_first else ("sdp", "dq")):
+                if part == "sdp":
+                    yield from self._sdp(t)
+                else:
+                    yield from self._dq(t)
 
-    def issuer(self):
+    def _sdp(self, t):
+        T = self.T
+        if True:
+            if t < T:
+                m = self.steps[t][0]
+                st, x = t % self.QS, m % self.KVB
+                if self.steps[t][1] == 0:
+                    while not self.kv_full[x].test(m // self.KVB): yield
+                while not self.q_full[st].test(t // self.QS): yield
+                if t > 0:
+                    while not self.sd_free.test(t - 1): yield
+                assert self.q_step[st] == t and self.kv_item[x] == m
+                self.q_readers[st] += 1; self.kv_readers[x] += 1; self.sd_pending += 1
+                def ex_s(t=t, st=st, x=x, m=m):
+                    assert not self.sd_reading, "S/dP overwritten while the EW reads them"
+                    assert self.q_step[st] == t and self.kv_item[x] == m
+                    self.q_readers[st] -= 1; self.kv_readers[x] -= 1; self.sd_pending -= 1
+                    self.sd_step = t
+                self.mq["sdq"].append(("mma", ex_s))
+                self.mq["sdq"].append(("commit", self.sd_full))
+                yield
+
+    def _dq(self, t):
+        if True:
+            if t >= 1:
+                tq = t - 1
+                m, i = self.steps[tq]
+                x = m % self.KVB
+                while not self.ps_full.test(tq): yield
+                if tq >= 2:
+                    while not self.dq_free[tq & 1].test((tq >> 1) - 1): yield
+                assert self.ps_step == tq and self.kv_item[x] == m
+                self.ps_pending += 1; self.kv_readers[x] += 1; self.dq_pending[tq & 1] += 1
+                def ex_q(tq=tq, x=x, m=m):
+                    assert self.ps_step == tq and self.kv_item[x] == m
+                    self.ps_pending -= 1; self.kv_readers[x] -= 1; self.dq_pending[tq & 1] -= 1
+                    self.dq_step[tq & 1] = tq
+                q = self.mq["sdq"]
+                q.append(("mma", ex_q))
+                q.append(("commit", self.ps_free))
+                q.append(("commit", self.dq_full[tq & 1]))
+                if i == self.nis[m] - 1 and self.plant != "no_kv_empty_commit":
+                    q.append(("commit", self.kv_empty[x]))
+                yield
+
+    def issuer_dkv(self, kind):
         T = self.T
         for t in range(T):
             (m, i), st = self.steps[t], t % self.QS
-            x, d = m % self.KVB, m % self.DKB
+            d = m % self.DKB
             while not self.ps_full.test(t): yield
             if i == 0 and m >= self.DKB and self.plant != "no_dkv_free_wait":
                 while not self.dkv_free[d].test(m // self.DKB - 1): yield
-            if t >= 2:
-                while not self.dq_free[t & 1].test((t >> 1) - 1): yield
-            assert self.ps_step == t and self.q_step[st] == t and self.kv_item[x] == m
+            assert self.ps_step == t and self.q_step[st] == t
             assert self.sd_step is not None and self.sd_step >= t, "products before S/dP of the step"
             if i == 0:
-                assert self.dkv_pending[d] == 0
                 assert not self.dkv_reading[d], "dK/dV accumulator reset while the epilogue reads it"
-                self.dkv_item[d] = m; self.dkv_steps[d] = 0
-            assert self.dkv_item[d] == m, "dK/dV buffer reused before its epilogue"
-            self.ps_pending += 1; self.q_readers[st] += 1; self.kv_readers[x] += 1
-            self.dq_pending[t & 1] += 1; self.dkv_pending[d] += 1
-            def ex(t=t, st=st, x=x, d=d, m=m):
-                assert self.ps_step == t and self.q_step[st] == t and self.kv_item[x] == m
-                assert self.dkv_item[d] == m
-                self.ps_pending -= 1; self.q_readers[st] -= 1; self.kv_readers[x] -= 1
-                self.dq_pending[t & 1] -= 1; self.dkv_pending[d] -= 1; self.dkv_steps[d] += 1
-                self.dq_step[t & 1] = t
-            q = self.mq
+                self.acc_item[kind][d] = m; self.acc_steps[kind][d] = 0
+            assert self.acc_item[kind][d] == m, "dK/dV buffer reused before its epilogue"
+            self.ps_pending += 1; self.q_readers[st] += 1; self.dkv_pending[d] += 1
+            def ex(t=t, st=st, d=d, m=m):
+                assert self.ps_step == t and self.q_step[st] == t
+                assert self.acc_item[kind][d] == m and not self.dkv_reading[d]
+                self.ps_pending -= 1; self.q_readers[st] -= 1; self.dkv_pending[d] -= 1
+                self.acc_steps[kind][d] += 1
+            q = self.mq[kind]
             q.append(("mma", ex))
             q.append(("commit", self.ps_free))
             q.append(("commit", self.q_empty[st]))
-            q.append(("commit", self.dq_full[t & 1]))
             if i == self.nis[m] - 1:
                 q.append(("commit", self.dkv_full[d]))
-                q.append(("commit", self.kv_empty[x]))
             yield
 
     def ew(self):
@@ -437,19 +533,23 @@ class BwdSim:
             if i == self.nis[m] - 1:
                 d = m % self.DKB
                 while not self.dkv_full[d].test(m // self.DKB): yield
-                assert self.dkv_item[d] == m and self.dkv_pending[d] == 0 and self.dkv_steps[d] == self.nis[m]
+                assert self.dkv_pending[d] == 0
+                for kind in ("dv", "dk"):
+                    assert self.acc_item[kind][d] == m and self.acc_steps[kind][d] == self.nis[m]
                 self.epi_done.append(m)
                 self.dkv_reading[d] = True
                 yield
-                assert self.dkv_item[d] == m, "dK/dV changed under the epilogue"
+                assert all(self.acc_item[kind][d] == m for kind in ("dv", "dk")), "dK/dV changed under the epilogue"
                 self.dkv_reading[d] = False
                 self.dkv_free[d].arrive()
 
     def run(self):
-        live = {"prod": self.producer(), "sdp": self.issuer_sdp(), "mma": self.issuer(), "ew": self.ew(), "epi": self.epi()}
+        live = {"prod": self.producer(), "sdq": self.issuer_sdq(), "dv": self.issuer_dkv("dv"),
+                "dk": self.issuer_dkv("dk"), "ew": self.ew(), "epi": self.epi()}
         idle = 0
-        while live or self.tma or self.mq or self.mq_s:
-            opts = list(live) + (["async"] * 2 if (self.tma or self.mq or self.mq_s) else [])
+        while live or self.tma or any(self.mq.values()):
+            busy = self.tma or any(self.mq.values())
+            opts = list(live) + (["async"] * 2 if busy else [])
             c = self.rng.choice(opts)
             if c == "async":
                 self.step_async(); idle = 0; continue
@@ -463,24 +563,25 @@ class BwdSim:
 class DbiasSim:
     """The dbias kernel (pba_bwd.cuh): one producer fills NS stages (Q, dOa, K and V tiles, row
     statistics and mask words of one broadcast row each) after the bias tile; one MMA issuer
-    computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; two
-    element-wise warpgroups (128 arrivals each) read the TMEM buffer, the stage's row
-    statistics and mask words, and release both."""
+    computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; four
+    element-wise warpgroups (one 32-key quarter each, 128 arrivals each) read the TMEM buffer,
+    the stage's row statistics and mask words, and release both."""
 
-    def __init__(self, nb, NS, seed, plant=None):
+    def __init__(self, nb, NS, seed, plant=None, nwg=4):
         self.rng = random.Random(seed)
         self.plant = plant
-        self.nb, self.NS = nb, NS
+        self.nb, self.NS, self.nwg = nb, NS, nwg
         B = Bar
         self.bias = B("bias", 1)
         self.full = [B("full%d" % x, 1) for x in range(NS)]
-        self.empty = [B("empty%d" % x, 1 + 256) for x in range(NS)]   # MMA commit + 256 threads
+        # MMA commit + every element-wise thread
+        self.empty = [B("empty%d" % x, 1 + 128 * nwg) for x in range(NS)]
         self.sd_full = [B("sd_full%d" % x, 1) for x in range(2)]
-        self.sd_free = [B("sd_free%d" % x, 256) for x in range(2)]
+        self.sd_free = [B("sd_free%d" % x, 128 * nwg) for x in range(2)]
         self.tma, self.mq = [], []
         self.stage_row = [None] * NS; self.stage_readers = [0] * NS; self.mask_row = [None] * NS
         self.tm_row = [None, None]; self.tm_readers = [0, 0]; self.tm_pending = [0, 0]
-        self.summed = [[], []]
+        self.summed = [[] for _ in range(nwg)]
 
     def step_async(self):
         opts = (["tma"] if self.tma else []) + (["mma"] if self.mq else [])
@@ -543,7 +644,9 @@ class DbiasSim:
             self.sd_free[x].arrive(128); self.empty[st].arrive(128)
 
     def run(self):
-        live = {"prod": self.producer(), "mma": self.issuer(), "ew0": self.ew(0), "ew1": self.ew(1)}
+        live = {"prod": self.producer(), "mma": self.issuer()}
+        for e in range(self.nwg):
+            live["ew%d" % e] = self.ew(e)
         idle = 0
         while live or self.tma or self.mq:
             opts = list(live) + (["async"] * 2 if (self.tma or self.mq) else [])
@@ -554,7 +657,7 @@ class DbiasSim:
             except StopIteration: del live[c]
             idle += 1
             if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
-        assert self.summed == [list(range(self.nb))] * 2
+        assert self.summed == [list(range(self.nb))] * self.nwg
 
 
 class PwaGemmSim:

@@ -6,15 +6,18 @@ import pytest
 from pba_protocol_models import BwdSim, DbiasSim, FwdSim, PwaGemmSim
 
 
-# ring depths as the forward instantiates them: c=16 -> (3, 2), c=32 -> (2, 2), c=64 -> (2, 1)
-@pytest.mark.parametrize("KVS,BS", [(2, 2), (3, 2), (2, 1)])
-def test_forward_protocol(KVS, BS):
+# rings as the forward instantiates them (K/V stages per row group, bias buffers, slots):
+# c=16 -> (2, 2, 8), c=32 -> (2, 2, 4), c=64 -> (1, 2, 2); a deeper ring too
+@pytest.mark.parametrize("KVS,BS,BC", [(2, 2, 8), (2, 2, 4), (1, 2, 2), (3, 2, 4)])
+def test_forward_protocol(KVS, BS, BC):
     # items of nb rows over nJ key tiles (the last chunk of rows can be shorter)
-    for nJ in (1, 2, 3):
-        for nbs in ([1], [2, 2], [2, 1], [4, 4, 3], [1, 1, 1, 1]):
+    chunks = [[BC], [BC, BC], [BC, 1], [1], [2, 1, BC], [BC, BC - 1, 1], [BC, 1, 1, 2, 1]]
+    for nJ in (1, 2, 3, 5):
+        for nbs in chunks:
+            nbs = [min(nb, BC) for nb in nbs]
             for row_mask in (False, True):
-                for seed in range(12):
-                    FwdSim(nJ, nbs, KVS, BS, seed, row_mask).run()
+                for seed in range(8):
+                    FwdSim(nJ, nbs, KVS, BS, BC, seed, row_mask).run()
 
 
 # c=32 -> (2, 2, 2, 2), c=16 -> (3, 2, 2, 2), c=64 -> (2, 1, 1, 1); the last mixes depths
@@ -36,9 +39,17 @@ def _caught(make, seeds=40):
     return False
 
 
-def test_planted_forward_mistake_is_caught():
-    # Q of the next item loaded before the previous item's last Q K^T is done
-    assert _caught(lambda seed: FwdSim(2, [2, 2, 2], 2, 2, seed, plant="no_q_empty_wait"))
+def test_planted_forward_mistakes_are_caught():
+    # a slot's Q of the next item loaded before the previous item's last Q K^T on it is done
+    assert _caught(lambda seed: FwdSim(2, [4, 4, 4], 4, 2, 4, seed, plant="no_q_empty_wait"))
+    # a group's next Q K^T issued before its softmax has read the previous S
+    assert _caught(lambda seed: FwdSim(2, [4, 4], 4, 2, 4, seed, plant="no_s_free_wait"))
+    # the epilogue released before the group's last P V
+    assert _caught(lambda seed: FwdSim(2, [4, 4], 4, 2, 4, seed, plant="early_ofinal"))
+    # a group's completion barrier also completed for items without rows of the group
+    assert _caught(lambda seed: FwdSim(1, [4, 1, 1, 4], 4, 2, 4, seed, plant="idle_ofinal"))
+    # a group's last P V held back across an item without rows of the group: deadlock
+    assert _caught(lambda seed: FwdSim(2, [2, 1, 4], 4, 2, 4, seed, plant="keep_pending"))
 
 
 def test_planted_backward_mistakes_are_caught():
@@ -46,6 +57,9 @@ def test_planted_backward_mistakes_are_caught():
     assert _caught(lambda seed: BwdSim(4, 2, 2, 2, 2, 2, seed, plant="no_ps_free_wait"))
     # a dK/dV accumulator reused before its epilogue has read it (one buffer, one step per item)
     assert _caught(lambda seed: BwdSim(4, 1, 2, 2, 2, 1, seed, plant="no_dkv_free_wait"))
+    # with one K/V stage, S/dP of an item's first step issued before the previous item's last
+    # dQ, which is what frees the stage: deadlock
+    assert _caught(lambda seed: BwdSim(3, 2, 2, 1, 1, 1, seed, plant="sdp_before_dq"))
 
 
 # dbias kernel stages: c=64 -> 2, otherwise 3
