@@ -275,15 +275,20 @@ pba_status launch_fwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
     a.lse = lse;
     a.skip_step = g_debug_skip_step;
     a.win = win;
-    if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_LAUNCH)) != PBA_OK) return st;
+    if ((st = set_smem(pba::pba_fwd_kernel<CP>, T::SMEM_BYTES)) != PBA_OK) return st;
+    // two CTAs per SM need (almost) all of the unified L1 / shared memory as shared memory
+    cudaError_t ce = cudaFuncSetAttribute(pba::pba_fwd_kernel<CP>,
+                                          cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          cudaSharedmemCarveoutMaxShared);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute (carveout)");
     const long long items = tiles * a.nChunks;
     if (items > INT_MAX) return fail(PBA_ERR_UNSUPPORTED, "too many forward work items");
     a.items = (int)items;
-    // persistent: one CTA per SM (its shared memory and tensor memory allow no more)
-    const long long grid = std::min<long long>(items, num_sms());
+    // persistent: at most two CTAs per SM (their shared memory allows no more)
+    const long long grid = std::min<long long>(items, 2LL * num_sms());
     {
         ProfScope ps(K_FWD, stream);
-        pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_LAUNCH, stream>>>(tq, tk, tv, tb, a);
+        pba::pba_fwd_kernel<CP><<<(unsigned)grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, tb, a);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pba_fwd_kernel launch");
@@ -505,7 +510,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_zero_kernel launch");
             {
                 ProfScope ps(K_DBIAS, s);
-                pba::pba_dbias_kernel<CP><<<(unsigned)g2, DT::THREADS, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
             // (the last CTA of every tile sums the split partials in split order)

@@ -162,35 +162,30 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
     }
 }
 
-// P and dS of NK keys (NK = 64: one half of a 128-key tile; NK = 32: one quarter) for one
-// query row, in KC-key chunks.
-//   tS, tdP: this lane's S and dP columns of those keys in TMEM; bias_row: the row's 64-key
-//   half of the bias tile (bf16, a 128-byte swizzled shared-memory row) and c8_base the
-//   first of its 16-byte chunks that the keys start at (0, or 4 for the second quarter of
-//   a half); mw0, mw1: mask words of keys 0-31 and 32-63 of the NK (all ones when `full`);
-//   sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
+// P and dS of 64 keys (one half of a 128-key tile) for one query row, in KC-key chunks.
+//   tS, tdP: this lane's S and dP columns in TMEM; bias_row: the row's 64 bf16 bias values
+//   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
+//   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
 //   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
 // For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS.
-// The masked and the unmasked loop are separate instantiations (MASKED), chosen per call by
-// `full`, so that tiles without masked keys carry no per-key select.
-template <int NK, int KC, bool MASKED, typename Use>
-__device__ __forceinline__ void p_ds_keys_impl(uint32_t tS, uint32_t tdP, uint32_t bias_row, int c8_base,
-                                               int row, bool has_bias, uint32_t mw0, uint32_t mw1,
-                                               float sl2e, float lse2, float D, Use &&use) {
-    // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers
+template <int KC, typename Use>
+__device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
+                                          bool has_bias, uint32_t mw0, uint32_t mw1, bool full,
+                                          float sl2e, float lse2, float D, Use &&use) {
+    // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers; the main kernel
+    // uses 16 to stay within the 128 registers a thread has at 512 threads per CTA
     static_assert(KC == 16 || KC == 32, "chunk");
-    static_assert(NK == 32 || NK == 64, "keys");
     const float2 sl2 = make_float2(sl2e, sl2e), l2e2 = make_float2(kLog2eB, kLog2eB);
     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
 #pragma unroll
-    for (int q = 0; q < NK / KC; ++q) {
+    for (int q = 0; q < 64 / KC; ++q) {
         uint32_t r[2 * KC];   // S of keys KC q .. KC q + KC - 1 in r[0, KC), dP in r[KC, 2 KC)
         if constexpr (KC == 32) tmem_ld32x2(tS + q * KC, tdP + q * KC, r);
         else tmem_ld16x2(tS + q * KC, tdP + q * KC, r);
         const uint32_t mw = ((q * KC) < 32 ? mw0 : mw1) >> ((q * KC) & 31);
 #pragma unroll
         for (int c2 = 0; c2 < KC / 8; ++c2) {
-            const int c8 = c8_base + q * (KC / 8) + c2;
+            const int c8 = q * (KC / 8) + c2;
             uint4 bw = make_uint4(0, 0, 0, 0);
             if (has_bias) bw = lds128(bias_row + ((c8 ^ (row & 7)) << 4));
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
@@ -200,7 +195,7 @@ __device__ __forceinline__ void p_ds_keys_impl(uint32_t tS, uint32_t tdP, uint32
                 float2 u = ffma2(make_float2(bf16lo(bb[e]), bf16hi(bb[e])), l2e2, nl2);
                 u = ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, u);
                 float2 p = make_float2(ex2(u.x), ex2(u.y));
-                if constexpr (MASKED) {
+                if (!full) {
                     p.x = ((mw >> k) & 1u) ? p.x : 0.f;
                     p.y = ((mw >> (k + 1)) & 1u) ? p.y : 0.f;
                 }
@@ -209,16 +204,6 @@ __device__ __forceinline__ void p_ds_keys_impl(uint32_t tS, uint32_t tdP, uint32
             }
         }
     }
-}
-
-template <int NK, int KC, typename Use>
-__device__ __forceinline__ void p_ds_keys(uint32_t tS, uint32_t tdP, uint32_t bias_row, int c8_base,
-                                          int row, bool has_bias, uint32_t mw0, uint32_t mw1,
-                                          bool full, float sl2e, float lse2, float D, Use &&use) {
-    if (full)
-        p_ds_keys_impl<NK, KC, false>(tS, tdP, bias_row, c8_base, row, has_bias, mw0, mw1, sl2e, lse2, D, use);
-    else
-        p_ds_keys_impl<NK, KC, true>(tS, tdP, bias_row, c8_base, row, has_bias, mw0, mw1, sl2e, lse2, D, use);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -451,15 +436,13 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (!okk) return false;
                 tc_fence_after();
                 const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                const uint32_t sDO = sQ + T::TILE_BYTES;
-                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
-                const uint32_t sV = sbase + T::OFF_V + x * T::TILE_BYTES;
+                const uint64_t dQd = sdesc(sQ, 16, SBO, T::SWZ), dDO = sdesc(sQ + T::TILE_BYTES, 16, SBO, T::SWZ);
+                const uint64_t dK = sdesc(sbase + T::OFF_K + x * T::TILE_BYTES, 16, SBO, T::SWZ);
+                const uint64_t dV = sdesc(sbase + T::OFF_V + x * T::TILE_BYTES, 16, SBO, T::SWZ);
 #pragma unroll
-                for (int kk = 0; kk < CP / 16; ++kk) {
-                    umma_ss(tbase + T::T_S, sdesc(sQ + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(sK + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
-                    umma_ss(tbase + T::T_DP, sdesc(sDO + kk * 32, 16, SBO, T::SWZ),
-                            sdesc(sV + kk * 32, 16, SBO, T::SWZ), id_s, kk > 0);
+                for (int kk = 0; kk < CP / 16; ++kk) {   // K steps of 16 channels: 32 bytes on
+                    umma_ss(tbase + T::T_S, sdesc_add(dQd, kk * 32), sdesc_add(dK, kk * 32), id_s, kk > 0);
+                    umma_ss(tbase + T::T_DP, sdesc_add(dDO, kk * 32), sdesc_add(dV, kk * 32), id_s, kk > 0);
                 }
                 umma_commit(b_sd_full);
                 return true;
@@ -472,13 +455,14 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     okk = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
                 if (!okk) return false;
                 tc_fence_after();
-                const uint32_t sK = sbase + T::OFF_K + x * T::TILE_BYTES;
+                const uint64_t dA = sdesc(sDS, 16, 1024, kSw128);
+                const uint64_t dB = sdesc(sbase + T::OFF_K + x * T::TILE_BYTES, T::TILE_BYTES, SBO, T::SWZ);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half
-                    const uint32_t a_addr = sDS + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc(a_addr, 16, 1024, kSw128),
-                            sdesc(sK + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_q, kk > 0);
+                    // K steps over 16 keys: A (dS, K-major) advances 32 B within a 64-key half,
+                    // B (K, MN-major) 16 rows
+                    umma_ss(tbase + T::T_DQ + (t & 1) * CP, sdesc_add(dA, (kk >> 2) * 16384 + (kk & 3) * 32),
+                            sdesc_add(dB, kk * 16 * T::ROWB), id_q, kk > 0);
                 }
                 umma_commit(b_ps_free);
                 umma_commit(b_dq_full(t & 1));
@@ -525,16 +509,15 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     }
                     tc_fence_after();
                     const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
-                    const uint32_t sB = is_dv ? sQ + T::TILE_BYTES : sQ;   // dOa or Q
+                    const uint64_t dA = sdesc(sA, 16384, 1024, kSw128);
+                    const uint64_t dB = sdesc(is_dv ? sQ + T::TILE_BYTES : sQ, T::TILE_BYTES, SBO, T::SWZ);   // dOa or Q
                     const uint32_t tD = tbase + T::T_DK + d * 2 * CP + (is_dv ? CP : 0);
+                    // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
+                    // B (dOa / Q, MN-major) rows advance 16 rows
+                    umma_ss(tD, dA, dB, id_kv, i > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        // K steps over 16 queries: A (P^T / dS^T, MN-major) rows advance 2 KB,
-                        // B (dOa / Q, MN-major) rows advance 16 rows
-                        umma_ss(tD, sdesc(sA + kk * 2048, 16384, 1024, kSw128),
-                                sdesc(sB + kk * 16 * T::ROWB, T::TILE_BYTES, SBO, T::SWZ), id_kv,
-                                (i > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 1; kk < 8; ++kk)
+                        umma_ss(tD, sdesc_add(dA, kk * 2048), sdesc_add(dB, kk * 16 * T::ROWB), id_kv, 1u);
                     umma_commit(b_ps_free);
                     umma_commit(b_q_empty(st));
                     if (i == ni - 1) umma_commit(b_dkv_full(d));
@@ -575,8 +558,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
                 uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
                 const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
-                p_ds_keys<64, 16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
-                          0, row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
+                p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
+                          row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
                           [&](int c, float2 p, float2 ds) {
                               pp[c >> 1] = pack_bf16x2(p.x, p.y);
                               dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
@@ -806,15 +789,10 @@ struct DbTraits {
     static constexpr int SMEM_BYTES = OFF_MASK + NS * 32 + 1024;
     static constexpr uint32_t SWZ = CP == 64 ? kSw128 : (CP == 32 ? kSw64 : kSw32);
     static constexpr uint32_t ROWB = CP * 2;
-    // warps 0-15: element-wise, four warpgroups of one 32-key quarter each (four warps per
-    // scheduler keep the exponential unit fed); warp 16 TMA producer; warp 17 TMEM and MMA
-    static constexpr int EW_THREADS = 512;
-    static constexpr int THREADS = EW_THREADS + 64;
-    static constexpr int W_PROD = 16, W_MMA = 17;
 };
 
 template <int CP>
-__global__ void __launch_bounds__(DbTraits<CP>::THREADS)
+__global__ void __launch_bounds__(320, 1)
 pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
@@ -853,16 +831,16 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(b_drain, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_sd_full(x), 1);
-            mbar_init(b_sd_free(x), T::EW_THREADS);
+            mbar_init(b_sd_free(x), 256);
         }
         for (int x = 0; x < NS; ++x) {
             mbar_init(b_full(x), 1);
-            mbar_init(b_empty(x), 1 + T::EW_THREADS);
+            mbar_init(b_empty(x), 1 + 256);
         }
         s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == T::W_MMA) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(&s_tmem_base), 512);
         tmem_relinquish();
     }
@@ -873,7 +851,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     volatile int *abort_flag = &s_abort;
     int n_done = 0;   // rows b whose stage loads were issued: [0, n_done)
 
-    if (warp == T::W_PROD) {
+    if (warp == 8) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -914,7 +892,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
             n_done = n + 1;
         }
-    } else if (warp == T::W_MMA) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
@@ -942,17 +920,16 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------------ elementwise
-        // warpgroup e owns keys [32 e, 32 e + 32) of the tile for all 128 query rows
         const int e = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const float sl2e = a.scale * kLog2eB;
-        float2 acc[16];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
+        float2 acc[32];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
 #pragma unroll
-        for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.f, 0.f);
+        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
         bool ok = mbar_wait(b_bias, 0, abort_flag, SITE_DB_EW);
         ok = __all_sync(0xffffffffu, ok);
-        const uint32_t bias_row = sbase + T::OFF_BIAS + (e >> 1) * 16384 + row * 128;
+        const uint32_t bias_row = sbase + T::OFF_BIAS + e * 16384 + row * 128;
         for (int n = 0; n < nb && ok; ++n) {
             const int st = n % NS, x = n & 1;
             ok = mbar_wait(b_sd_full(x), (n >> 1) & 1, abort_flag, SITE_DB_EW);
@@ -962,11 +939,10 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tc_fence_after();
             const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
             const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
-            const uint32_t mwe = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK)[st * 8 + e];
-            p_ds_keys<32, 16>(tbase + x * 256 + e * 32 + lane_off, tbase + x * 256 + 128 + e * 32 + lane_off,
-                              bias_row, (e & 1) * 4, row, a.has_bias != 0, mwe, 0u, mwe == 0xffffffffu,
-                              sl2e, rs.x, rs.y,
-                              [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
+            const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
+            p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
+                      bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
+                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
             tc_fence_before();
             mbar_arrive(b_sd_free(x));
             mbar_arrive(b_empty(st));
@@ -974,9 +950,9 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (ok) {
             // this split's partial tile: [split][h][tile][128][128]
             float *dst = a.dbias_part +
-                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 32;
+                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 64;
 #pragma unroll
-            for (int c = 0; c < 16; c += 2)
+            for (int c = 0; c < 32; c += 2)
                 *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
             __threadfence();   // this thread's partial row, before the tile counter moves
         }
@@ -985,18 +961,18 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) {
-        if (warp == T::W_PROD && lane == 0) {
+        if (warp == 8 && lane == 0) {
             mbar_wait_drain(b_bias, 0);
             for (int nn = max(0, n_done - NS); nn < n_done; ++nn) mbar_wait_drain(b_full(nn % NS), (nn / NS) & 1);
         }
-        if (warp == T::W_MMA && lane == 0) {
+        if (warp == 9 && lane == 0) {
             umma_commit(b_drain);
             mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
         __syncthreads();
     }
-    if (warp == T::W_MMA) {
+    if (warp == 9) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tbase, 512);
@@ -1014,36 +990,35 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (!s_last) return;
     __threadfence();
     // Only the tile's valid part (rows i < Nq, four-key groups starting below Nk) is summed,
-    // U positions of four keys per thread at a time.  Every position adds its partials in
-    // split order, starting from zero; the loads of four splits of the U positions are all
-    // issued before their additions, so their latencies overlap.
-    constexpr int U = 2;
+    // four positions per thread at a time.  Every position adds its partials in split order,
+    // starting from zero; the loads of four splits of the four positions are all issued
+    // before their additions, so their latencies overlap.
     const long long plane = (long long)a.H * a.ntiles * 128 * 128;
     const float *part = a.dbias_part + ((long long)h * a.ntiles + bt) * 128 * 128;
     const int groups = (min(128, a.Nk - j0) + 3) >> 2;
     const int nv = min(128, a.Nq - i0) * groups;
-    for (int v0 = threadIdx.x; v0 < nv; v0 += U * blockDim.x) {
-        int off[U];   // row * 128 + column within the tile, or -1
-        float4 sum[U];
+    for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * blockDim.x) {
+        int off[4];   // row * 128 + column within the tile, or -1
+        float4 sum[4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < 4; ++u) {
             const int v = v0 + u * blockDim.x;
             off[u] = v < nv ? (v / groups) * 128 + (v % groups) * 4 : -1;
             sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int q = 0;
         for (; q + 4 <= a.splits; q += 4) {
-            float4 x[4][U];
+            float4 x[4][4];
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
-                for (int u = 0; u < U; ++u)
+                for (int u = 0; u < 4; ++u)
                     x[s][u] = off[u] >= 0 ? __ldcg(reinterpret_cast<const float4 *>(part + (q + s) * plane + off[u]))
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     sum[u].x += x[s][u].x;
                     sum[u].y += x[s][u].y;
                     sum[u].z += x[s][u].z;
@@ -1052,7 +1027,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         for (; q < a.splits; ++q) {
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 if (off[u] < 0) continue;
                 const float4 x = __ldcg(reinterpret_cast<const float4 *>(part + q * plane + off[u]));
                 sum[u].x += x.x;
@@ -1062,7 +1037,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < 4; ++u) {
             if (off[u] < 0) continue;
             const int i = i0 + (off[u] >> 7), j = j0 + (off[u] & 127);
             float *dst = a.dbias + ((long long)h * a.Nq + i) * a.Nk + j;

@@ -251,6 +251,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)swz << 61);
 }
 
+// The descriptor of the same matrix `bytes` further on: the start address field holds
+// (address >> 4) in its low 14 bits, and shared-memory addresses stay below 2^18, so adding
+// bytes >> 4 (a multiple of 16 bytes) never carries out of the field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 // ------------------------------------------------------------------------------------
 // TMEM <-> registers (32 lanes x 32-bit pattern: thread t of the warp owns lane t)
 // Each load waits for its own completion, so the registers are valid on return.
@@ -260,19 +265,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 #define PBA_W8(a, i) "r"(a[i]), "r"(a[i + 1]), "r"(a[i + 2]), "r"(a[i + 3]), \
                      "r"(a[i + 4]), "r"(a[i + 5]), "r"(a[i + 6]), "r"(a[i + 7])
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : PBA_R8(r, 0)
-        : "r"(taddr)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-                 PBA_W8(r, 0)
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -383,18 +375,16 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t a1, uint32_t (
         : "memory");
 }
 
-// Load CP fp32 columns (CP = 8, 16, 32 or 64) of this thread's lane.
+// Load CP fp32 columns (CP = 16, 32 or 64) of this thread's lane.
 template <int CP>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CP]) {
-    if constexpr (CP == 8) tmem_ld8(taddr, r);
-    else if constexpr (CP == 16) tmem_ld16(taddr, r);
+    if constexpr (CP == 16) tmem_ld16(taddr, r);
     else if constexpr (CP == 32) tmem_ld32(taddr, r);
     else tmem_ld64(taddr, r);
 }
 template <int CP>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[CP]) {
-    if constexpr (CP == 8) tmem_st8(taddr, r);
-    else if constexpr (CP == 16) tmem_st16(taddr, r);
+    if constexpr (CP == 16) tmem_st16(taddr, r);
     else if constexpr (CP == 32) tmem_st32(taddr, r);
     else tmem_st64(taddr, r);
 }
@@ -407,11 +397,34 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// Packed two-lane fp32 arithmetic (one instruction for two values), through the compiler's
-// sm_100 builtins so that operand pairs stay in place in the register file.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// Packed two-lane fp32 arithmetic (one instruction for two values).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

@@ -43,121 +43,103 @@ class Bar:
 
 
 class FwdSim:
-    """The persistent forward kernel (pba_fwd.cuh): a producer (Q tile per slot, K and V rings,
-    bias tiles), a mask-fold warp, one MMA issuer per row group, and two row groups g
-    (the slots s with s & 1 == g), each of two key halves e that exchange the row maximum
-    at every step and the row sums at every item's end through a two-slot buffer guarded
-    by one barrier per slot (two arrivals).  Each softmax half is its own role here (the
-    four row quads of a half behave alike and share every barrier but their exchange
-    barriers, so one quad stands for all)."""
-
-    def __init__(self, nJ, nbs, KVS, BS, BC, seed, row_mask=False, plant=None):
-        # KVS: K and V stages of each row group's own rings
+    def __init__(self, nJ, nbs, KVS, BS, seed, row_mask=False, plant=None):
         self.rng = random.Random(seed)
         self.plant = plant
-        self.nJ, self.nbs, self.KVS, self.BS, self.BC = nJ, nbs, KVS, BS, BC
-        assert all(1 <= nb <= BC for nb in nbs)
+        self.nJ, self.nbs, self.KVS, self.BS = nJ, nbs, KVS, BS
         self.row_mask = row_mask
         self.items = len(nbs)
+        # global step list: (item, j, s)
+        self.steps = [(n, j, s) for n, nb in enumerate(nbs) for j in range(nJ) for s in range(nb)]
+        self.K = len(self.steps)
         self.tiles = [(n, j) for n in range(self.items) for j in range(nJ)]
         B = Bar
-        self.q_full = [B("q_full%d" % i, 1) for i in range(BC)]
-        self.q_empty = [B("q_empty%d" % i, 1) for i in range(BC)]
-        self.k_full = [[B("k_full%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
-        self.k_empty = [[B("k_empty%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
-        self.v_full = [[B("v_full%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
-        self.v_empty = [[B("v_empty%d%d" % (g, i), 1) for i in range(KVS)] for g in range(2)]
+        self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
+        self.k_full = [B("k_full%d" % i, 1) for i in range(KVS)]
+        self.k_empty = [B("k_empty%d" % i, 1) for i in range(KVS)]
+        self.v_full = [B("v_full%d" % i, 1) for i in range(KVS)]
+        self.v_empty = [B("v_empty%d" % i, 1) for i in range(KVS)]
         self.bias_full = [B("bias_full%d" % i, 1) for i in range(BS)]
         self.bias_ready = [B("bias_ready%d" % i, 1) for i in range(BS)]
-        self.bias_empty = [B("bias_empty%d" % i, 4) for i in range(BS)]   # 2 groups x 2 halves
-        self.s_full = [B("s_full%d" % g, 1) for g in range(2)]
-        self.s_free = [B("s_free%d" % g, 2) for g in range(2)]
-        self.p_full = [B("p_full%d" % g, 2) for g in range(2)]
-        self.p_free = [B("p_free%d" % g, 1) for g in range(2)]
-        self.ofinal = [B("ofinal%d" % g, 1) for g in range(2)]
-        self.xbar = [[B("xbar%d%d" % (g, par), 2) for par in range(2)] for g in range(2)]
-        self.tma, self.mq_g = [], [[], []]
-        self.q_slot = [None] * BC; self.q_readers = [0] * BC
-        self.k_stage = [[None] * KVS for _ in range(2)]; self.k_readers = [[0] * KVS for _ in range(2)]
-        self.v_stage = [[None] * KVS for _ in range(2)]; self.v_readers = [[0] * KVS for _ in range(2)]
-        self.words = [[None] * KVS for _ in range(2)]; self.words_readers = [[0] * KVS for _ in range(2)]
+        self.bias_empty = [B("bias_empty%d" % i, 1) for i in range(BS)]
+        self.s_full, self.s_free = B("s_full", 1), B("s_free", 1)
+        self.p_full, self.p_free = B("p_full", 1), B("p_free", 1)
+        self.ofinal = B("ofinal", 1)
+        self.tma, self.mq_qk, self.mq_pv = [], [], []
+        self.q_item = None; self.q_readers = 0
+        self.k_stage = [None] * KVS; self.k_readers = [0] * KVS
+        self.v_stage = [None] * KVS; self.v_readers = [0] * KVS
+        self.words = [None] * KVS; self.words_readers = [0] * KVS
         self.bias_tile = [None] * BS; self.bias_state = ["free"] * BS; self.bias_left = [0] * BS
-        self.S_step = [None, None]; self.S_reading = [0, 0]; self.S_pend = [0, 0]
-        self.P_step = [{}, {}]; self.P_pend = [0, 0]
-        self.O_item = {}; self.O_pend = {}; self.O_reading = set()
-        self.xval = [[[None, None] for _ in range(2)] for _ in range(2)]   # [g][par][e] = exchange id
-        self.done = [[[], []], [[], []]]
+        self.S_step = None; self.S_reading = False; self.S_pend = 0
+        self.P_step = None; self.P_pend = 0
+        self.O_item = {}       # slot -> item whose products it holds
+        self.O_pend = {}       # slot -> PVs in flight
+        self.O_reading = set()
+        self.done_items = []
 
     def step_async(self):
         ch = []
         if self.tma: ch.append("tma")
-        for g in range(2):
-            if self.mq_g[g]: ch.append(g)
+        if self.mq_qk: ch.append("qk")
+        if self.mq_pv: ch.append("pv")
         if not ch: return
         c = self.rng.choice(ch)
         if c == "tma":
             bar, n, fn = self.tma.pop(self.rng.randrange(len(self.tma)))
             fn(); bar.complete_tx(n)
         else:
-            kind, x = self.mq_g[c].pop(0)
+            q = self.mq_qk if c == "qk" else self.mq_pv
+            kind, x = q.pop(0)
             if kind == "mma": x()
             else: x.arrive()
 
     def producer(self):
         KVS, BS = self.KVS, self.BS
-        kg = 0; jg = 0; qloads = [0] * self.BC
+        kg = 0; jg = 0
         def load_bias(jg, tile):
             bs = jg % BS
             if jg >= BS:
                 while not self.bias_empty[bs].test(jg // BS - 1): yield
-            assert self.bias_state[bs] in ("free", "folded") and self.bias_left[bs] == 0, \
-                "bias buffer refilled while it is read"
+            assert self.bias_state[bs] in ("free", "folded") and self.bias_left[bs] == 0
             self.bias_state[bs] = "loading"; self.bias_tile[bs] = tile
             self.bias_full[bs].arrive_tx(1)
             self.tma.append((self.bias_full[bs], 1, lambda bs=bs: self.bias_state.__setitem__(bs, "landed")))
             yield
-        gsteps = [0, 0]
-        def load_k(k, g, gs):
-            st, use = gs % KVS, gs // KVS
+        def load_k(k):
+            st, use = k % KVS, k // KVS
             if use >= 1:
-                while not self.k_empty[g][st].test(use - 1): yield
-            assert self.k_readers[g][st] == 0
-            self.k_stage[g][st] = None
-            self.k_full[g][st].arrive_tx(1)
-            self.tma.append((self.k_full[g][st], 1, lambda st=st, k=k, g=g: self.k_stage[g].__setitem__(st, k)))
+                while not self.k_empty[st].test(use - 1): yield
+            assert self.k_readers[st] == 0
+            self.k_stage[st] = None
+            self.k_full[st].arrive_tx(1)
+            self.tma.append((self.k_full[st], 1, lambda st=st, k=k: self.k_stage.__setitem__(st, k)))
             yield
-        def load_v(k, g, gs):
-            st, use = gs % KVS, gs // KVS
+        def load_v(k):
+            st, use = k % KVS, k // KVS
             if use >= 1:
-                while not self.v_empty[g][st].test(use - 1): yield
-            assert self.v_readers[g][st] == 0 and self.words_readers[g][st] == 0
-            self.v_stage[g][st] = None; self.words[g][st] = k
-            self.v_full[g][st].arrive_tx(1)
-            self.tma.append((self.v_full[g][st], 1, lambda st=st, k=k, g=g: self.v_stage[g].__setitem__(st, k)))
+                while not self.v_empty[st].test(use - 1): yield
+            assert self.v_readers[st] == 0 and self.words_readers[st] == 0
+            self.v_stage[st] = None; self.words[st] = k
+            self.v_full[st].arrive_tx(1)
+            self.tma.append((self.v_full[st], 1, lambda st=st, k=k: self.v_stage.__setitem__(st, k)))
             yield
         for n, nb in enumerate(self.nbs):
             Kn = self.nJ * nb
             k0 = kg
-            # each step's group and its step count within the group
-            grp = [(kl % nb) & 1 for kl in range(Kn)]
-            gsk = []
-            for kl in range(Kn):
-                gsk.append(gsteps[grp[kl]]); gsteps[grp[kl]] += 1
             yield from load_bias(jg, (n, 0))
-            yield from load_k(k0, grp[0], gsk[0])
-            for s in range(nb):
-                # slot s's Q tile: the previous item's last Q K^T on the slot must be done
-                if qloads[s] >= 1 and self.plant != "no_q_empty_wait":
-                    while not self.q_empty[s].test(qloads[s] - 1): yield
-                assert self.q_readers[s] == 0, "Q refilled while a Q K^T reads it"
-                self.q_slot[s] = None
-                self.q_full[s].arrive_tx(1)
-                self.tma.append((self.q_full[s], 1, lambda s=s, n=n: self.q_slot.__setitem__(s, n)))
-                qloads[s] += 1
-                yield
+            yield from load_k(k0)
+            # the item's Q tiles: the previous item's Q K^T products must be done
+            if n >= 1 and self.plant != "no_q_empty_wait":
+                while not self.q_empty.test(n - 1): yield
+            assert self.q_readers == 0, "Q refilled while a Q K^T reads it"
+            self.q_item = None
+            self.q_full.arrive_tx(1)
+            self.tma.append((self.q_full, 1, lambda n=n: setattr(self, "q_item", n)))
+            yield
             for kl in range(Kn):
-                if kl + 1 < Kn: yield from load_k(k0 + kl + 1, grp[kl + 1], gsk[kl + 1])
-                yield from load_v(k0 + kl, grp[kl], gsk[kl])
+                if kl + 1 < Kn: yield from load_k(k0 + kl + 1)
+                yield from load_v(k0 + kl)
                 if kl + 1 < Kn and (kl + 1) % nb == 0:
                     yield from load_bias(jg + (kl + 1) // nb, (n, (kl + 1) // nb))
             kg += Kn; jg += self.nJ
@@ -167,158 +149,111 @@ class FwdSim:
             bs = jg % self.BS
             while not self.bias_full[bs].test(jg // self.BS): yield
             assert self.bias_state[bs] == "landed" and self.bias_tile[bs] == tile
-            self.bias_state[bs] = "folded"; self.bias_left[bs] = 4
+            self.bias_state[bs] = "folded"; self.bias_left[bs] = self.nbs[tile[0]]
             yield
             self.bias_ready[bs].arrive()
 
-    def issuer(self, g):
-        # row group g's issuer: Q K^T of each of the group's steps, then P V of the group's
-        # previous step (so a step's scores never wait behind the previous step's P V)
-        kg = 0; gk = 0; quse = [0] * self.BC
-        q = self.mq_g[g]
-        pend = None
-        def pv(pk, pj, ps, pst, pn, pnb, pgk):
-            while not self.p_full[g].test(pgk): yield
-            while not self.v_full[g][pst].test(pgk // self.KVS): yield
-            assert self.v_stage[g][pst] == pk
-            if pj == 0:   # first tile: the slot starts over
-                assert not any(x[0] == ps for x in self.O_reading), "O overwritten while the epilogue reads it"
-                self.O_item[ps] = pn
-            assert self.O_item[ps] == pn
-            self.v_readers[g][pst] += 1; self.P_pend[g] += 1; self.O_pend[ps] = self.O_pend.get(ps, 0) + 1
-            def ex(st=pst, k=pk, s=ps, n=pn):
-                assert self.P_step[g] == {0: k, 1: k}, "P V read a P that is not this step's"
-                assert self.v_stage[g][st] == k and self.O_item[s] == n
-                assert not any(x[0] == s for x in self.O_reading)
-                self.v_readers[g][st] -= 1; self.P_pend[g] -= 1; self.O_pend[s] -= 1
-            q.append(("mma", ex))
-            q.append(("commit", self.p_free[g]))
-            q.append(("commit", self.v_empty[g][pst]))
-            if pj == self.nJ - 1 and ps + 2 >= pnb and self.plant != "early_ofinal":
-                q.append(("commit", self.ofinal[g]))
-            if self.plant == "early_ofinal" and pj == 0 and ps == g:
-                q.append(("commit", self.ofinal[g]))
-            yield
+    def issuer_qk(self):
+        kg = 0
         for n, nb in enumerate(self.nbs):
             Kn = self.nJ * nb
-            if nb <= g:
-                # no row of this group in the item: its last P V goes out now (the group's
-                # epilogue waits for it, and the item's loads wait for that epilogue's group
-                # to hand back the item's bias tiles)
-                if pend is not None and self.plant != "keep_pending":
-                    yield from pv(*pend); pend = None
-                if self.plant == "idle_ofinal":
-                    # (a planted mistake: completing the barrier for an item without rows of
-                    # the group lets it run two phases ahead of the group's epilogue)
-                    q.append(("commit", self.ofinal[g]))
-                yield
+            while not self.q_full.test(n): yield
             for kl in range(Kn):
-                k = kg + kl; j, s = divmod(kl, nb)
-                if s & 1 != g: continue
-                st = gk % self.KVS
-                if gk > 0 and self.plant != "no_s_free_wait":
-                    while not self.s_free[g].test(gk - 1): yield
-                while not self.k_full[g][st].test(gk // self.KVS): yield
-                if j == 0:
-                    while not self.q_full[s].test(quse[s]): yield
-                assert self.k_stage[g][st] == k and self.q_slot[s] == n
-                self.q_readers[s] += 1; self.k_readers[g][st] += 1; self.S_pend[g] += 1
-                def ex(st=st, k=k, n=n, s=s):
-                    assert self.S_reading[g] == 0, "S overwritten while the softmax reads it"
-                    assert self.k_stage[g][st] == k and self.q_slot[s] == n
-                    self.q_readers[s] -= 1; self.k_readers[g][st] -= 1; self.S_pend[g] -= 1
-                    self.S_step[g] = k
-                q.append(("mma", ex))
-                q.append(("commit", self.s_full[g]))
-                q.append(("commit", self.k_empty[g][st]))
-                if j == self.nJ - 1:
-                    q.append(("commit", self.q_empty[s]))
+                k = kg + kl; st = k % self.KVS
+                if k > 0:
+                    while not self.s_free.test(k - 1): yield
+                while not self.k_full[st].test(k // self.KVS): yield
+                assert self.k_stage[st] == k and self.q_item == n
+                self.q_readers += 1; self.k_readers[st] += 1; self.S_pend += 1
+                def ex(st=st, k=k, n=n):
+                    assert not self.S_reading
+                    assert self.k_stage[st] == k and self.q_item == n
+                    self.q_readers -= 1; self.k_readers[st] -= 1; self.S_pend -= 1
+                    self.S_step = k
+                self.mq_qk.append(("mma", ex))
+                self.mq_qk.append(("commit", self.s_full))
+                self.mq_qk.append(("commit", self.k_empty[st]))
+                if kl == Kn - 1:
+                    self.mq_qk.append(("commit", self.q_empty))
                 yield
-                if pend is not None:
-                    yield from pv(*pend)
-                pend = (k, j, s, st, n, nb, gk)
-                gk += 1
-            for s in range(nb): quse[s] += 1
             kg += Kn
-        if pend is not None:
-            yield from pv(*pend)
 
-    def softmax(self, g, e):
-        kg = 0; jg = 0; gk = 0; xc = 0
-        gitems = 0   # items with a row of this group: the phases of its ofinal barrier
-        def exchange(tag):
-            nonlocal xc
-            par = xc & 1
-            self.xval[g][par][e] = (xc, tag)
-            self.xbar[g][par].arrive()
-            while not self.xbar[g][par].test(xc >> 1): yield
-            yield
-            assert self.xval[g][par][1 - e] == (xc, tag), "exchange slot rewritten before it was read"
-            xc += 1
+    def issuer_pv(self):
+        kg = 0
         for n, nb in enumerate(self.nbs):
-            mine = [s for s in range(nb) if s % 2 == g]
+            Kn = self.nJ * nb
+            for kl in range(Kn):
+                k = kg + kl; st = k % self.KVS; s = kl % nb
+                while not self.p_full.test(k): yield
+                while not self.v_full[st].test(k // self.KVS): yield
+                assert self.v_stage[st] == k
+                if kl < nb:   # first tile: the slot starts over
+                    assert s not in self.O_reading, "O overwritten while the epilogue reads it"
+                    self.O_item[s] = n
+                assert self.O_item[s] == n
+                self.v_readers[st] += 1; self.P_pend += 1; self.O_pend[s] = self.O_pend.get(s, 0) + 1
+                def ex(st=st, k=k, s=s, n=n):
+                    assert self.P_step == k and self.v_stage[st] == k and self.O_item[s] == n
+                    assert s not in self.O_reading
+                    self.v_readers[st] -= 1; self.P_pend -= 1; self.O_pend[s] -= 1
+                self.mq_pv.append(("mma", ex))
+                self.mq_pv.append(("commit", self.p_free))
+                self.mq_pv.append(("commit", self.v_empty[st]))
+                yield
+            self.mq_pv.append(("commit", self.ofinal))
+            kg += Kn
+
+    def softmax(self):
+        kg = 0; jg = 0
+        for n, nb in enumerate(self.nbs):
             for j in range(self.nJ):
                 bs = (jg + j) % self.BS
-                if not mine:
-                    while not self.bias_ready[bs].test((jg + j) // self.BS): yield
-                    self.bias_left[bs] -= 1
-                    self.bias_empty[bs].arrive()
-                    yield
-                    continue
-                for t, s in enumerate(mine):
-                    k = kg + j * nb + s; st = gk % self.KVS
-                    while not self.s_full[g].test(gk): yield
-                    if t == 0:
+                for s in range(nb):
+                    k = kg + j * nb + s; st = k % self.KVS
+                    while not self.s_full.test(k): yield
+                    if s == 0:
                         while not self.bias_ready[bs].test((jg + j) // self.BS): yield
                     if self.row_mask:
-                        while not self.v_full[g][st].test(gk // self.KVS): yield
-                        assert self.words[g][st] == k
-                        self.words_readers[g][st] += 1
-                    assert self.S_step[g] == k and self.S_pend[g] == 0
-                    self.S_reading[g] += 1
+                        while not self.v_full[st].test(k // self.KVS): yield
+                        assert self.words[st] == k
+                        self.words_readers[st] += 1
+                    assert self.S_step == k and self.S_pend == 0
+                    self.S_reading = True
                     yield
-                    self.S_reading[g] -= 1
-                    self.s_free[g].arrive()
+                    self.S_reading = False
+                    self.s_free.arrive()
                     assert self.bias_tile[bs] == (n, j) and self.bias_state[bs] == "folded"
                     yield
-                    if t == len(mine) - 1:
-                        self.bias_left[bs] -= 1
+                    self.bias_left[bs] -= 1
+                    if s == nb - 1:
+                        assert self.bias_left[bs] == 0
                         self.bias_empty[bs].arrive()
-                    yield from exchange(("max", k))
-                    if gk > 0:
-                        while not self.p_free[g].test(gk - 1): yield
-                    assert self.P_pend[g] == 0, "P rewritten while a P V reads it"
+                    if k > 0:
+                        while not self.p_free.test(k - 1): yield
+                    assert self.P_pend == 0
                     assert self.O_pend.get(s, 0) == 0
-                    self.P_step[g][e] = k
+                    self.P_step = k
                     yield
                     if self.row_mask:
-                        assert self.words[g][st] == k
-                        self.words_readers[g][st] -= 1
-                    self.p_full[g].arrive()
-                    gk += 1
-            # epilogue of item n: the group's slots (no wait when it had none)
-            if mine:
-                while not self.ofinal[g].test(gitems): yield
-                gitems += 1
-            assert all(self.O_pend.get(s, 0) == 0 and self.O_item.get(s) == n for s in mine), \
-                "O read before its products are done"
-            yield from exchange(("sum", n))
-            for s in mine: self.O_reading.add((s, e))
+                        assert self.words[st] == k
+                        self.words_readers[st] -= 1
+                    self.p_full.arrive()
+            # epilogue of item n
+            while not self.ofinal.test(n): yield
+            assert all(self.O_pend.get(s, 0) == 0 for s in range(nb))
+            assert all(self.O_item.get(s) == n for s in range(nb))
+            self.O_reading = set(range(nb))
             yield
-            for s in mine: self.O_reading.discard((s, e))
-            self.done[g][e].append(n)
+            self.O_reading = set()
+            self.done_items.append(n)
             kg += self.nJ * nb; jg += self.nJ
 
     def run(self):
-        live = {"prod": self.producer(), "fold": self.fold(), "iss0": self.issuer(0),
-                "iss1": self.issuer(1)}
-        for g in range(2):
-            for e in range(2):
-                live["smx%d%d" % (g, e)] = self.softmax(g, e)
+        live = {"prod": self.producer(), "fold": self.fold(), "qk": self.issuer_qk(),
+                "pv": self.issuer_pv(), "smx": self.softmax()}
         idle = 0
-        while live or self.tma or self.mq_g[0] or self.mq_g[1]:
-            busy = self.tma or self.mq_g[0] or self.mq_g[1]
-            opts = list(live) + (["async"] * 2 if busy else [])
+        while live or self.tma or self.mq_qk or self.mq_pv:
+            opts = list(live) + (["async"] * 2 if (self.tma or self.mq_qk or self.mq_pv) else [])
             c = self.rng.choice(opts)
             if c == "async":
                 self.step_async(); idle = 0; continue
@@ -326,7 +261,8 @@ class FwdSim:
             except StopIteration: del live[c]
             idle += 1
             if idle > 200000: raise RuntimeError("deadlock: live=%s" % list(live))
-        assert self.done == [[list(range(self.items))] * 2] * 2
+        assert self.done_items == list(range(self.items))
+
 
 
 class BwdSim:
@@ -563,11 +499,11 @@ class BwdSim:
 class DbiasSim:
     """The dbias kernel (pba_bwd.cuh): one producer fills NS stages (Q, dOa, K and V tiles, row
     statistics and mask words of one broadcast row each) after the bias tile; one MMA issuer
-    computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; four
-    element-wise warpgroups (one 32-key quarter each, 128 arrivals each) read the TMEM buffer,
+    computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; nwg
+    element-wise warpgroups (128 / nwg keys each, 128 arrivals each) read the TMEM buffer,
     the stage's row statistics and mask words, and release both."""
 
-    def __init__(self, nb, NS, seed, plant=None, nwg=4):
+    def __init__(self, nb, NS, seed, plant=None, nwg=2):
         self.rng = random.Random(seed)
         self.plant = plant
         self.nb, self.NS, self.nwg = nb, NS, nwg

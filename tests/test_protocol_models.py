@@ -6,18 +6,15 @@ import pytest
 from pba_protocol_models import BwdSim, DbiasSim, FwdSim, PwaGemmSim
 
 
-# rings as the forward instantiates them (K/V stages per row group, bias buffers, slots):
-# c=16 -> (2, 2, 8), c=32 -> (2, 2, 4), c=64 -> (1, 2, 2); a deeper ring too
-@pytest.mark.parametrize("KVS,BS,BC", [(2, 2, 8), (2, 2, 4), (1, 2, 2), (3, 2, 4)])
-def test_forward_protocol(KVS, BS, BC):
+# ring depths as the forward instantiates them: c=16 -> (3, 2), c=32 -> (2, 2), c=64 -> (2, 1)
+@pytest.mark.parametrize("KVS,BS", [(2, 2), (3, 2), (2, 1)])
+def test_forward_protocol(KVS, BS):
     # items of nb rows over nJ key tiles (the last chunk of rows can be shorter)
-    chunks = [[BC], [BC, BC], [BC, 1], [1], [2, 1, BC], [BC, BC - 1, 1], [BC, 1, 1, 2, 1]]
-    for nJ in (1, 2, 3, 5):
-        for nbs in chunks:
-            nbs = [min(nb, BC) for nb in nbs]
+    for nJ in (1, 2, 3):
+        for nbs in ([1], [2, 2], [2, 1], [4, 4, 3], [1, 1, 1, 1]):
             for row_mask in (False, True):
-                for seed in range(8):
-                    FwdSim(nJ, nbs, KVS, BS, BC, seed, row_mask).run()
+                for seed in range(12):
+                    FwdSim(nJ, nbs, KVS, BS, seed, row_mask).run()
 
 
 # c=32 -> (2, 2, 2, 2), c=16 -> (3, 2, 2, 2), c=64 -> (2, 1, 1, 1); the last mixes depths
@@ -39,17 +36,9 @@ def _caught(make, seeds=40):
     return False
 
 
-def test_planted_forward_mistakes_are_caught():
-    # a slot's Q of the next item loaded before the previous item's last Q K^T on it is done
-    assert _caught(lambda seed: FwdSim(2, [4, 4, 4], 4, 2, 4, seed, plant="no_q_empty_wait"))
-    # a group's next Q K^T issued before its softmax has read the previous S
-    assert _caught(lambda seed: FwdSim(2, [4, 4], 4, 2, 4, seed, plant="no_s_free_wait"))
-    # the epilogue released before the group's last P V
-    assert _caught(lambda seed: FwdSim(2, [4, 4], 4, 2, 4, seed, plant="early_ofinal"))
-    # a group's completion barrier also completed for items without rows of the group
-    assert _caught(lambda seed: FwdSim(1, [4, 1, 1, 4], 4, 2, 4, seed, plant="idle_ofinal"))
-    # a group's last P V held back across an item without rows of the group: deadlock
-    assert _caught(lambda seed: FwdSim(2, [2, 1, 4], 4, 2, 4, seed, plant="keep_pending"))
+def test_planted_forward_mistake_is_caught():
+    # Q of the next item loaded before the previous item's last Q K^T is done
+    assert _caught(lambda seed: FwdSim(2, [2, 2, 2], 2, 2, seed, plant="no_q_empty_wait"))
 
 
 def test_planted_backward_mistakes_are_caught():
