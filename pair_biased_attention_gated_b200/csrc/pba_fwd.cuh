@@ -147,8 +147,11 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     const int warp = warp_id(), lane = lane_id();
     const bool row_mask = a.mask != nullptr && !a.mask_shared;
-    // item n of this CTA is blockIdx.x + n gridDim.x: query tile fastest, then the chunk of
-    // rows, then the head (CTAs running at the same time share K/V and bias tiles in L2)
+    // item n of this CTA is blockIdx.x + n gridDim.x: query tile fastest, then the head, then
+    // the chunk of rows.  CTAs running at the same time share K/V tiles in L2, and they cover
+    // every head of the rows they read: one 128-byte line of Q, K, V or the gate holds the
+    // channels of several heads (c = 32: 64 bytes per head), so with the heads apart in time
+    // each line would be fetched from DRAM once per head that reads it.
     struct FItem {
         int h, i0, b0, nb;
         int jlo, nj;   // the item's key tiles [jlo, jlo + nj)
@@ -157,9 +160,9 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         int idx = blockIdx.x + n * gridDim.x;
         const int itile = idx % a.nI;
         idx /= a.nI;
-        const int chunk = idx % a.nChunks;
         FItem it;
-        it.h = idx / a.nChunks;
+        it.h = idx % a.H;
+        const int chunk = idx / a.H;
         it.i0 = itile * 128;
         it.b0 = chunk * BC;
         it.nb = min(BC, a.B - it.b0);
