@@ -167,11 +167,13 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
 //   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
 //   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
 //   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
-// For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS.
-template <int KC, typename Use>
+// For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS;
+// `loaded()` is called once the last chunk's S and dP are in registers (the TMEM columns
+// may then be handed back before the chunk is computed).
+template <int KC, typename Use, typename Loaded>
 __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
                                           bool has_bias, uint32_t mw0, uint32_t mw1, bool full,
-                                          float sl2e, float lse2, float D, Use &&use) {
+                                          float sl2e, float lse2, float D, Use &&use, Loaded &&loaded) {
     // KC-key chunks (32 or 16): S and dP of one chunk take 2 KC registers; the main kernel
     // uses 16 to stay within the 128 registers a thread has at 512 threads per CTA
     static_assert(KC == 16 || KC == 32, "chunk");
@@ -182,6 +184,7 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
         uint32_t r[2 * KC];   // S of keys KC q .. KC q + KC - 1 in r[0, KC), dP in r[KC, 2 KC)
         if constexpr (KC == 32) tmem_ld32x2(tS + q * KC, tdP + q * KC, r);
         else tmem_ld16x2(tS + q * KC, tdP + q * KC, r);
+        if (q == 64 / KC - 1) loaded();
         const uint32_t mw = ((q * KC) < 32 ? mw0 : mw1) >> ((q * KC) & 31);
 #pragma unroll
         for (int c2 = 0; c2 < KC / 8; ++c2) {
@@ -563,9 +566,11 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                           [&](int c, float2 p, float2 ds) {
                               pp[c >> 1] = pack_bf16x2(p.x, p.y);
                               dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
+                          },
+                          [&]() {   // S/dP read out: the next step's S/dP MMAs may start
+                              tc_fence_before();
+                              mbar_arrive(b_sd_free);
                           });
-                tc_fence_before();
-                mbar_arrive(b_sd_free);
                 mbar_arrive(b_bias_empty(bs));
                 mbar_arrive(b_q_empty(st));
                 if (t > 0) {
@@ -942,7 +947,10 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
             p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
                       bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
-                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); });
+                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); },
+                      []() {});
+            // (handing the TMEM buffer back after the last load instead, before the last
+            // chunk is computed, measured slower here)
             tc_fence_before();
             mbar_arrive(b_sd_free(x));
             mbar_arrive(b_empty(st));
