@@ -431,11 +431,10 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // S/dP of step t: its item's K/V, its Q/dOa, and S/dP of step t - 1 read out
             auto issue_sdp = [&](int t, int m, int ii) -> bool {
                 const int st = t % QS, x = m % KVB;
-                bool okk = true;
-                if (ii == 0)
-                    okk = mbar_wait(b_kv_full(x), (m / KVB) & 1, abort_flag, SITE_BWD_MMA | 0x80 | (t << 12));
-                if (okk) okk = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_MMA | 0x90 | (t << 12));
-                if (okk && t > 0) okk = mbar_wait(b_sd_free, (t - 1) & 1, abort_flag, SITE_BWD_MMA | 0xA0 | (t << 12));
+                const bool okk = mbar_wait_all(abort_flag,
+                                               b_kv_full(x), (m / KVB) & 1, ii == 0, SITE_BWD_MMA | 0x80 | (t << 12),
+                                               b_q_full(st), (t / QS) & 1, true, SITE_BWD_MMA | 0x90 | (t << 12),
+                                               b_sd_free, (t - 1) & 1, t > 0, SITE_BWD_MMA | 0xA0 | (t << 12));
                 if (!okk) return false;
                 tc_fence_after();
                 const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
@@ -453,9 +452,9 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // dQ of step t (item m, its step i of ni): P/dS written, the dQ buffer free
             auto issue_dq = [&](int t, int m, int i, int ni) -> bool {
                 const int x = m % KVB;
-                bool okk = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
-                if (okk && t >= 2)
-                    okk = mbar_wait(b_dq_free(t & 1), ((t >> 1) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x70 | (t << 12));
+                const bool okk = mbar_wait_all(abort_flag,
+                                               b_ps_full, t & 1, true, SITE_BWD_MMA | 0x20 | (t << 12),
+                                               b_dq_free(t & 1), ((t >> 1) - 1) & 1, t >= 2, SITE_BWD_MMA | 0x70 | (t << 12));
                 if (!okk) return false;
                 tc_fence_after();
                 const uint64_t dA = sdesc(sDS, 16, 1024, kSw128);
@@ -503,13 +502,12 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const int ni = item(m).ni;
                 for (int i = 0; i < ni && ok; ++i, ++t) {   // i: the item's step (query tile ilo + i)
                     const int st = t % QS, d = m % DKB;
-                    ok = mbar_wait(b_ps_full, t & 1, abort_flag, SITE_BWD_MMA | 0x20 | (t << 12));
+                    // P/dS of the step, and at an item's first step its dK/dV buffer (read out by
+                    // the epilogue of item m - DKB)
+                    ok = mbar_wait_all(abort_flag,
+                                       b_ps_full, t & 1, true, SITE_BWD_MMA | 0x20 | (t << 12),
+                                       b_dkv_free(d), ((m / DKB) - 1) & 1, i == 0 && m >= DKB, SITE_BWD_MMA | 0x60 | (t << 12));
                     if (!ok) break;
-                    if (i == 0 && m >= DKB) {
-                        // this item's dK/dV buffer: the epilogue of item m - DKB has read it
-                        ok = mbar_wait(b_dkv_free(d), ((m / DKB) - 1) & 1, abort_flag, SITE_BWD_MMA | 0x60 | (t << 12));
-                        if (!ok) break;
-                    }
                     tc_fence_after();
                     const uint32_t sQ = sbase + T::OFF_Q + st * 2 * T::TILE_BYTES;
                     const uint64_t dA = sdesc(sA, 16384, 1024, kSw128);
@@ -542,21 +540,21 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int ni = item(m).ni;
             for (int i = 0; i < ni && ok; ++i, ++t) {
                 const int st = t % QS, bs = t % BS;
+                // the item's K/V tiles (with its mask words) at its first step, the step's S/dP,
+                // Q stage (row statistics) and bias tile: probed together
+                ok = mbar_wait_all(abort_flag,
+                                   b_kv_full(m % KVB), (m / KVB) & 1, i == 0, SITE_BWD_EW | 0x30 | (t << 12),
+                                   b_sd_full, t & 1, true, SITE_BWD_EW | (t << 12),
+                                   b_q_full(st), (t / QS) & 1, true, SITE_BWD_EW | 0x40 | (t << 12),
+                                   b_bias_full(bs), (t / BS) & 1, true, SITE_BWD_EW | 0x50 | (t << 12));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
                 if (i == 0) {
-                    // this item's mask words come with its K/V tiles
-                    ok = mbar_wait(b_kv_full(m % KVB), (m / KVB) & 1, abort_flag, SITE_BWD_EW | 0x30 | (t << 12));
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
                     const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + (m % KVB) * 8;
                     mw0 = mw[2 * e];
                     mw1 = mw[2 * e + 1];
                     full = mw[4 + e] != 0;
                 }
-                ok = mbar_wait(b_sd_full, t & 1, abort_flag, SITE_BWD_EW | (t << 12));
-                if (ok) ok = mbar_wait(b_q_full(st), (t / QS) & 1, abort_flag, SITE_BWD_EW | 0x40 | (t << 12));
-                if (ok) ok = mbar_wait(b_bias_full(bs), (t / BS) & 1, abort_flag, SITE_BWD_EW | 0x50 | (t << 12));
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
                 tc_fence_after();
                 const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
                 uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
@@ -905,8 +903,8 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             bool ok = true;
             for (int n = 0; n < nb && ok; ++n) {
                 const int st = n % NS, x = n & 1;
-                ok = mbar_wait(b_full(st), (n / NS) & 1, abort_flag, SITE_DB_MMA);
-                if (ok && n >= 2) ok = mbar_wait(b_sd_free(x), ((n >> 1) - 1) & 1, abort_flag, SITE_DB_MMA);
+                ok = mbar_wait_all(abort_flag, b_full(st), (n / NS) & 1, true, SITE_DB_MMA,
+                                   b_sd_free(x), ((n >> 1) - 1) & 1, n >= 2, SITE_DB_MMA);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t s0 = sbase + T::OFF_STAGE + st * T::STAGE_BYTES;
@@ -937,8 +935,8 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t bias_row = sbase + T::OFF_BIAS + e * 16384 + row * 128;
         for (int n = 0; n < nb && ok; ++n) {
             const int st = n % NS, x = n & 1;
-            ok = mbar_wait(b_sd_full(x), (n >> 1) & 1, abort_flag, SITE_DB_EW);
-            if (ok) ok = mbar_wait(b_full(st), (n / NS) & 1, abort_flag, SITE_DB_EW);
+            ok = mbar_wait_all(abort_flag, b_sd_full(x), (n >> 1) & 1, true, SITE_DB_EW,
+                               b_full(st), (n / NS) & 1, true, SITE_DB_EW);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();

@@ -110,6 +110,31 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Wait for up to four barrier phases (slot k is skipped when need_k is false).  A probe of
+// a phase takes ~150 cycles on B200 even when the phase is already complete (measured), and
+// probes that do not depend on each other overlap; so every needed phase is probed first, all
+// together, and only the phases still open are then waited for one by one (bounded, as in
+// mbar_wait).  When everything is complete, which is the usual case for the element-wise
+// warps, the call costs one probe latency instead of one per barrier.
+__device__ __forceinline__ bool mbar_wait_all(volatile int *abort_flag,
+                                              uint32_t b0, uint32_t p0, bool n0, unsigned s0,
+                                              uint32_t b1, uint32_t p1, bool n1, unsigned s1,
+                                              uint32_t b2 = 0, uint32_t p2 = 0, bool n2 = false, unsigned s2 = 0,
+                                              uint32_t b3 = 0, uint32_t p3 = 0, bool n3 = false, unsigned s3 = 0) {
+    bool r0 = true, r1 = true, r2 = true, r3 = true;
+    if (n0) r0 = mbar_test(b0, p0);
+    if (n1) r1 = mbar_test(b1, p1);
+    if (n2) r2 = mbar_test(b2, p2);
+    if (n3) r3 = mbar_test(b3, p3);
+    if (r0 && r1 && r2 && r3) return true;
+    bool ok = true;
+    if (!r0) ok = mbar_wait(b0, p0, abort_flag, s0);
+    if (ok && !r1) ok = mbar_wait(b1, p1, abort_flag, s1);
+    if (ok && !r2) ok = mbar_wait(b2, p2, abort_flag, s2);
+    if (ok && !r3) ok = mbar_wait(b3, p3, abort_flag, s3);
+    return ok;
+}
+
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
     const long long t0 = sm_cycles();

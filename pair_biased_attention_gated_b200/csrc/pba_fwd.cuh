@@ -336,8 +336,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 // step k: S must have been read out by the softmax of step k - 1
                 for (int kl = 0; kl < Kn && ok; ++kl) {
                     const int k = kg + kl, s = kl % nb, st = k % KVS;
-                    if (k > 0) ok = mbar_wait(b_s_free, (k - 1) & 1, abort_flag, SITE_FWD_MMA | 0x20 | (k << 12));
-                    if (ok) ok = mbar_wait(b_k_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x10 | (k << 12));
+                    ok = mbar_wait_all(abort_flag, b_s_free, (k - 1) & 1, k > 0, SITE_FWD_MMA | 0x20 | (k << 12),
+                                       b_k_full(st), (k / KVS) & 1, true, SITE_FWD_MMA | 0x10 | (k << 12));
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t dq = sdesc(sbase + T::OFF_Q + s * T::TILE_BYTES, 16, SBO, T::SWZ);
@@ -366,8 +366,8 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 // step k: P of step k written (and O[s] rescaled) by the softmax, V landed
                 for (int kl = 0; kl < Kn && ok; ++kl) {
                     const int k = kg + kl, j = kl / nb, s = kl % nb, st = k % KVS;
-                    ok = mbar_wait(b_p_full, k & 1, abort_flag, SITE_FWD_MMA | 0x30 | (k << 12));
-                    if (ok) ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag, SITE_FWD_MMA | 0x40 | (k << 12));
+                    ok = mbar_wait_all(abort_flag, b_p_full, k & 1, true, SITE_FWD_MMA | 0x30 | (k << 12),
+                                       b_v_full(st), (k / KVS) & 1, true, SITE_FWD_MMA | 0x40 | (k << 12));
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t dv = sdesc(sbase + T::OFF_V + st * T::TILE_BYTES, T::TILE_BYTES, SBO, T::SWZ);
@@ -478,13 +478,12 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const int bs = jg % BS;
                 for (int s = 0; s < nb; ++s, ++k) {
                     const int st = k % KVS;
-                    ok = mbar_wait(b_s_full, k & 1, abort_flag, SITE_FWD_SOFTMAX | (k << 12));
-                    if (ok && s == 0)
-                        ok = mbar_wait(b_bias_ready(bs), (jg / BS) & 1, abort_flag,
-                                       SITE_FWD_SOFTMAX | 0x10 | (k << 12));
-                    if (ok && row_mask)   // this step's mask words come with its V tile
-                        ok = mbar_wait(b_v_full(st), (k / KVS) & 1, abort_flag,
-                                       SITE_FWD_SOFTMAX | 0x20 | (k << 12));
+                    // S of the step, the folded bias tile at a tile's first row, and with
+                    // per-row masks the step's V stage (its mask words come with it): probed
+                    // together
+                    ok = mbar_wait_all(abort_flag, b_s_full, k & 1, true, SITE_FWD_SOFTMAX | (k << 12),
+                                       b_bias_ready(bs), (jg / BS) & 1, s == 0, SITE_FWD_SOFTMAX | 0x10 | (k << 12),
+                                       b_v_full(st), (k / KVS) & 1, row_mask, SITE_FWD_SOFTMAX | 0x20 | (k << 12));
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
