@@ -558,6 +558,7 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 tc_fence_after();
                 const float2 rs = reinterpret_cast<const float2 *>(gbase + T::OFF_RS + st * 1024)[row];
                 uint32_t pp[32], dsp[32];   // P and dS as bf16 pairs, keys 2 c and 2 c + 1
+                bool prod_done = t == 0;    // the previous step's products, probed below
                 const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
                 p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
                           row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
@@ -568,10 +569,14 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                           [&]() {   // S/dP read out: the next step's S/dP MMAs may start
                               tc_fence_before();
                               mbar_arrive(b_sd_free);
+                              // probe the previous step's products now, so that the probe's
+                              // latency overlaps the last chunk (a complete phase stays
+                              // complete: the next one needs this step's P/dS)
+                              if (t > 0) prod_done = mbar_test(b_ps_free, (t - 1) & 1);
                           });
                 mbar_arrive(b_bias_empty(bs));
                 mbar_arrive(b_q_empty(st));
-                if (t > 0) {
+                if (!__all_sync(0xffffffffu, prod_done)) {
                     ok = mbar_wait(b_ps_free, (t - 1) & 1, abort_flag, SITE_BWD_EW | 0x60 | (t << 12));
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;

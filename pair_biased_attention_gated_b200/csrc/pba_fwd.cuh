@@ -559,6 +559,10 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     // The exponentials go into registers first: only the store of P (and a
                     // rescale of O[s]) has to wait for the previous P V, so the exponential
                     // unit's share of the step overlaps that product instead of following it.
+                    // P and O[s] may only be written once the previous P V is done: probe that
+                    // now, so the probe's latency overlaps the exponentials (a phase found
+                    // complete stays complete: the next one needs this step's P)
+                    const bool pv_done = k == 0 || mbar_test(b_p_free, (k - 1) & 1);
                     float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
                     uint32_t p0[32], p1[32];   // P of keys 0..63 and 64..127 as bf16 pairs
 #pragma unroll
@@ -571,13 +575,12 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         else p1[c - 32] = pack_bf16x2(pv.x, pv.y);
                     }
                     const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-                    // P and O[s] may only be written once the previous P V is done
-                    if (k > 0) {
+                    if (!__all_sync(0xffffffffu, pv_done)) {
                         ok = mbar_wait(b_p_free, (k - 1) & 1, abort_flag, SITE_FWD_SOFTMAX | 0x30 | (k << 12));
                         ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
-                        tc_fence_after();
                     }
+                    tc_fence_after();
                     tmem_st32(tP, p0);
                     tmem_st32(tP + 32, p1);
                     if (__any_sync(0xffffffffu, resc)) {
