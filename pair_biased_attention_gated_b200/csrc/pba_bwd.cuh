@@ -181,6 +181,14 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
 #pragma unroll
     for (int q = 0; q < 64 / KC; ++q) {
+        // the chunk's bias words first: their shared-memory loads are then in flight while
+        // the TMEM load below waits
+        uint4 bws[KC / 8];
+#pragma unroll
+        for (int c2 = 0; c2 < KC / 8; ++c2) {
+            bws[c2] = make_uint4(0, 0, 0, 0);
+            if (has_bias) bws[c2] = lds128(bias_row + (((q * (KC / 8) + c2) ^ (row & 7)) << 4));
+        }
         uint32_t r[2 * KC];   // S of keys KC q .. KC q + KC - 1 in r[0, KC), dP in r[KC, 2 KC)
         if constexpr (KC == 32) tmem_ld32x2(tS + q * KC, tdP + q * KC, r);
         else tmem_ld16x2(tS + q * KC, tdP + q * KC, r);
@@ -188,9 +196,7 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
         const uint32_t mw = ((q * KC) < 32 ? mw0 : mw1) >> ((q * KC) & 31);
 #pragma unroll
         for (int c2 = 0; c2 < KC / 8; ++c2) {
-            const int c8 = q * (KC / 8) + c2;
-            uint4 bw = make_uint4(0, 0, 0, 0);
-            if (has_bias) bw = lds128(bias_row + ((c8 ^ (row & 7)) << 4));
+            const uint4 bw = bws[c2];
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {

@@ -488,6 +488,13 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     if (!ok) break;
                     tc_fence_after();
 
+                    // the first half of this row's bias words: their shared-memory loads are in
+                    // flight while the TMEM load of S below waits
+                    const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + row * 128;
+                    uint4 bw0[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) bw0[q] = lds128(bias_row + (((q & 7) ^ (row & 7)) << 4));
+
                     // S of this row, then hand the S columns back for the next Q K^T
                     uint32_t xr[128];
                     tmem_ld128(tS, xr);
@@ -496,10 +503,10 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
                     // logits in place: x = scale * S + bias (natural-log units; -inf if masked)
                     {
-                        const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + row * 128;
 #pragma unroll
                         for (int q = 0; q < 16; ++q) {  // 16-byte chunk q holds keys 8q .. 8q+7
-                            const uint4 bw = lds128(bias_row + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4));
+                            const uint4 bw = q < 8 ? bw0[q & 7]
+                                                   : lds128(bias_row + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4));
                             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
