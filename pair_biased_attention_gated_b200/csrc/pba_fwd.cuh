@@ -500,13 +500,16 @@ pba_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     tmem_ld128(tS, xr);
                     tc_fence_before();
                     mbar_arrive(b_s_free);
+                    // the second half's bias words, all issued before any of them is used
+                    uint4 bw1[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) bw1[q] = lds128(bias_row + 16384 + ((q ^ (row & 7)) << 4));
 
                     // logits in place: x = scale * S + bias (natural-log units; -inf if masked)
                     {
 #pragma unroll
                         for (int q = 0; q < 16; ++q) {  // 16-byte chunk q holds keys 8q .. 8q+7
-                            const uint4 bw = q < 8 ? bw0[q & 7]
-                                                   : lds128(bias_row + (q >> 3) * 16384 + (((q & 7) ^ (row & 7)) << 4));
+                            const uint4 bw = q < 8 ? bw0[q & 7] : bw1[q & 7];
                             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
