@@ -167,7 +167,8 @@ __device__ __forceinline__ void mask_words(const BwdArgs &a, int b, int j0, uint
 //   in a 128-byte swizzled shared-memory row; mw0, mw1: mask words of those 64 keys (all
 //   ones when `full`); sl2e = scale log2 e; lse2 = lse log2 e; D = sum_c dout out.
 //   P = exp2(S sl2e + bias log2 e - lse2) (0 for masked keys), dS = P (dP - D).
-// For each pair of keys (c, c + 1), c even, `use(c, p, ds)` receives the two P and dS;
+// For each pair of keys (c, c + 1), c even, `use(c, p, dpd)` receives the two P and dP - D
+// (dS = P (dP - D) is formed by the caller: a product, or a fused multiply-add into a sum);
 // `loaded()` is called once the last chunk's S and dP are in registers (the TMEM columns
 // may then be handed back before the chunk is computed).
 template <int KC, typename Use, typename Loaded>
@@ -208,8 +209,8 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
                     p.x = ((mw >> k) & 1u) ? p.x : 0.f;
                     p.y = ((mw >> (k + 1)) & 1u) ? p.y : 0.f;
                 }
-                const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(r[KC + k]), __uint_as_float(r[KC + 1 + k])), nD2));
-                use(q * KC + k, p, ds);
+                const float2 dpd = fadd2(make_float2(__uint_as_float(r[KC + k]), __uint_as_float(r[KC + 1 + k])), nD2);
+                use(q * KC + k, p, dpd);
             }
         }
     }
@@ -568,7 +569,8 @@ pba_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const uint32_t bias_row = sbase + T::OFF_BIAS + bs * T::BIAS_BYTES + e * 16384 + row * 128;
                 p_ds_half<16>(tbase + T::T_S + e * 64 + lane_off, tbase + T::T_DP + e * 64 + lane_off, bias_row,
                           row, a.has_bias != 0, mw0, mw1, full, sl2e, rs.x, rs.y,
-                          [&](int c, float2 p, float2 ds) {
+                          [&](int c, float2 p, float2 dpd) {
+                              const float2 ds = fmul2(p, dpd);
                               pp[c >> 1] = pack_bf16x2(p.x, p.y);
                               dsp[c >> 1] = pack_bf16x2(ds.x, ds.y);
                           },
@@ -956,7 +958,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
             p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
                       bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
-                      rs.x, rs.y, [&](int c, float2, float2 ds) { acc[c >> 1] = fadd2(acc[c >> 1], ds); },
+                      rs.x, rs.y, [&](int c, float2 p, float2 dpd) { acc[c >> 1] = ffma2(p, dpd, acc[c >> 1]); },
                       []() {});
             // (handing the TMEM buffer back after the last load instead, before the last
             // chunk is computed, measured slower here)
