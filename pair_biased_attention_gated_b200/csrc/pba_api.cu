@@ -416,6 +416,28 @@ pba_status launch_zero_rows(pba_bf16 *dk, pba_bf16 *dv, const pba_dims *d, cudaS
     return e == cudaSuccess ? PBA_OK : cuda_fail(e, "zero_rows_kernel launch");
 }
 
+// ---------------------------------------------------------------------------- side stream
+// The dbias kernel needs only the pre kernel's row statistics and the dq conversion only the
+// dq/dk/dv kernel, and the two share an SM well (the dbias kernel is bound by the exponential
+// unit and instruction issue, the conversion by DRAM).  So once the dq/dk/dv kernel is done the
+// dbias kernel runs on a second stream of higher priority (its CTAs are placed first) while
+// the conversion runs on the caller's stream, which then waits for the second stream.  The
+// stream and its two events are created once per CUDA context (keyed by the context's unique
+// id, outside any stream capture) and shared by every call in that context under g_side_mu,
+// which also keeps each call's event record and the wait on it together.  Inside a capture the
+// fork and the join become graph dependencies.
+struct SideStream {
+    unsigned long long ctx;
+    cudaStream_t s;
+    cudaEvent_t fork, join;
+};
+std::mutex g_side_mu;
+std::vector<SideStream> g_side;
+// The side stream of the current context (created on first use; never while `s` is being
+// captured); false if it does not exist and cannot be made, and the caller then stays on `s`.
+// The caller holds g_side_mu.
+bool side_stream(cudaStream_t s, SideStream *out);
+
 template <int CP>
 pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                       const pba_bf16 *bias, const uint8_t *mask, const pba_bf16 *gate,
@@ -501,19 +523,38 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_bwd_main_kernel launch");
         if (dbias) {
             if ((st = set_smem(pba::pba_dbias_kernel<CP>, DT::SMEM_BYTES)) != PBA_OK) return st;
+            std::lock_guard<std::mutex> g(g_side_mu);
+            SideStream side;
+            const bool fork = side_stream(s, &side);
+            cudaStream_t ds = s;   // the dbias kernels' stream
+            if (fork) {
+                if ((e = cudaEventRecord(side.fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+                if ((e = cudaStreamWaitEvent(side.s, side.fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+                ds = side.s;
+            }
             const long long g2 = (long long)pl.splits * d->H * pl.ntiles;
             if (win >= 0) {
-                ProfScope ps(K_DBIAS_ZERO, s);
+                ProfScope ps(K_DBIAS_ZERO, ds);
                 const long long rows = (long long)d->H * d->Nq;
-                pba::pba_dbias_zero_kernel<<<(unsigned)std::min<long long>(rows, 8 * kSmCount), 256, 0, s>>>(a);
+                pba::pba_dbias_zero_kernel<<<(unsigned)std::min<long long>(rows, 8 * kSmCount), 256, 0, ds>>>(a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_zero_kernel launch");
             {
-                ProfScope ps(K_DBIAS, s);
-                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, s>>>(tq, tk, tv, tdo, tb, a);
+                ProfScope ps(K_DBIAS, ds);
+                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, ds>>>(tq, tk, tv, tdo, tb, a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
             // (the last CTA of every tile sums the split partials in split order)
+            {
+                ProfScope ps(K_DQ_CONVERT, s);
+                pba::pba_dq_convert_kernel<<<grid_for((long long)elems / 8, 256), 256, 0, s>>>(a);
+            }
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dq_convert_kernel launch");
+            if (fork) {
+                if ((e = cudaEventRecord(side.join, side.s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+                if ((e = cudaStreamWaitEvent(s, side.join, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+            }
+            return PBA_OK;
         }
     }
     {
@@ -586,6 +627,38 @@ pba_status noalloc_scratch(void **out) {
     return PBA_OK;
 }
 
+
+bool side_stream(cudaStream_t s, SideStream *out) {
+    unsigned long long id = 0;
+    {
+        // a failure here only means no side stream: keep the caller's last error untouched
+        const std::string keep = g_last_error;
+        const pba_status st = current_context_id(&id);
+        g_last_error = keep;
+        if (st != PBA_OK) return false;
+    }
+    for (const auto &ent : g_side)
+        if (ent.ctx == id) {
+            *out = ent;
+            return true;
+        }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return false;
+    SideStream ent{id, nullptr, nullptr, nullptr};
+    if (cudaStreamCreateWithPriority(&ent.s, cudaStreamNonBlocking, hi) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&ent.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ent.join, cudaEventDisableTiming) != cudaSuccess) {
+        if (ent.fork) cudaEventDestroy(ent.fork);
+        cudaStreamDestroy(ent.s);
+        cudaGetLastError();
+        return false;
+    }
+    g_side.push_back(ent);
+    *out = ent;
+    return true;
+}
 
 // ---------------------------------------------------------------------------- pair-weighted
 // The [H, N, Wld] bf16 weights as a 3-D map (N, N, H), box (64, 128, 1), 128-byte swizzle:
