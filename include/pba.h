@@ -102,6 +102,12 @@ size_t pba_bwd_workspace_size(const pba_dims *dims);
  * logits' gradient, reduced in a fixed order, so it is bit-identical from run to run.
  * workspace: caller-owned device memory of at least pba_bwd_workspace_size(dims) bytes,
  * 256-byte aligned; its contents on entry do not matter and on return are undefined.
+ * With dbias, the dbias kernel runs on a second stream of the library's beside the dq
+ * conversion; `stream` waits for it before the call's work ends, so everything stays
+ * ordered on `stream` (in a stream capture both become part of the graph).  That stream and
+ * its two events are created by the first such call in a CUDA context and kept for the
+ * context's lifetime; if that first call is made while `stream` is being captured, the call
+ * runs on `stream` alone (same results), so make one call before capturing to get the overlap.
  */
 pba_status pba_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
                    const pba_bf16 *bias, const uint8_t *key_mask, const pba_bf16 *gate,
