@@ -541,7 +541,7 @@ pba_status launch_bwd(const pba_bf16 *q, const pba_bf16 *k, const pba_bf16 *v,
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_zero_kernel launch");
             {
                 ProfScope ps(K_DBIAS, ds);
-                pba::pba_dbias_kernel<CP><<<(unsigned)g2, 320, DT::SMEM_BYTES, ds>>>(tq, tk, tv, tdo, tb, a);
+                pba::pba_dbias_kernel<CP><<<(unsigned)g2, DT::THREADS, DT::SMEM_BYTES, ds>>>(tq, tk, tv, tdo, tb, a);
             }
             if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_dbias_kernel launch");
             // (the last CTA of every tile sums the split partials in split order)

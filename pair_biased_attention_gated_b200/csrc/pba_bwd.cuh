@@ -25,6 +25,8 @@
 // main kernel's items step over those, the dbias kernel covers only those tile pairs.
 #pragma once
 
+#include <type_traits>
+
 #include "pba_device.cuh"
 
 namespace pba {
@@ -211,6 +213,66 @@ __device__ __forceinline__ void p_ds_half(uint32_t tS, uint32_t tdP, uint32_t bi
                 }
                 const float2 dpd = fadd2(make_float2(__uint_as_float(r[KC + k]), __uint_as_float(r[KC + 1 + k])), nD2);
                 use(q * KC + k, p, dpd);
+            }
+        }
+    }
+}
+
+// The bits of mask word w (keys 32 w .. 32 w + 31) that fall in the keys k0 .. k0 + nk - 1.
+__host__ __device__ constexpr uint32_t key_bits(int k0, int nk, int w) {
+    const int lo = (k0 > 32 * w ? k0 : 32 * w) - 32 * w;
+    const int hi = (k0 + nk < 32 * w + 32 ? k0 + nk : 32 * w + 32) - 32 * w;
+    return hi <= lo ? 0u : (hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u) << lo);
+}
+static_assert(key_bits(48, 48, 1) == 0xffff0000u && key_bits(48, 48, 2) == 0xffffffffu &&
+              key_bits(0, 48, 1) == 0x0000ffffu && key_bits(96, 32, 3) == 0xffffffffu &&
+              key_bits(96, 32, 2) == 0u, "key_bits");
+
+// P and dS of the NK keys K0 .. K0 + NK - 1 of a 128-key tile for one query row, in 16-key
+// chunks (as p_ds_half, for a key range that need not be a half):
+//   tS, tdP: this lane's S and dP column 0 in TMEM; bias_row: the row in the first 64-key
+//   half of the bias tile (128-byte swizzled rows, the second half 16 KB further); mw: the
+//   four mask words of the tile's keys (all ones when `full`).
+// `use(c, p, dpd)` receives keys K0 + c and K0 + c + 1 (c even); `loaded()` is called once the
+// last chunk's S and dP are in registers.
+template <int K0, int NK, typename Use, typename Loaded>
+__device__ __forceinline__ void p_ds_keys(uint32_t tS, uint32_t tdP, uint32_t bias_row, int row,
+                                          bool has_bias, const uint32_t *mw, bool full, float sl2e,
+                                          float lse2, float D, Use &&use, Loaded &&loaded) {
+    static_assert(K0 % 16 == 0 && NK % 16 == 0 && K0 + NK <= 128, "key range");
+    const float2 sl2 = make_float2(sl2e, sl2e), l2e2 = make_float2(kLog2eB, kLog2eB);
+    const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-D, -D);
+#pragma unroll
+    for (int q = 0; q < NK / 16; ++q) {
+        const int kc = K0 + 16 * q;   // first key of the chunk
+        uint4 bws[2];
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+            const int k8 = kc + 8 * c2;
+            bws[c2] = make_uint4(0, 0, 0, 0);
+            if (has_bias)
+                bws[c2] = lds128(bias_row + (k8 >> 6) * 16384 + ((((k8 & 63) >> 3) ^ (row & 7)) << 4));
+        }
+        uint32_t r[32];   // S of the chunk's keys in r[0, 16), dP in r[16, 32)
+        tmem_ld16x2(tS + kc, tdP + kc, r);
+        if (q == NK / 16 - 1) loaded();
+        const uint32_t m = full ? 0xffffffffu : (mw[kc >> 5] >> (kc & 31));
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+            const uint4 bw = bws[c2];
+            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = c2 * 8 + 2 * e;   // key within the chunk
+                float2 u = ffma2(make_float2(bf16lo(bb[e]), bf16hi(bb[e])), l2e2, nl2);
+                u = ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, u);
+                float2 p = make_float2(ex2(u.x), ex2(u.y));
+                if (!full) {
+                    p.x = ((m >> k) & 1u) ? p.x : 0.f;
+                    p.y = ((m >> (k + 1)) & 1u) ? p.y : 0.f;
+                }
+                const float2 dpd = fadd2(make_float2(__uint_as_float(r[16 + k]), __uint_as_float(r[17 + k])), nD2);
+                use(kc - K0 + k, p, dpd);
             }
         }
     }
@@ -796,7 +858,14 @@ __global__ void __launch_bounds__(256) pba_dbias_zero_kernel(const BwdArgs a) {
 // ---------------------------------------------------------------------------------------
 template <int CP>
 struct DbTraits {
-    static constexpr int NS = (CP == 64) ? 2 : 3;                 // stages (one row b each)
+    // element-wise warpgroups: keys 0-47, 48-95 and 96-127 (three warps per SM
+    // sub-partition, for latency hiding), then the producer and the MMA issuer warps
+    static constexpr int NWG = 3;
+    static constexpr int THREADS = 32 * (4 * NWG + 2);
+    static constexpr int W_PROD = 4 * NWG, W_MMA = 4 * NWG + 1;
+    // stages (one row b each): as many as fit beside the bias tile, so that the TMA loads of
+    // several rows are in flight
+    static constexpr int NS = (CP == 64) ? 2 : (CP == 32 ? 5 : 8);
     static constexpr int TILE_BYTES = 128 * CP * 2;
     static constexpr int STAGE_BYTES = 4 * TILE_BYTES + 1024;     // Q, dOa, K, V, row stats
     static constexpr int OFF_BIAS = 0;
@@ -807,8 +876,13 @@ struct DbTraits {
     static constexpr uint32_t ROWB = CP * 2;
 };
 
+// one CTA per SM: the dynamic shared memory (with its alignment slack) within the 227 KB a
+// CTA may have
+static_assert(DbTraits<16>::SMEM_BYTES <= 232448 && DbTraits<32>::SMEM_BYTES <= 232448 &&
+              DbTraits<64>::SMEM_BYTES <= 232448, "dbias shared memory");
+
 template <int CP>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DbTraits<CP>::THREADS, 1)
 pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmBias, const BwdArgs a) {
@@ -847,16 +921,16 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_init(b_drain, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(b_sd_full(x), 1);
-            mbar_init(b_sd_free(x), 256);
+            mbar_init(b_sd_free(x), 128 * T::NWG);
         }
         for (int x = 0; x < NS; ++x) {
             mbar_init(b_full(x), 1);
-            mbar_init(b_empty(x), 1 + 256);
+            mbar_init(b_empty(x), 1 + 128 * T::NWG);
         }
         s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == T::W_MMA) {
         tmem_alloc(smem_u32(&s_tmem_base), 512);
         tmem_relinquish();
     }
@@ -867,7 +941,7 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     volatile int *abort_flag = &s_abort;
     int n_done = 0;   // rows b whose stage loads were issued: [0, n_done)
 
-    if (warp == 8) {
+    if (warp == T::W_PROD) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -885,13 +959,15 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         bool ok = true;
         int n = 0;
+        // a row's mask words are read before its stage is free, so that their global loads
+        // overlap the wait
+        uint32_t w[4];
+        if (nb > 0) mask_words(a, bstart, j0, w);
         for (; n < nb; ++n) {
             const int st = n % NS, b = bstart + n;
             if (n >= NS) ok = mbar_wait(b_empty(st), ((n / NS) - 1) & 1, abort_flag, SITE_DB_PROD);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            uint32_t w[4];
-            mask_words(a, b, j0, w);
             if (lane == 0) {
                 uint32_t *mw = reinterpret_cast<uint32_t *>(gbase + T::OFF_MASK) + st * 8;
                 mw[0] = w[0]; mw[1] = w[1]; mw[2] = w[2]; mw[3] = w[3];
@@ -907,8 +983,9 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                           1024, b_full(st));
             }
             n_done = n + 1;
+            if (n + 1 < nb) mask_words(a, b + 1, j0, w);
         }
-    } else if (warp == 9) {
+    } else if (warp == T::W_MMA) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t SBO = 8 * T::ROWB;
@@ -936,62 +1013,74 @@ pba_dbias_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------------ elementwise
-        const int e = warp >> 2;
+        // warpgroup g: keys 48 g .. 48 g + 47 (g < 2) or 96 .. 127 (g = 2) of its 32 rows
+        const int g = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
         const float sl2e = a.scale * kLog2eB;
-        float2 acc[32];   // sum over this split's rows b of dS, keys 2 c and 2 c + 1
-#pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
+        const uint32_t bias_row = sbase + T::OFF_BIAS + row * 128;
         bool ok = mbar_wait(b_bias, 0, abort_flag, SITE_DB_EW);
         ok = __all_sync(0xffffffffu, ok);
-        const uint32_t bias_row = sbase + T::OFF_BIAS + e * 16384 + row * 128;
-        for (int n = 0; n < nb && ok; ++n) {
-            const int st = n % NS, x = n & 1;
-            ok = mbar_wait_all(abort_flag, b_sd_full(x), (n >> 1) & 1, true, SITE_DB_EW,
-                               b_full(st), (n / NS) & 1, true, SITE_DB_EW);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
-            const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
-            const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
-            p_ds_half<32>(tbase + x * 256 + e * 64 + lane_off, tbase + x * 256 + 128 + e * 64 + lane_off,
-                      bias_row, row, a.has_bias != 0, mw[2 * e], mw[2 * e + 1], mw[4 + e] != 0, sl2e,
-                      rs.x, rs.y, [&](int c, float2 p, float2 dpd) { acc[c >> 1] = ffma2(p, dpd, acc[c >> 1]); },
-                      []() {});
-            // (handing the TMEM buffer back after the last load instead, before the last
-            // chunk is computed, measured slower here)
-            tc_fence_before();
-            mbar_arrive(b_sd_free(x));
-            mbar_arrive(b_empty(st));
-        }
-        if (ok) {
-            // this split's partial tile: [split][h][tile][128][128]
-            float *dst = a.dbias_part +
-                         ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + e * 64;
+        auto run = [&](auto k0c, auto nkc) {
+            constexpr int K0 = decltype(k0c)::value, NK = decltype(nkc)::value;
+            float2 acc[NK / 2];   // sum over this split's rows b of dS, keys K0 + 2 c and K0 + 2 c + 1
 #pragma unroll
-            for (int c = 0; c < 32; c += 2)
-                *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
-            __threadfence();   // this thread's partial row, before the tile counter moves
-        }
+            for (int c = 0; c < NK / 2; ++c) acc[c] = make_float2(0.f, 0.f);
+            for (int n = 0; n < nb && ok; ++n) {
+                const int st = n % NS, x = n & 1;
+                ok = mbar_wait_all(abort_flag, b_sd_full(x), (n >> 1) & 1, true, SITE_DB_EW,
+                                   b_full(st), (n / NS) & 1, true, SITE_DB_EW);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const uint8_t *s0 = gbase + T::OFF_STAGE + st * T::STAGE_BYTES;
+                const float2 rs = reinterpret_cast<const float2 *>(s0 + 4 * T::TILE_BYTES)[row];
+                const uint32_t *mw = reinterpret_cast<const uint32_t *>(gbase + T::OFF_MASK) + st * 8;
+                // every key of the range attended
+                bool full = true;
+#pragma unroll
+                for (int w = K0 >> 5; w <= (K0 + NK - 1) >> 5; ++w) {
+                    const uint32_t bits = key_bits(K0, NK, w);
+                    full = full && (mw[w] & bits) == bits;
+                }
+                p_ds_keys<K0, NK>(tbase + x * 256 + lane_off, tbase + x * 256 + 128 + lane_off, bias_row, row,
+                                  a.has_bias != 0, mw, full, sl2e, rs.x, rs.y,
+                                  [&](int c, float2 p, float2 dpd) { acc[c >> 1] = ffma2(p, dpd, acc[c >> 1]); },
+                                  []() {});
+                tc_fence_before();
+                mbar_arrive(b_sd_free(x));
+                mbar_arrive(b_empty(st));
+            }
+            if (ok) {
+                // this split's partial tile: [split][h][tile][128][128]
+                float *dst = a.dbias_part +
+                             ((((long long)sp * a.H + h) * a.ntiles + bt) * 128 + row) * 128 + K0;
+#pragma unroll
+                for (int c = 0; c < NK / 2; c += 2)
+                    *reinterpret_cast<float4 *>(dst + 2 * c) = make_float4(acc[c].x, acc[c].y, acc[c + 1].x, acc[c + 1].y);
+                __threadfence();   // this thread's partial row, before the tile counter moves
+            }
+        };
+        if (g == 0) run(std::integral_constant<int, 0>(), std::integral_constant<int, 48>());
+        else if (g == 1) run(std::integral_constant<int, 48>(), std::integral_constant<int, 48>());
+        else run(std::integral_constant<int, 96>(), std::integral_constant<int, 32>());
     }
 
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) {
-        if (warp == 8 && lane == 0) {
+        if (warp == T::W_PROD && lane == 0) {
             mbar_wait_drain(b_bias, 0);
             for (int nn = max(0, n_done - NS); nn < n_done; ++nn) mbar_wait_drain(b_full(nn % NS), (nn / NS) & 1);
         }
-        if (warp == 9 && lane == 0) {
+        if (warp == T::W_MMA && lane == 0) {
             umma_commit(b_drain);
             mbar_wait_drain(b_drain, 0);
         }
         tc_fence_before();
         __syncthreads();
     }
-    if (warp == 9) {
+    if (warp == T::W_MMA) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tbase, 512);

@@ -500,10 +500,10 @@ class DbiasSim:
     """The dbias kernel (pba_bwd.cuh): one producer fills NS stages (Q, dOa, K and V tiles, row
     statistics and mask words of one broadcast row each) after the bias tile; one MMA issuer
     computes S and dP of row n into TMEM buffer n & 1 and releases the stage by a commit; nwg
-    element-wise warpgroups (128 / nwg keys each, 128 arrivals each) read the TMEM buffer,
+    element-wise warpgroups (a key range each, 128 arrivals each) read the TMEM buffer,
     the stage's row statistics and mask words, and release both."""
 
-    def __init__(self, nb, NS, seed, plant=None, nwg=2):
+    def __init__(self, nb, NS, seed, plant=None, nwg=3):
         self.rng = random.Random(seed)
         self.plant = plant
         self.nb, self.NS, self.nwg = nb, NS, nwg

@@ -52,7 +52,7 @@ def test_planted_backward_mistakes_are_caught():
 
 
 # dbias kernel stages: c=64 -> 2, otherwise 3
-@pytest.mark.parametrize("NS", [2, 3])
+@pytest.mark.parametrize("NS", [2, 3, 5, 8])
 def test_dbias_protocol(NS):
     for nb in (0, 1, 2, 3, 4, 7):
         for seed in range(40):
