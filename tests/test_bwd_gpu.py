@@ -86,6 +86,14 @@ CASES = {
     "multi_item_c24": (30, 4, 200, 200, 24, ((190, 200),), True, True),
     "multi_item_c16": (40, 4, 72, 72, 16, (), True, True),
     "multi_item_c64": (24, 4, 136, 136, 64, ((0, 3),), True, True),
+    # the dbias kernel's element-wise warpgroups own keys 0-47, 48-95 and 96-127 of a key
+    # tile and skip the mask test when their whole range is attended: masked keys on and
+    # around those edges, in both key tiles, and ranges left wholly attended beside them
+    "mask_on_dbias_group_edges": (6, 2, 256, 256, 32,
+                                  ((40, 50), (94, 97), (120, 121), (176, 180), (200, 208)), True, True),
+    "mask_single_edge_keys": (5, 2, 256, 256, 32, ((47, 49), (95, 97), (223, 225)), True, True),
+    "mask_on_dbias_group_edges_c16": (6, 2, 256, 256, 16, ((40, 50), (94, 97), (176, 180)), True, True),
+    "mask_on_dbias_group_edges_c64": (4, 2, 256, 256, 64, ((47, 49), (95, 97), (200, 208)), True, True),
 }
 
 
@@ -97,6 +105,11 @@ def test_bwd_matches_oracle(pba, name):
 
 def test_bwd_per_row_mask(pba):
     _check_full(pba, _inputs(6, 2, 136, 136, 32, ((130, 136),), per_row_mask=True))
+
+
+def test_bwd_per_row_mask_on_dbias_group_edges(pba):
+    # per-row masks (about 20 % of keys dropped per row b) on top of masked group edges
+    _check_full(pba, _inputs(6, 2, 256, 256, 32, ((46, 50), (94, 98)), per_row_mask=True, seed=3))
 
 
 def test_bwd_fully_masked_rows_give_zero(pba):
