@@ -117,8 +117,9 @@ __global__ void __launch_bounds__(256) pba_bwd_pre_kernel(const BwdArgs a) {
                     const float d0 = bf16lo(dw[e]), d1 = bf16hi(dw[e]);
                     D = fmaf(d0, o0, D);
                     D = fmaf(d1, o1, D);
-                    const float s0 = 1.f / (1.f + __expf(-bf16lo(gw[e])));
-                    const float s1 = 1.f / (1.f + __expf(-bf16hi(gw[e])));
+                    // the forward epilogue's sigmoid, so both passes use the same gate values
+                    const float s0 = sigmoid_fast(bf16lo(gw[e]));
+                    const float s1 = sigmoid_fast(bf16hi(gw[e]));
                     daw[e] = pack_bf16x2(d0 * s0, d1 * s1);
                     dgw[e] = pack_bf16x2(d0 * o0 * (1.f - s0), d1 * o1 * (1.f - s1));
                 }
