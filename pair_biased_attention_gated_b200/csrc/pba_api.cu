@@ -955,9 +955,13 @@ pba_status launch_pb(bool bwd, const CUtensorMap &tm, pba::PbArgs a, const pba_p
     pba_status st;
     cudaError_t e;
     if (!bwd) {
-        if ((st = set_smem(pba::pba_pair_bias_fwd_kernel<CZ, HP>, T::SMEM_BYTES)) != PBA_OK) return st;
+        // the forward has its own shared-memory layout (and so its own grid); nothing of the
+        // backward's reduction order depends on it
+        using F = pba::PbFwdTraits<CZ>;
+        const long long fgrid = pb_grid(d, F::SMEM_BYTES);
+        if ((st = set_smem(pba::pba_pair_bias_fwd_kernel<CZ, HP>, F::SMEM_BYTES)) != PBA_OK) return st;
         ProfScope ps(K_PB_FWD, s);
-        pba::pba_pair_bias_fwd_kernel<CZ, HP><<<(unsigned)grid, 128, T::SMEM_BYTES, s>>>(tm, a);
+        pba::pba_pair_bias_fwd_kernel<CZ, HP><<<(unsigned)fgrid, F::THREADS, F::SMEM_BYTES, s>>>(tm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_fwd_kernel launch");
         return PBA_OK;
     }

@@ -172,58 +172,218 @@ __device__ __forceinline__ void pb_row_stats(const float *sW, uint32_t buf, int 
     rstd = rsqrtf((var2.x + var2.y) * (1.f / CZ) + eps);
 }
 
+// Forward on the tensor core: per tile, acc[p,h] = sum_c z[p,c] w'[c,h] is one M = 128, N = 32
+// product per 16 channels, accumulated in TMEM: w' = gamma w as two bf16 terms for fp32
+// accuracy, hi in columns 0-15 and lo in columns 16-31 (heads padded with zeros to 16), added
+// in the epilogue, so the two terms cost no extra MMA instructions; the threads only make each row's
+// mean and 1 / sqrt(var + eps) and the epilogue bias_h = rstd (acc_h - mean S_h) + sum_c beta_c w[c,h].
+// Warp roles (160 threads): warps 0-3 thread = position (TMEM lane); warp 4 allocates TMEM and,
+// on lane 0, loads the tiles and issues the products.
+template <int CZ>
+struct PbFwdTraits {
+    static constexpr int TILE_BYTES = 128 * CZ * 2;            // CZ / 64 boxes of 16 KB
+    // tile buffers (a ring): more than two measured no faster, the kernel being issue-bound
+    static constexpr int NBUF = 2;
+    static constexpr int WT_BYTES = 32 * CZ * 2;               // w'^T: rows 0-15 hi, 16-31 lo, x CZ
+    static constexpr int OFF_Z = 0;                            // 1024-byte aligned (SW128)
+    static constexpr int OFF_WT = OFF_Z + NBUF * TILE_BYTES;   // 1024-byte aligned (SW128)
+    static constexpr int OFF_S = OFF_WT + WT_BYTES;            // S_h [16]
+    static constexpr int OFF_BB = OFF_S + 64;                  // sum_c beta_c w[c,h] [16]
+    static constexpr int OFF_BAR = OFF_BB + 64;   // full[NBUF] z_free[NBUF] mma_done[2] acc_free[2] drain
+    static constexpr int OFF_MISC = OFF_BAR + 8 * (2 * NBUF + 5);   // abort flag, TMEM base
+    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+    static constexpr int THREADS = 160;
+    static_assert(WT_BYTES % 1024 == 0, "w' terms stay 1024-byte aligned");
+    static_assert(SMEM_BYTES + 1024 <= 233472, "one CTA per SM at least");
+};
+
+// byte offset of w'^T element (row n, channel c) in a 32 x CZ K-major tile: 64-channel blocks
+// of 32 rows x 128 bytes, 16-byte chunks swizzled by the row (the 128-byte swizzle)
+__device__ __forceinline__ uint32_t pb_wt_off(int n, int c) {
+    return (uint32_t)((c >> 6) * 4096 + n * 128 + ((((c & 63) >> 3) ^ (n & 7)) << 4) + (c & 7) * 2);
+}
+
 template <int CZ, int HP>
-__global__ void __launch_bounds__(128) pba_pair_bias_fwd_kernel(const __grid_constant__ CUtensorMap tmZ,
+__global__ void __launch_bounds__(160) pba_pair_bias_fwd_kernel(const __grid_constant__ CUtensorMap tmZ,
                                                                  const PbArgs a) {
-    using T = PbTraits<CZ, HP>;
+    using T = PbFwdTraits<CZ>;
+    static_assert(HP <= 16, "heads");
     extern __shared__ __align__(1024) uint8_t dsmem[];
     const uint32_t sbase = smem_u32(dsmem);
     if (sbase & 1023u) {
         if (threadIdx.x == 0) watchdog_fire(SITE_PB_ALIGN);
         return;
     }
-    const int tid = threadIdx.x;
-    const float *sW = reinterpret_cast<const float *>(dsmem + T::OFF_W);
-    const float *sB = reinterpret_cast<const float *>(dsmem + T::OFF_BB);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *sS = reinterpret_cast<float *>(dsmem + T::OFF_S);
+    float *sB = reinterpret_cast<float *>(dsmem + T::OFF_BB);
     uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
+    constexpr int NB = T::NBUF;
+    auto b_full = [&](int y) { return smem_u32(&bars[y]); };             // tile buffer y landed
+    auto b_zfree = [&](int y) { return smem_u32(&bars[NB + y]); };       // its rows read by the threads
+    auto b_mma = [&](int x) { return smem_u32(&bars[2 * NB + x]); };     // products into accumulator x done
+    auto b_afree = [&](int x) { return smem_u32(&bars[2 * NB + 2 + x]); };   // accumulator x read out
+    const uint32_t b_drain = smem_u32(&bars[2 * NB + 4]);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MISC + 4);
     const int n_items = (int)blockIdx.x < a.tiles ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
 
-    pb_setup<CZ, HP>(a, dsmem, true);
-    int issued = 0;
     if (tid == 0) {
-        tma_prefetch_desc(&tmZ);
-        for (; issued < 2 && issued < n_items; ++issued)
-            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, smem_u32(&bars[issued]),
-                         tile_of(issued), a.nJt);
-    }
-    int n = 0;
-    for (; n < n_items; ++n) {
-        const int buf = n & 1;
-        bool ok = mbar_wait(smem_u32(&bars[buf]), (n >> 1) & 1, abort_flag, SITE_PB_FWD | (n << 12));
-        if (!__syncthreads_and(ok)) break;
-        const uint32_t zb = sbase + T::OFF_Z + buf * T::TILE_BYTES;
-        float mu, rstd, acc[HP];
-        pb_row_stats<CZ, HP>(sW, zb, tid, a.eps, mu, rstd, acc);
-        __syncthreads();   // every row has been read: the buffer may be refilled
-        if (tid == 0 && issued < n_items) {
-            pb_issue<CZ>(&tmZ, zb, smem_u32(&bars[buf]), tile_of(issued), a.nJt);
-            ++issued;
+        for (int y = 0; y < NB; ++y) {
+            mbar_init(b_full(y), 1);
+            mbar_init(b_zfree(y), 128);
         }
-        const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
-        if (j < a.Nj) {
-            __nv_bfloat16 *dst = a.bias + (long long)i * a.sb1 + j;
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(b_mma(x), 1);
+            mbar_init(b_afree(x), 128);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // w'^T as hi + lo bf16 terms (zero rows for padded heads), and the per-head constants
+    for (int e = tid; e < 16 * CZ; e += blockDim.x) {
+        const int n = e / CZ, c = e % CZ;
+        const float wv = n < a.H ? a.gamma[c] * a.w[c * a.H + n] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(wv - __bfloat162float(hi));
+        *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WT + pb_wt_off(n, c)) = hi;
+        *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WT + pb_wt_off(16 + n, c)) = lo;
+    }
+    if (warp < 4) {
+        // S_h = sum_c gamma_c w[c,h] and sum_c beta_c w[c,h]: warp w takes heads w, w + 4, ...
+        for (int h = warp; h < 16; h += 4) {
+            float sv = 0.f, bb = 0.f;
+            if (h < a.H)
+                for (int c = lane; c < CZ; c += 32) {
+                    sv = fmaf(a.gamma[c], a.w[c * a.H + h], sv);
+                    bb = fmaf(a.beta[c], a.w[c * a.H + h], bb);
+                }
 #pragma unroll
-            for (int h = 0; h < HP; ++h)
-                if (h < a.H) dst[h * a.sb0] = __float2bfloat16_rn(fmaf(rstd, acc[h], sB[h]));
+            for (int o = 16; o > 0; o >>= 1) {
+                sv += __shfl_xor_sync(0xffffffffu, sv, o);
+                bb += __shfl_xor_sync(0xffffffffu, bb, o);
+            }
+            if (lane == 0) {
+                sS[h] = sv;
+                sB[h] = bb;
+            }
+        }
+    } else {
+        tmem_alloc(smem_u32(s_tmem), 64);
+        tmem_relinquish();
+    }
+    fence_proxy_async();   // the w' terms are read by the tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    int issued = 0;        // warp 4, lane 0: tiles whose loads were issued
+
+    if (warp == 4) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(128, 32, false, false);
+            tma_prefetch_desc(&tmZ);
+            for (; issued < NB && issued < n_items; ++issued)
+                pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, b_full(issued), tile_of(issued), a.nJt);
+            bool ok = true;
+            for (int n = 0; n < n_items && ok; ++n) {
+                const int x = n & 1, y = n % NB;   // accumulator, tile buffer
+                ok = mbar_wait_all(abort_flag, b_full(y), (n / NB) & 1, true, SITE_PB_FWD | (n << 12),
+                                   b_afree(x), ((n >> 1) - 1) & 1, n >= 2, SITE_PB_FWD | 0x10 | (n << 12));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t zb = sbase + T::OFF_Z + y * T::TILE_BYTES;
+                const uint64_t dz = sdesc(zb, 16, 1024, kSw128);
+                const uint64_t dw = sdesc(sbase + T::OFF_WT, 16, 1024, kSw128);
+#pragma unroll
+                for (int kk = 0; kk < CZ / 16; ++kk) {
+                    const uint32_t za = (kk >> 2) * 16384 + (kk & 3) * 32, wa = (kk >> 2) * 4096 + (kk & 3) * 32;
+                    umma_ss(tbase + x * 32, sdesc_add(dz, za), sdesc_add(dw, wa), idesc, kk > 0);
+                }
+                umma_commit(b_mma(x));
+                // the previous tile's buffer, once its rows are read and its products done,
+                // takes tile n - 1 + NB
+                if (n >= 1 && issued < n_items) {
+                    const int m = n - 1, ym = m % NB;
+                    ok = mbar_wait_all(abort_flag, b_zfree(ym), (m / NB) & 1, true, SITE_PB_FWD | 0x20 | (n << 12),
+                                       b_mma(m & 1), (m >> 1) & 1, true, SITE_PB_FWD | 0x30 | (n << 12));
+                    if (!ok) break;
+                    pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + ym * T::TILE_BYTES, b_full(ym), tile_of(issued), a.nJt);
+                    ++issued;
+                }
+            }
+        }
+    } else {
+        // thread = position p of the tile = TMEM lane
+        const uint32_t lane_off = ((uint32_t)(warp * 32)) << 16;
+        bool ok = true;
+        for (int n = 0; n < n_items && ok; ++n) {
+            const int x = n & 1, y = n % NB;
+            const uint32_t zb = sbase + T::OFF_Z + y * T::TILE_BYTES;
+            ok = mbar_wait(b_full(y), (n / NB) & 1, abort_flag, SITE_PB_FWD | 0x40 | (n << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            // the row's mean, then 1 / sqrt(var + eps) in a second pass
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+            for (int q = 0; q < CZ / 8; ++q) {
+                const uint4 v = lds128(pb_chunk(zb, tid, q));
+                const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    s0 += bf16lo(xw[e]);
+                    s1 += bf16hi(xw[e]);
+                }
+            }
+            const float mu = (s0 + s1) * (1.f / CZ);
+            float2 var2 = make_float2(0.f, 0.f);
+            const float2 nmu = make_float2(-mu, -mu);
+#pragma unroll 4
+            for (int q = 0; q < CZ / 8; ++q) {
+                const uint4 v = lds128(pb_chunk(zb, tid, q));
+                const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 d = fadd2(make_float2(bf16lo(xw[e]), bf16hi(xw[e])), nmu);
+                    var2 = ffma2(d, d, var2);
+                }
+            }
+            const float rstd = rsqrtf((var2.x + var2.y) * (1.f / CZ) + a.eps);
+            mbar_arrive(b_zfree(y));
+            ok = mbar_wait(b_mma(x), (n >> 1) & 1, abort_flag, SITE_PB_FWD | 0x50 | (n << 12));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t acc[32];   // sum_c z w'_hi in columns 0-15, sum_c z w'_lo in 16-31
+            tmem_ld32(tbase + x * 32 + lane_off, acc);
+            tc_fence_before();
+            mbar_arrive(b_afree(x));
+            const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
+            if (j < a.Nj) {
+                __nv_bfloat16 *dst = a.bias + (long long)i * a.sb1 + j;
+#pragma unroll
+                for (int h = 0; h < HP; ++h)
+                    if (h < a.H)
+                        dst[h * a.sb0] = __float2bfloat16_rn(
+                            fmaf(rstd, fmaf(-mu, sS[h], __uint_as_float(acc[h]) + __uint_as_float(acc[16 + h])), sB[h]));
+            }
         }
     }
-    if (*abort_flag && tid == 0) {
-        // loads issued for tiles [n, issued) may still be in flight: let them land
-        for (int m = n; m < issued; ++m) mbar_wait_drain(smem_u32(&bars[m & 1]), (m >> 1) & 1);
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && warp == 4 && lane == 0) {
+        // loads issued for tiles not yet consumed may still land, products may still run
+        for (int m = max(0, issued - NB); m < issued; ++m) mbar_wait_drain(b_full(m % NB), (m / NB) & 1);
+        umma_commit(b_drain);
+        mbar_wait_drain(b_drain, 0);
     }
     __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 64);
+    }
 }
 
 template <int CZ, int HP>
