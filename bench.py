@@ -863,6 +863,7 @@ def pb_work(N, Cz, H, Ni=None):
     bwd = P * Cz * 2 + H * P * 4 + P * Cz * 2
     return {"fwd_bytes": fwd, "bwd_bytes": bwd,
             "kernels": {"pba_pair_bias_fwd_kernel": (0, fwd), "pba_pair_bias_bwd_kernel": (0, bwd),
+                        "pba_pair_bias_bwd_tc_kernel": (0, bwd),   # the backward at Cz = 128
                         "pba_pair_bias_reduce_kernel": (0, 0), "pba_pair_bias_param_kernel": (0, 0)}}
 
 

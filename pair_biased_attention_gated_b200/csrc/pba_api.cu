@@ -45,7 +45,8 @@ pba_status cuda_fail(cudaError_t e, const char *what) {
 // ---------------------------------------------------------------------------- profiling
 enum KernelId { K_FWD = 0, K_BWD_PRE, K_BWD_MAIN, K_DBIAS, K_DQ_CONVERT, K_ZERO_ROWS,
                 K_PWA_WEIGHTS, K_PWA_FWD, K_PWA_PRE, K_PWA_DV, K_PWA_DW, K_PWA_DBIAS,
-                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_DBIAS_ZERO, K_DBIAS_SUM, K_COUNT };
+                K_PB_FWD, K_PB_BWD, K_PB_REDUCE, K_PB_PARAM, K_DBIAS_ZERO, K_DBIAS_SUM, K_PB_BWD_TC,
+                K_COUNT };
 const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel", "pba_bwd_main_kernel",
                                            "pba_dbias_kernel",
                                            "pba_dq_convert_kernel", "zero_rows_kernel",
@@ -54,7 +55,8 @@ const char *const kKernelNames[K_COUNT] = {"pba_fwd_kernel", "pba_bwd_pre_kernel
                                            "pba_pwa_dw_kernel", "pba_pwa_dbias_kernel",
                                            "pba_pair_bias_fwd_kernel", "pba_pair_bias_bwd_kernel",
                                            "pba_pair_bias_reduce_kernel", "pba_pair_bias_param_kernel",
-                                           "pba_dbias_zero_kernel", "pba_dbias_sum_kernel"};
+                                           "pba_dbias_zero_kernel", "pba_dbias_sum_kernel",
+                                           "pba_pair_bias_bwd_tc_kernel"};
 struct ProfRec {
     int kid;
     cudaEvent_t a, b;
@@ -902,7 +904,11 @@ long long pb_grid(const pba_pair_bias_dims *d, int smem_bytes) {
 }
 
 template <int CZ, int HP>
-int pb_smem() { return pba::PbTraits<CZ, HP>::SMEM_BYTES; }
+int pb_smem() {
+    // the backward's layout (its grid fixes the partials): Cz = 128 has its own kernel
+    if constexpr (CZ == 128) return pba::PbBwdTcTraits<HP>::SMEM_BYTES;
+    else return pba::PbTraits<CZ, HP>::SMEM_BYTES;
+}
 
 int pb_smem_for(int Cz, int HP) {
 #define PB_CASE(cz, hp) if (Cz == cz && HP == hp) return pb_smem<cz, hp>();
@@ -950,7 +956,8 @@ pba::PbArgs pb_args(const pba_pair_bias_dims *d, const float *gamma, const float
 template <int CZ, int HP>
 pba_status launch_pb(bool bwd, const CUtensorMap &tm, pba::PbArgs a, const pba_pair_bias_dims *d, cudaStream_t s) {
     using T = pba::PbTraits<CZ, HP>;
-    const long long grid = pb_grid(d, T::SMEM_BYTES);
+    const int bwd_smem = pb_smem<CZ, HP>();
+    const long long grid = pb_grid(d, bwd_smem);
     a.nparts = (int)grid;
     pba_status st;
     cudaError_t e;
@@ -965,8 +972,13 @@ pba_status launch_pb(bool bwd, const CUtensorMap &tm, pba::PbArgs a, const pba_p
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pba_pair_bias_fwd_kernel launch");
         return PBA_OK;
     }
-    if ((st = set_smem(pba::pba_pair_bias_bwd_kernel<CZ, HP>, T::SMEM_BYTES)) != PBA_OK) return st;
-    {
+    if constexpr (CZ == 128) {
+        // parameter sums on the tensor core
+        if ((st = set_smem(pba::pba_pair_bias_bwd_tc_kernel<HP>, bwd_smem)) != PBA_OK) return st;
+        ProfScope ps(K_PB_BWD_TC, s);
+        pba::pba_pair_bias_bwd_tc_kernel<HP><<<(unsigned)grid, 128, bwd_smem, s>>>(tm, a);
+    } else {
+        if ((st = set_smem(pba::pba_pair_bias_bwd_kernel<CZ, HP>, T::SMEM_BYTES)) != PBA_OK) return st;
         ProfScope ps(K_PB_BWD, s);
         pba::pba_pair_bias_bwd_kernel<CZ, HP><<<(unsigned)grid, 128, T::SMEM_BYTES, s>>>(tm, a);
     }

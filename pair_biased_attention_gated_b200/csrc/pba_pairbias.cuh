@@ -77,9 +77,8 @@ __device__ __forceinline__ int pb_widx(int c, int h, int HP) { return ((c >> 1) 
 
 // Block setup: w' = gamma w (zero-padded to HP columns), its column sums S and the beta
 // projection; initialises the two tile barriers.
-template <int CZ, int HP>
+template <int CZ, int HP, typename T = PbTraits<CZ, HP>>
 __device__ __forceinline__ void pb_setup(const PbArgs &a, uint8_t *dsmem, bool with_bb) {
-    using T = PbTraits<CZ, HP>;
     float *sW = reinterpret_cast<float *>(dsmem + T::OFF_W);
     float *sS = reinterpret_cast<float *>(dsmem + T::OFF_S);
     float *sB = reinterpret_cast<float *>(dsmem + T::OFF_BB);
@@ -525,6 +524,200 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_kernel(const __grid_con
         if (tid < HP) dst[CZ * HP + tid] = G;
     }
     __syncthreads();
+}
+
+// Backward for Cz = 128 with the parameter sums on the tensor core.  Phase 1 is the kernel
+// above's (thread = position: the row's statistics, dz); the sums A[c,h] = sum_pos xh_c g_h
+// become A = Z^T G1 - (sum_pos mean_pos G1[pos,:]) with G1[pos,h] = rstd_pos g_pos,h: per tile,
+// one M = 128 (channels) x N = 32 x K = 16 (positions) product per 16 positions, accumulated
+// in TMEM over all of the block's tiles.  The z tile itself is the A operand: its rows are
+// positions (K) of 128 bytes of channels (M), which is the MN-major layout with the 128-byte
+// swizzle (64-channel blocks 16 KB apart).  G1 enters as two bf16 terms (hi in rows 0-15, lo in
+// 16-31) for fp32 accuracy.  The per-block partials have the layout of the kernel above.
+template <int HP>
+struct PbBwdTcTraits {
+    static constexpr int CZ = 128;
+    static constexpr int TILE_BYTES = 128 * CZ * 2;
+    static constexpr int OFF_Z = 0;                            // 1024-byte aligned (SW128)
+    static constexpr int OFF_GT = OFF_Z + 2 * TILE_BYTES;      // G1^T: 32 rows x 128 positions bf16
+    static constexpr int OFF_W = OFF_GT + 32 * 128 * 2;        // w' fp32, channel pairs interleaved
+    static constexpr int OFF_S = OFF_W + CZ * HP * 4;          // S [HP]
+    static constexpr int OFF_BB = OFF_S + HP * 4;              // (unused here) [HP]
+    static constexpr int OFF_BAR = OFF_BB + HP * 4;            // full[2], mma_done, drain
+    static constexpr int OFF_MISC = OFF_BAR + 32;              // abort flag, TMEM base
+    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+    static_assert(OFF_GT % 1024 == 0, "G1^T 1024-byte aligned");
+    static_assert(2 * TILE_BYTES >= 128 * 2 * HP * 4, "the tile buffers hold the final per-thread sums");
+};
+
+template <int HP>
+__global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmZ,
+                                                                    const PbArgs a) {
+    constexpr int CZ = 128;
+    using T = PbBwdTcTraits<HP>;
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    const uint32_t sbase = smem_u32(dsmem);
+    if (sbase & 1023u) {
+        if (threadIdx.x == 0) watchdog_fire(SITE_PB_ALIGN);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const float *sW = reinterpret_cast<const float *>(dsmem + T::OFF_W);
+    const float *sS = reinterpret_cast<const float *>(dsmem + T::OFF_S);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
+    const uint32_t b_mma = smem_u32(&bars[2]), b_drain = smem_u32(&bars[3]);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MISC + 4);
+    const int n_items = (int)blockIdx.x < a.tiles ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
+
+    if (tid == 0) {
+        mbar_init(b_mma, 1);
+        mbar_init(b_drain, 1);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(s_tmem), 32);
+        tmem_relinquish();
+    }
+    // G1^T starts zero: the rows of padded heads stay zero
+    for (int e = tid; e < 32 * 128 * 2 / 16; e += 128)
+        sts128(sbase + T::OFF_GT + e * 16, make_uint4(0, 0, 0, 0));
+    tc_fence_before();
+    pb_setup<CZ, HP, T>(a, dsmem, false);   // barriers full[0..1], abort flag, w', S (synchronises)
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    float Gs[HP], Ms[HP];   // this thread's positions: sum of g_h, sum of mean G1_h
+#pragma unroll
+    for (int h = 0; h < HP; ++h) Gs[h] = Ms[h] = 0.f;
+    int issued = 0;
+    if (tid == 0) {
+        tma_prefetch_desc(&tmZ);
+        for (; issued < 2 && issued < n_items; ++issued)
+            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, smem_u32(&bars[issued]),
+                         tile_of(issued), a.nJt);
+    }
+    constexpr uint32_t idesc = idesc_bf16(128, 32, true, false);
+    int n = 0;
+    for (; n < n_items; ++n) {
+        const int buf = n & 1;
+        const uint32_t zb = sbase + T::OFF_Z + buf * T::TILE_BYTES;
+        bool ok = mbar_wait(smem_u32(&bars[buf]), (n >> 1) & 1, abort_flag, SITE_PB_BWD | (n << 12));
+        if (!__syncthreads_and(ok)) break;
+        const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
+        const bool valid = j < a.Nj;
+        // ---- phase 1: thread = position j; dz of its row, and its row of G1^T
+        {
+            float mu, rstd, acc[HP];
+            pb_row_stats<CZ, HP>(sW, zb, tid, a.eps, mu, rstd, acc);
+            float g[HP];
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+                g[h] = (valid && h < a.H) ? a.dbias[h * a.sd0 + (long long)i * a.sd1 + j] : 0.f;
+            float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+                s1 = fmaf(g[h], sS[h], s1);
+                s2 = fmaf(g[h], acc[h], s2);
+            }
+            const float m1 = s1 * (1.f / CZ);             // mean_c dxh
+            const float m2r = s2 * rstd * rstd * (1.f / CZ);   // mean_c(dxh xh) * rstd
+            if (valid) {
+                __nv_bfloat16 *dst = a.dz + (long long)i * a.sz0 + (long long)j * a.sz1;
+#pragma unroll 1
+                for (int q = 0; q < CZ / 8; ++q) {
+                    const uint4 v = lds128(pb_chunk(zb, tid, q));
+                    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 *wp = reinterpret_cast<const float4 *>(sW + pb_widx(q * 8 + 2 * e, 0, HP));
+                        float2 dx = make_float2(0.f, 0.f);   // dxh of the channel pair
+#pragma unroll
+                        for (int h2 = 0; h2 < HP / 2; ++h2) {
+                            const float4 w4 = wp[h2];
+                            dx = ffma2(make_float2(w4.x, w4.y), make_float2(g[2 * h2], g[2 * h2]), dx);
+                            dx = ffma2(make_float2(w4.z, w4.w), make_float2(g[2 * h2 + 1], g[2 * h2 + 1]), dx);
+                        }
+                        const float d0 = bf16lo(x[e]) - mu, d1 = bf16hi(x[e]) - mu;
+                        ow[e] = pack_bf16x2(rstd * (dx.x - m1 - d0 * m2r), rstd * (dx.y - m1 - d1 * m2r));
+                    }
+                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+            }
+            // G1 = rstd g (zero for positions past the row's end); the previous tile's products,
+            // which read G1^T, were waited for by thread 0 before this tile began
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+                const float g1 = valid ? rstd * g[h] : 0.f;
+                Gs[h] += g[h];
+                Ms[h] = fmaf(mu, g1, Ms[h]);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(g1);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(g1 - __bfloat162float(hi));
+                *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(h, tid)) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(16 + h, tid)) = lo;
+            }
+            fence_proxy_async();   // read by the tensor core
+        }
+        __syncthreads();
+        // ---- the tile's products (thread 0), then its buffer's refill once they are done
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t da = sdesc(zb, 16384, 1024, kSw128);
+            const uint64_t dg = sdesc(sbase + T::OFF_GT, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_ss(tbase, sdesc_add(da, kk * 2048), sdesc_add(dg, (kk >> 2) * 4096 + (kk & 3) * 32), idesc,
+                        (n > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(b_mma);
+            ok = mbar_wait(b_mma, n & 1, abort_flag, SITE_PB_BWD | 0x10 | (n << 12));
+            if (ok && issued < n_items) {
+                pb_issue<CZ>(&tmZ, zb, smem_u32(&bars[buf]), tile_of(issued), a.nJt);
+                ++issued;
+            }
+        }
+    }
+    __syncthreads();
+    const bool aborted = *abort_flag != 0;
+    if (aborted && tid == 0) {
+        for (int m = n; m < issued; ++m) mbar_wait_drain(smem_u32(&bars[m & 1]), (m >> 1) & 1);
+        umma_commit(b_drain);
+        mbar_wait_drain(b_drain, 0);
+    }
+    if (!aborted) {
+        // the block's sums of g and of mean G1 over its positions: per thread, then over the
+        // threads in order (through the idle tile buffers)
+        float *red = reinterpret_cast<float *>(dsmem + T::OFF_Z);
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+            red[tid * 2 * HP + h] = Gs[h];
+            red[tid * 2 * HP + HP + h] = Ms[h];
+        }
+        __syncthreads();
+        float *tot = red + 128 * 2 * HP;   // [2 HP]
+        if (tid < 2 * HP) {
+            float v = 0.f;
+            for (int r = 0; r < 128; ++r) v += red[r * 2 * HP + tid];
+            tot[tid] = v;
+        }
+        __syncthreads();
+        // thread = channel = TMEM lane: A[c,h] = (Z^T G1_hi)[c,h] + (Z^T G1_lo)[c,h] - sum mean G1_h
+        float *dst = a.part + (long long)blockIdx.x * (CZ * HP + HP);
+        uint32_t d[32];
+        if (n_items > 0) {
+            tc_fence_after();
+            tmem_ld32(tbase + (((uint32_t)(warp * 32)) << 16), d);
+        }
+#pragma unroll
+        for (int h = 0; h < HP; ++h)
+            dst[tid * HP + h] = n_items > 0 ? (__uint_as_float(d[h]) + __uint_as_float(d[16 + h])) - tot[HP + h] : 0.f;
+        if (tid < HP) dst[CZ * HP + tid] = tot[tid];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 32);
+    }
 }
 
 // Sums of the per-block partials, column by column: block = 32 columns x 16 warps; warp w

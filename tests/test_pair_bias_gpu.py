@@ -79,6 +79,10 @@ CASES = {
     "c256_h4_ragged": (3, 200, 256, 4),
     "h3_padded": (5, 130, 128, 3),
     "msa_row_pair_256": (256, 256, 128, 8),
+    # Cz = 128 runs the backward whose parameter sums are tensor-core products: every padded
+    # head count (4, 8, 16), one head, and a ragged row end
+    "c128_h16_ragged": (3, 200, 128, 16),
+    "c128_h1_ragged": (4, 77, 128, 1),
 }
 
 
