@@ -526,29 +526,43 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_kernel(const __grid_con
     __syncthreads();
 }
 
-// Backward for Cz = 128 with the parameter sums on the tensor core.  Phase 1 is the kernel
-// above's (thread = position: the row's statistics, dz); the sums A[c,h] = sum_pos xh_c g_h
-// become A = Z^T G1 - (sum_pos mean_pos G1[pos,:]) with G1[pos,h] = rstd_pos g_pos,h: per tile,
-// one M = 128 (channels) x N = 32 x K = 16 (positions) product per 16 positions, accumulated
-// in TMEM over all of the block's tiles.  The z tile itself is the A operand: its rows are
-// positions (K) of 128 bytes of channels (M), which is the MN-major layout with the 128-byte
-// swizzle (64-channel blocks 16 KB apart).  G1 enters as two bf16 terms (hi in rows 0-15, lo in
-// 16-31) for fp32 accuracy.  The per-block partials have the layout of the kernel above.
+// Backward for Cz = 128 with its three contractions on the tensor core; the threads keep the
+// LayerNorm statistics and the elementwise part of dz.  Per tile of 128 positions:
+//   acc[p,h]  = sum_c z[p,c] w'[c,h]         M = 128 positions, N = 32, K = 128 channels (the
+//               z tile as the K-major A operand; w' as hi and lo bf16 rows, as in the forward)
+//   dxh[p,c]  = sum_h g[p,h] w'[c,h]         M = 128 positions, N = 128 channels, K = 3 x 16:
+//               g_hi w_hi + g_hi w_lo + g_lo w_hi (fp32 accuracy), one 64-wide K block
+//   A[c,h]   += sum_p z[p,c] G1[p,h]          M = 128 channels, N = 32, K = 16 positions per
+//               product: the z tile as the MN-major A operand (rows = positions of 128 bytes of
+//               channels, the 128-byte swizzle, 64-channel blocks 16 KB apart), G1 = rstd g as
+//               hi and lo rows, accumulated in TMEM over all of the block's tiles
+// and A = sum_p (z - mean) G1 = that sum - sum_p mean_p G1[p,:].  The per-block partials have the
+// layout of the kernel above, so their reduction stays bit-stable.
 template <int HP>
 struct PbBwdTcTraits {
     static constexpr int CZ = 128;
     static constexpr int TILE_BYTES = 128 * CZ * 2;
-    static constexpr int OFF_Z = 0;                            // 1024-byte aligned (SW128)
+    static constexpr int OFF_Z = 0;                            // 2 tiles, 1024-byte aligned (SW128)
     static constexpr int OFF_GT = OFF_Z + 2 * TILE_BYTES;      // G1^T: 32 rows x 128 positions bf16
-    static constexpr int OFF_W = OFF_GT + 32 * 128 * 2;        // w' fp32, channel pairs interleaved
-    static constexpr int OFF_S = OFF_W + CZ * HP * 4;          // S [HP]
-    static constexpr int OFF_BB = OFF_S + HP * 4;              // (unused here) [HP]
-    static constexpr int OFF_BAR = OFF_BB + HP * 4;            // full[2], mma_done, drain
-    static constexpr int OFF_MISC = OFF_BAR + 32;              // abort flag, TMEM base
+    static constexpr int OFF_WF = OFF_GT + 32 * 128 * 2;       // w'^T: 32 rows (hi, lo) x 128 channels
+    static constexpr int OFF_G = OFF_WF + 32 * 128 * 2;        // g: 128 positions x 64 (g_hi, g_hi, g_lo, 0)
+    static constexpr int OFF_WB = OFF_G + 128 * 128;           // w': 128 channels x 64 (w_hi, w_lo, w_hi, 0)
+    static constexpr int OFF_S = OFF_WB + 128 * 128;           // S_h = sum_c w'[c,h] [16]
+    static constexpr int OFF_RED = OFF_S + 64;                 // setup: per-warp head sums [4][16]
+    static constexpr int OFF_BAR = OFF_RED + 256;              // full[2], acc, dx, all, drain
+    static constexpr int OFF_MISC = OFF_BAR + 48;              // abort flag, TMEM base
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
-    static_assert(OFF_GT % 1024 == 0, "G1^T 1024-byte aligned");
-    static_assert(2 * TILE_BYTES >= 128 * 2 * HP * 4, "the tile buffers hold the final per-thread sums");
+    static constexpr uint32_t T_ACC = 0, T_A = 32, T_DX = 128;   // TMEM columns (256 allocated)
+    static_assert(OFF_GT % 1024 == 0 && OFF_WF % 1024 == 0 && OFF_G % 1024 == 0 && OFF_WB % 1024 == 0,
+                  "operands 1024-byte aligned");
+    static_assert(2 * TILE_BYTES >= 128 * 2 * HP * 4 + 2 * HP * 4, "the tile buffers hold the final sums");
+    static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two blocks per SM");
 };
+
+// byte offset of element (row r, k) of a 128-row x 64 K-major tile with the 128-byte swizzle
+__device__ __forceinline__ uint32_t pb_k64_off(int r, int k) {
+    return (uint32_t)(r * 128 + (((k >> 3) ^ (r & 7)) << 4) + (k & 7) * 2);
+}
 
 template <int HP>
 __global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmZ,
@@ -561,117 +575,207 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_
         if (threadIdx.x == 0) watchdog_fire(SITE_PB_ALIGN);
         return;
     }
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const float *sW = reinterpret_cast<const float *>(dsmem + T::OFF_W);
-    const float *sS = reinterpret_cast<const float *>(dsmem + T::OFF_S);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *sS = reinterpret_cast<float *>(dsmem + T::OFF_S);
     uint64_t *bars = reinterpret_cast<uint64_t *>(dsmem + T::OFF_BAR);
-    const uint32_t b_mma = smem_u32(&bars[2]), b_drain = smem_u32(&bars[3]);
+    auto b_full = [&](int x) { return smem_u32(&bars[x]); };
+    const uint32_t b_acc = smem_u32(&bars[2]), b_dx = smem_u32(&bars[3]), b_all = smem_u32(&bars[4]),
+                   b_drain = smem_u32(&bars[5]);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(dsmem + T::OFF_MISC);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dsmem + T::OFF_MISC + 4);
     const int n_items = (int)blockIdx.x < a.tiles ? (a.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     auto tile_of = [&](int n) { return (int)blockIdx.x + n * (int)gridDim.x; };
 
+    int issued = 0;   // thread 0: tiles whose loads were issued
     if (tid == 0) {
-        mbar_init(b_mma, 1);
+        mbar_init(b_full(0), 1);
+        mbar_init(b_full(1), 1);
+        mbar_init(b_acc, 1);
+        mbar_init(b_dx, 1);
+        mbar_init(b_all, 1);
         mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmZ);
+        for (; issued < 2 && issued < n_items; ++issued)
+            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, b_full(issued), tile_of(issued), a.nJt);
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(s_tmem), 32);
+        tmem_alloc(smem_u32(s_tmem), 256);
         tmem_relinquish();
     }
-    // G1^T starts zero: the rows of padded heads stay zero
-    for (int e = tid; e < 32 * 128 * 2 / 16; e += 128)
-        sts128(sbase + T::OFF_GT + e * 16, make_uint4(0, 0, 0, 0));
+    // operand tiles: w' = gamma w as hi and lo bf16 terms, zeros elsewhere (padded heads, the
+    // unused K slice); thread = channel c; all its loads issued before any is used
+    {
+        const int c = tid;
+        const float gc = __ldg(a.gamma + c);
+        float wv[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) wv[h] = h < a.H ? __ldg(a.w + c * a.H + h) : 0.f;
+        float *red = reinterpret_cast<float *>(dsmem + T::OFF_RED);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            const float v = gc * wv[h];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WF + pb_wt_off(h, c)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WF + pb_wt_off(16 + h, c)) = lo;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WB + pb_k64_off(c, h)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WB + pb_k64_off(c, 16 + h)) = lo;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WB + pb_k64_off(c, 32 + h)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_WB + pb_k64_off(c, 48 + h)) = __float2bfloat16_rn(0.f);
+            // S_h = sum_c w'[c,h]: each warp's butterfly, then the warps in order
+            float sv = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
+            if (lane == 0) red[warp * 16 + h] = sv;
+        }
+        // G1^T and g start zero (padded heads, the unused K slice)
+        for (int e = tid; e < 32 * 128 * 2 / 16; e += 128) sts128(sbase + T::OFF_GT + e * 16, make_uint4(0, 0, 0, 0));
+        for (int e = tid; e < 128 * 128 / 16; e += 128) sts128(sbase + T::OFF_G + e * 16, make_uint4(0, 0, 0, 0));
+        __syncthreads();
+        if (tid < 16) sS[tid] = ((red[tid] + red[16 + tid]) + red[32 + tid]) + red[48 + tid];
+    }
+    fence_proxy_async();   // the operand tiles are read by the tensor core
     tc_fence_before();
-    pb_setup<CZ, HP, T>(a, dsmem, false);   // barriers full[0..1], abort flag, w', S (synchronises)
+    __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *s_tmem;
+    const uint32_t lane_off = ((uint32_t)(warp * 32)) << 16;
     float Gs[HP], Ms[HP];   // this thread's positions: sum of g_h, sum of mean G1_h
 #pragma unroll
     for (int h = 0; h < HP; ++h) Gs[h] = Ms[h] = 0.f;
-    int issued = 0;
-    if (tid == 0) {
-        tma_prefetch_desc(&tmZ);
-        for (; issued < 2 && issued < n_items; ++issued)
-            pb_issue<CZ>(&tmZ, sbase + T::OFF_Z + issued * T::TILE_BYTES, smem_u32(&bars[issued]),
-                         tile_of(issued), a.nJt);
-    }
-    constexpr uint32_t idesc = idesc_bf16(128, 32, true, false);
+    constexpr uint32_t id_acc = idesc_bf16(128, 32, false, false);
+    constexpr uint32_t id_dx = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t id_a = idesc_bf16(128, 32, true, false);
     int n = 0;
     for (; n < n_items; ++n) {
         const int buf = n & 1;
         const uint32_t zb = sbase + T::OFF_Z + buf * T::TILE_BYTES;
-        bool ok = mbar_wait(smem_u32(&bars[buf]), (n >> 1) & 1, abort_flag, SITE_PB_BWD | (n << 12));
+        bool ok = mbar_wait(b_full(buf), (n >> 1) & 1, abort_flag, SITE_PB_BWD | (n << 12));
         if (!__syncthreads_and(ok)) break;
+        if (tid == 0) {   // acc = z w' for the tile
+            tc_fence_after();
+            const uint64_t dz = sdesc(zb, 16, 1024, kSw128), dw = sdesc(sbase + T::OFF_WF, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < CZ / 16; ++kk)
+                umma_ss(tbase + T::T_ACC, sdesc_add(dz, (kk >> 2) * 16384 + (kk & 3) * 32),
+                        sdesc_add(dw, (kk >> 2) * 4096 + (kk & 3) * 32), id_acc, kk > 0);
+            umma_commit(b_acc);
+        }
         const int t = tile_of(n), i = t / a.nJt, j = (t % a.nJt) * 128 + tid;
         const bool valid = j < a.Nj;
-        // ---- phase 1: thread = position j; dz of its row, and its row of G1^T
-        {
-            float mu, rstd, acc[HP];
-            pb_row_stats<CZ, HP>(sW, zb, tid, a.eps, mu, rstd, acc);
-            float g[HP];
+        float g[HP];
 #pragma unroll
-            for (int h = 0; h < HP; ++h)
-                g[h] = (valid && h < a.H) ? a.dbias[h * a.sd0 + (long long)i * a.sd1 + j] : 0.f;
-            float s1 = 0.f, s2 = 0.f;
+        for (int h = 0; h < HP; ++h)
+            g[h] = (valid && h < a.H) ? a.dbias[h * a.sd0 + (long long)i * a.sd1 + j] : 0.f;
+        // the row's mean, then 1 / sqrt(var + eps) in a second pass (thread = position)
+        float s0 = 0.f, s1p = 0.f;
+#pragma unroll 4
+        for (int q = 0; q < CZ / 8; ++q) {
+            const uint4 v = lds128(pb_chunk(zb, tid, q));
+            const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s0 += bf16lo(xw[e]);
+                s1p += bf16hi(xw[e]);
+            }
+        }
+        const float mu = (s0 + s1p) * (1.f / CZ);
+        float2 var2 = make_float2(0.f, 0.f);
+        const float2 nmu = make_float2(-mu, -mu);
+#pragma unroll 4
+        for (int q = 0; q < CZ / 8; ++q) {
+            const uint4 v = lds128(pb_chunk(zb, tid, q));
+            const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 d = fadd2(make_float2(bf16lo(xw[e]), bf16hi(xw[e])), nmu);
+                var2 = ffma2(d, d, var2);
+            }
+        }
+        const float rstd = rsqrtf((var2.x + var2.y) * (1.f / CZ) + a.eps);
+        ok = mbar_wait(b_acc, n & 1, abort_flag, SITE_PB_BWD | 0x10 | (n << 12));
+        ok = __all_sync(0xffffffffu, ok);
+        float s1 = 0.f, s2 = 0.f;
+        if (ok) {
+            tc_fence_after();
+            uint32_t d[32];
+            tmem_ld32(tbase + T::T_ACC + lane_off, d);
 #pragma unroll
             for (int h = 0; h < HP; ++h) {
+                const float acc = fmaf(-mu, sS[h], __uint_as_float(d[h]) + __uint_as_float(d[16 + h]));
                 s1 = fmaf(g[h], sS[h], s1);
-                s2 = fmaf(g[h], acc[h], s2);
+                s2 = fmaf(g[h], acc, s2);
             }
-            const float m1 = s1 * (1.f / CZ);             // mean_c dxh
-            const float m2r = s2 * rstd * rstd * (1.f / CZ);   // mean_c(dxh xh) * rstd
-            if (valid) {
-                __nv_bfloat16 *dst = a.dz + (long long)i * a.sz0 + (long long)j * a.sz1;
+        }
+        const float m1 = s1 * (1.f / CZ);                  // mean_c dxh
+        const float m2r = s2 * rstd * rstd * (1.f / CZ);   // mean_c(dxh xh) * rstd
+        // this position's g (for dxh) and G1 = rstd g (for A), as hi and lo bf16 terms
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+            const float g1 = valid ? rstd * g[h] : 0.f;
+            Gs[h] += g[h];
+            Ms[h] = fmaf(mu, g1, Ms[h]);
+            const __nv_bfloat16 ghi = __float2bfloat16_rn(g[h]);
+            const __nv_bfloat16 glo = __float2bfloat16_rn(g[h] - __bfloat162float(ghi));
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_G + pb_k64_off(tid, h)) = ghi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_G + pb_k64_off(tid, 16 + h)) = ghi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_G + pb_k64_off(tid, 32 + h)) = glo;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(g1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(g1 - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(h, tid)) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(16 + h, tid)) = lo;
+        }
+        fence_proxy_async();   // read by the tensor core
+        tc_fence_before();
+        if (!__syncthreads_and(ok)) break;
+        if (tid == 0) {   // dxh = g w'^T, then A += z^T G1
+            tc_fence_after();
+            const uint64_t dg = sdesc(sbase + T::OFF_G, 16, 1024, kSw128), dwb = sdesc(sbase + T::OFF_WB, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 3; ++kk)
+                umma_ss(tbase + T::T_DX, sdesc_add(dg, kk * 32), sdesc_add(dwb, kk * 32), id_dx, kk > 0);
+            umma_commit(b_dx);
+            const uint64_t da = sdesc(zb, 16384, 1024, kSw128), dt = sdesc(sbase + T::OFF_GT, 16, 1024, kSw128);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_ss(tbase + T::T_A, sdesc_add(da, kk * 2048), sdesc_add(dt, (kk >> 2) * 4096 + (kk & 3) * 32), id_a,
+                        (n > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(b_all);
+        }
+        // dz = rstd (dxh - mean dxh - xh mean(dxh xh)), 32 channels at a time
+        ok = mbar_wait(b_dx, n & 1, abort_flag, SITE_PB_BWD | 0x20 | (n << 12));
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16 *dst = a.dz + (long long)i * a.sz0 + (long long)j * a.sz1;
 #pragma unroll 1
-                for (int q = 0; q < CZ / 8; ++q) {
+            for (int cb = 0; cb < CZ / 32; ++cb) {
+                uint32_t dxr[32];
+                tmem_ld32(tbase + T::T_DX + cb * 32 + lane_off, dxr);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int q = cb * 4 + q4;   // 16-byte chunk: channels 8 q .. 8 q + 7
                     const uint4 v = lds128(pb_chunk(zb, tid, q));
-                    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+                    const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
                     uint32_t ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float4 *wp = reinterpret_cast<const float4 *>(sW + pb_widx(q * 8 + 2 * e, 0, HP));
-                        float2 dx = make_float2(0.f, 0.f);   // dxh of the channel pair
-#pragma unroll
-                        for (int h2 = 0; h2 < HP / 2; ++h2) {
-                            const float4 w4 = wp[h2];
-                            dx = ffma2(make_float2(w4.x, w4.y), make_float2(g[2 * h2], g[2 * h2]), dx);
-                            dx = ffma2(make_float2(w4.z, w4.w), make_float2(g[2 * h2 + 1], g[2 * h2 + 1]), dx);
-                        }
-                        const float d0 = bf16lo(x[e]) - mu, d1 = bf16hi(x[e]) - mu;
-                        ow[e] = pack_bf16x2(rstd * (dx.x - m1 - d0 * m2r), rstd * (dx.y - m1 - d1 * m2r));
+                        const float dx0 = __uint_as_float(dxr[q4 * 8 + 2 * e]), dx1 = __uint_as_float(dxr[q4 * 8 + 2 * e + 1]);
+                        const float d0 = bf16lo(xw[e]) - mu, d1 = bf16hi(xw[e]) - mu;
+                        ow[e] = pack_bf16x2(rstd * (dx0 - m1 - d0 * m2r), rstd * (dx1 - m1 - d1 * m2r));
                     }
-                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    if (valid) *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
-            // G1 = rstd g (zero for positions past the row's end); the previous tile's products,
-            // which read G1^T, were waited for by thread 0 before this tile began
-#pragma unroll
-            for (int h = 0; h < HP; ++h) {
-                const float g1 = valid ? rstd * g[h] : 0.f;
-                Gs[h] += g[h];
-                Ms[h] = fmaf(mu, g1, Ms[h]);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(g1);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(g1 - __bfloat162float(hi));
-                *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(h, tid)) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(dsmem + T::OFF_GT + pb_wt_off(16 + h, tid)) = lo;
-            }
-            fence_proxy_async();   // read by the tensor core
         }
-        __syncthreads();
-        // ---- the tile's products (thread 0), then its buffer's refill once they are done
+        tc_fence_before();
+        if (!__syncthreads_and(ok)) break;   // the tile's rows are read: its buffer may be refilled
         if (tid == 0) {
-            tc_fence_after();
-            const uint64_t da = sdesc(zb, 16384, 1024, kSw128);
-            const uint64_t dg = sdesc(sbase + T::OFF_GT, 16, 1024, kSw128);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                umma_ss(tbase, sdesc_add(da, kk * 2048), sdesc_add(dg, (kk >> 2) * 4096 + (kk & 3) * 32), idesc,
-                        (n > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(b_mma);
-            ok = mbar_wait(b_mma, n & 1, abort_flag, SITE_PB_BWD | 0x10 | (n << 12));
+            ok = mbar_wait(b_all, n & 1, abort_flag, SITE_PB_BWD | 0x30 | (n << 12));
             if (ok && issued < n_items) {
-                pb_issue<CZ>(&tmZ, zb, smem_u32(&bars[buf]), tile_of(issued), a.nJt);
+                pb_issue<CZ>(&tmZ, zb, b_full(buf), tile_of(issued), a.nJt);
                 ++issued;
             }
         }
@@ -679,7 +783,7 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_
     __syncthreads();
     const bool aborted = *abort_flag != 0;
     if (aborted && tid == 0) {
-        for (int m = n; m < issued; ++m) mbar_wait_drain(smem_u32(&bars[m & 1]), (m >> 1) & 1);
+        for (int m = max(0, issued - 2); m < issued; ++m) mbar_wait_drain(b_full(m & 1), (m >> 1) & 1);
         umma_commit(b_drain);
         mbar_wait_drain(b_drain, 0);
     }
@@ -705,7 +809,7 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_
         uint32_t d[32];
         if (n_items > 0) {
             tc_fence_after();
-            tmem_ld32(tbase + (((uint32_t)(warp * 32)) << 16), d);
+            tmem_ld32(tbase + T::T_A + lane_off, d);
         }
 #pragma unroll
         for (int h = 0; h < HP; ++h)
@@ -716,7 +820,7 @@ __global__ void __launch_bounds__(128) pba_pair_bias_bwd_tc_kernel(const __grid_
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tbase, 32);
+        tmem_dealloc(tbase, 256);
     }
 }
 
