@@ -10,14 +10,16 @@
 //   dP  = dOa V^T      dS = P (dP - D)
 //   dV  = P^T dOa      dK = scale dS^T Q      dQ = scale dS K      dbias = sum_b dS
 //
-// Kernels, in launch order on one stream:
+// Kernels, in launch order (the dbias kernel runs on a second stream, beside the dq
+// conversion, once the main kernel is done):
 //   pba_bwd_pre_kernel      per query row: dOa (bf16), dg, and (lse * log2 e, D) row stats
 //   pba_bwd_main_kernel     persistent, items (b, h, 128-key tile): steps over query tiles;
 //                           dK, dV accumulate in TMEM; each step's dQ partial is added to an
 //                           fp32 accumulator in global memory
 //   pba_dbias_zero_kernel   local attention only: zeros of dbias outside the window
 //   pba_dbias_kernel        CTA = (h, dbias tile, split of b): loops over its rows b with the
-//                           bias tile resident; dS summed in registers; one fp32 partial tile
+//                           bias tile resident; dS summed in registers by three element-wise
+//                           warpgroups (48, 48 and 32 keys); one fp32 partial tile
 //                           per split; the tile's last CTA to finish sums the partials in
 //                           split order (bit-stable dbias)
 //   pba_dq_convert_kernel   fp32 dQ accumulator -> bf16 dq (times scale)
