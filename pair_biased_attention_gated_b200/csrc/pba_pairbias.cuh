@@ -19,13 +19,16 @@
 //   dw[c,h] = gamma_c A[c,h] + beta_c G_h,  dgamma_c = sum_h w[c,h] A[c,h],
 //   dbeta_c = sum_h w[c,h] G_h.
 //
-// Work unit: a tile of 128 consecutive positions j of one row i.  Every block (128 threads,
-// thread = position in phase 1) is persistent over tiles blockIdx.x, blockIdx.x + gridDim.x,
-// ...; tiles arrive by TMA (the Cz channels as 64-channel boxes with the 128-byte swizzle,
-// so that each thread reads its own row without bank conflicts) into two buffers, the next
-// but one tile loading while the current one is processed.  HBM-bound: z is read once and
-// the bias (or dz) written once.  The backward's parameter sums are added per block in tile
-// order, then over the blocks in block order by two small kernels (bit-stable).
+// Work unit: a tile of 128 consecutive positions j of one row i.  Every block (thread =
+// position where a thread owns a row) is persistent over tiles blockIdx.x, blockIdx.x +
+// gridDim.x, ...; tiles arrive by TMA (the Cz channels as 64-channel boxes with the 128-byte
+// swizzle, so that each thread reads its own row without bank conflicts, and the layout the
+// tensor core reads) into two buffers, the next but one tile loading while the current one is
+// processed.  HBM-bound: z is read once and the bias (or dz) written once.  The forward, and
+// the backward at Cz = 128, run their contractions on the tensor core (tcgen05, TMEM
+// accumulators); the backward at the other widths on the CUDA cores.  The backward's
+// parameter sums are added per block in tile order, then over the blocks in block order by
+// two small kernels (bit-stable).
 #pragma once
 
 #include "pba_device.cuh"
