@@ -489,26 +489,53 @@ __global__ void __launch_bounds__(256) pba_pwa_dbias_kernel(const PwaArgs a) {
     const long long nrows = (long long)a.H * a.N;
     const long long plane = (long long)a.H * a.NPad * a.NPad;
     const long long wstride = (long long)gridDim.x * (blockDim.x >> 5);
+    constexpr int U = 8;   // keys per lane per round: their loads are all issued before any is used
     for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < nrows; r += wstride) {
         const int h = (int)(r / a.N), i = (int)(r % a.N);
         const float lse = a.lse[r];
         const __nv_bfloat16 *brow = a.has_bias ? a.bias + h * a.sb0 + (long long)i * a.sb1 : nullptr;
         const float *prow = a.dw_part + ((long long)h * a.NPad + i) * a.NPad;
-        auto wgt = [&](int j) -> float {   // w in fp32, recomputed from bias and lse_w
-            if (lse == -INFINITY || (a.mask && !a.mask[j])) return 0.f;
-            return __expf((brow ? __bfloat162float(brow[j]) : 0.f) - lse);
+        // keys j0 + 32 u + lane, u < U: w in fp32 (recomputed from bias and lse_w) and dW (the
+        // split partials summed in split order)
+        auto round = [&](int j0, float (&wv)[U], float (&dv)[U]) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + 32 * u + lane;
+                const bool in = j < a.N;
+                const float b = (in && brow) ? __bfloat162float(brow[j]) : 0.f;
+                const bool keep = in && lse != -INFINITY && !(a.mask && !a.mask[j]);
+                wv[u] = keep ? __expf(b - lse) : 0.f;
+                dv[u] = 0.f;
+            }
+            for (int q = 0; q < a.splits; ++q) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int j = j0 + 32 * u + lane;
+                    if (j < a.N) dv[u] += prow[q * plane + j];
+                }
+            }
         };
-        auto dw = [&](int j) -> float {    // sum of the split partials in split order
-            float s = 0.f;
-            for (int q = 0; q < a.splits; ++q) s += prow[q * plane + j];
-            return s;
-        };
+        // r = sum_j w dW: each lane over its keys in increasing order, then a fixed butterfly
         float rs = 0.f;
-        for (int j = lane; j < a.N; j += 32) rs += wgt(j) * dw(j);
+        for (int j0 = 0; j0 < a.N; j0 += 32 * U) {
+            float wv[U], dv[U];
+            round(j0, wv, dv);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (j0 + 32 * u + lane < a.N) rs += wv[u] * dv[u];
+        }
 #pragma unroll
         for (int x = 16; x > 0; x >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, x);
         float *drow = a.dbias + r * a.N;
-        for (int j = lane; j < a.N; j += 32) drow[j] = wgt(j) * (dw(j) - rs);
+        for (int j0 = 0; j0 < a.N; j0 += 32 * U) {
+            float wv[U], dv[U];
+            round(j0, wv, dv);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + 32 * u + lane;
+                if (j < a.N) drow[j] = wv[u] * (dv[u] - rs);
+            }
+        }
     }
 }
 
